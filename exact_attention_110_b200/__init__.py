@@ -1,0 +1,179 @@
+"""Exact softmax attention on NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libfa.so`` (declared in ``include/fa.h``). Every
+step of the computation runs in the library's CUDA kernels; this module only checks and
+marshals torch tensors (device memory and the current stream) into pointers and sizes. If
+the library is missing, every call raises -- there is no fallback implementation.
+
+    o, lse = forward(q, k, v, causal=False, block_mask=None, scale=None)
+    dq, dk, dv = backward(q, k, v, o, do, lse, causal=False, block_mask=None, scale=None)
+
+q, k, v, o, do: bf16 CUDA tensors [B, H, N, d], contiguous, d in {64, 128}, N % 128 == 0.
+lse: fp32 [B, H, N]. block_mask: uint8 CUDA tensor [ceil(N/128), ceil(N/128)] or None.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from pathlib import Path
+
+import torch
+
+__all__ = [
+    "FAError", "forward", "backward", "bwd_workspace_bytes", "bwd_preprocess", "bwd_main",
+    "bwd_dq_finish", "last_device_status", "library", "LIB_PATH",
+]
+
+LIB_PATH = Path(__file__).resolve().with_name("libfa.so")
+
+FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = library().fa_status_string(status).decode()
+        super().__init__(f"{what}: {msg} (status {status})")
+
+
+def library() -> ctypes.CDLL:
+    """Loads libfa.so (built in-tree by ``python -m exact_attention_110_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not LIB_PATH.exists():
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m exact_attention_110_b200.build` "
+                "(there is no fallback implementation)")
+        lib = ctypes.CDLL(str(LIB_PATH))
+        vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        lib.fa_status_string.restype = ctypes.c_char_p
+        lib.fa_status_string.argtypes = [i32]
+        lib.fa_fwd.restype = i32
+        lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, vp, vp]
+        lib.fa_bwd_workspace_bytes.restype = sz
+        lib.fa_bwd_workspace_bytes.argtypes = [i32, i32, i32, i32]
+        lib.fa_bwd.restype = i32
+        lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, vp, vp, sz, vp]
+        lib.fa_bwd_preprocess.restype = i32
+        lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, sz, vp]
+        lib.fa_bwd_main.restype = i32
+        lib.fa_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, vp, vp, sz, vp]
+        lib.fa_bwd_dq_finish.restype = i32
+        lib.fa_bwd_dq_finish.argtypes = [vp, i32, i32, i32, i32, vp, sz, vp]
+        lib.fa_last_device_status.restype = i32
+        lib.fa_last_device_status.argtypes = [vp]
+        _lib = lib
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != FA_OK:
+        raise FAError(status, what)
+
+
+def _stream(dev: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check_qkv(*ts):
+    q = ts[0]
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    for t in ts:
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError("q, k, v (o, do) must be contiguous bf16 CUDA tensors of one shape")
+        if t.device != q.device:
+            raise ValueError("all tensors must be on one device")
+    return q.shape
+
+
+def _check_mask(block_mask, N, dev):
+    if block_mask is None:
+        return None
+    nb = (N + 127) // 128
+    if (not block_mask.is_cuda or block_mask.dtype != torch.uint8 or not block_mask.is_contiguous()
+            or tuple(block_mask.shape) != (nb, nb) or block_mask.device != dev):
+        raise ValueError(f"block_mask must be a contiguous uint8 CUDA tensor of shape ({nb}, {nb})")
+    return block_mask
+
+
+def _scale(scale, d):
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def forward(q, k, v, causal: bool = False, block_mask=None, scale=None, out=None, lse=None):
+    """O = softmax(scale * Q K^T [masked]) V and the per-row log-sum-exp (natural log)."""
+    B, H, N, d = _check_qkv(q, k, v)
+    mask = _check_mask(block_mask, N, q.device)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    _check(library().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, N, d, _scale(scale, d),
+                            int(bool(causal)), _ptr(mask), _stream(q.device)), "fa_fwd")
+    return o, l
+
+
+def bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(library().fa_bwd_workspace_bytes(B, H, N, d))
+
+
+def _workspace(B, H, N, d, dev, workspace):
+    need = bwd_workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def backward(q, k, v, o, do, lse, causal: bool = False, block_mask=None, scale=None, workspace=None,
+             dq=None, dk=None, dv=None):
+    """dQ, dK, dV of sum(O * dO) by recomputation from the saved LSE."""
+    B, H, N, d = _check_qkv(q, k, v, o, do)
+    mask = _check_mask(block_mask, N, q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    ws, nbytes = _workspace(B, H, N, d, q.device, workspace)
+    _check(library().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
+                            _ptr(dv), B, H, N, d, _scale(scale, d), int(bool(causal)), _ptr(mask), _ptr(ws),
+                            nbytes, _stream(q.device)), "fa_bwd")
+    return dq, dk, dv
+
+
+def bwd_preprocess(o, do, lse, scale=None, workspace=None):
+    B, H, N, d = _check_qkv(o, do)
+    ws, nbytes = _workspace(B, H, N, d, o.device, workspace)
+    _check(library().fa_bwd_preprocess(_ptr(o), _ptr(do), _ptr(lse), B, H, N, d, _scale(scale, d), _ptr(ws),
+                                       nbytes, _stream(o.device)), "fa_bwd_preprocess")
+    return ws
+
+
+def bwd_main(q, k, v, do, workspace, causal=False, block_mask=None, scale=None, dk=None, dv=None):
+    B, H, N, d = _check_qkv(q, k, v, do)
+    mask = _check_mask(block_mask, N, q.device)
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(library().fa_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dk), _ptr(dv), B, H, N, d,
+                                 _scale(scale, d), int(bool(causal)), _ptr(mask), _ptr(workspace), nbytes,
+                                 _stream(q.device)), "fa_bwd_main")
+    return dk, dv
+
+
+def bwd_dq_finish(workspace, shape, device, dq=None):
+    B, H, N, d = shape
+    dq = torch.empty(shape, dtype=torch.bfloat16, device=device) if dq is None else dq
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(library().fa_bwd_dq_finish(_ptr(dq), B, H, N, d, _ptr(workspace), nbytes, _stream(device)),
+           "fa_bwd_dq_finish")
+    return dq
+
+
+def last_device_status(device=None) -> int:
+    """Synchronises the current stream and returns (and clears) the device status word."""
+    dev = torch.device("cuda") if device is None else device
+    return int(library().fa_last_device_status(_stream(dev)))

@@ -1,0 +1,218 @@
+// Host side of the C ABI declared in include/fa.h: argument validation, workspace layout,
+// TMA tensor-map encoding and kernel launches. No device memory is allocated here.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace {
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per bounded device wait
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// [BH][N][D] bf16 viewed as a 3-D tensor {D, N, BH}; box 64 x 128 x 1, 128-byte swizzle.
+bool encode_bhnd(CUtensorMap* map, const void* base, long long BH, int N, int D) {
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_common(int B, int H, int N, int d, float scale) {
+  if (B <= 0 || H <= 0 || N <= 0 || !isfinite(scale)) return FA_ERR_INVALID;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (N % 128 != 0) return FA_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH > 65535) return FA_ERR_UNSUPPORTED;               // grid.y limit
+  if ((long long)N * d > (1ll << 31) / 2) return FA_ERR_UNSUPPORTED;  // per-head elements
+  return FA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Workspace {
+  float* delta;
+  float* lse2;
+  float* dq_acc;
+  size_t bytes;
+};
+
+Workspace layout(void* base, int B, int H, int N, int d) {
+  const size_t BH = (size_t)B * H, Np = ((size_t)N + 127) / 128 * 128;
+  Workspace w;
+  const size_t s_vec = align256(BH * Np * sizeof(float));
+  const size_t s_acc = align256(BH * Np * d * sizeof(float));
+  char* p = static_cast<char*>(base);
+  w.delta = reinterpret_cast<float*>(p);
+  w.lse2 = reinterpret_cast<float*>(p + s_vec);
+  w.dq_acc = reinterpret_cast<float*>(p + 2 * s_vec);
+  w.bytes = 2 * s_vec + s_acc;
+  return w;
+}
+
+fa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID: return "FA_ERR_INVALID: invalid argument";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: valid but unsupported problem size";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call or kernel launch failed";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a device-side wait gave up";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace missing or too small";
+  }
+  return "unknown fa_status";
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, const uint8_t* block_mask, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID;
+  fa_status st = check_common(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!get_encoder()) return FA_ERR_CUDA;
+  const long long BH = (long long)B * H;
+  alignas(64) CUtensorMap tq, tk, tv, to;
+  if (!encode_bhnd(&tq, q, BH, N, d) || !encode_bhnd(&tk, k, BH, N, d) || !encode_bhnd(&tv, v, BH, N, d) ||
+      !encode_bhnd(&to, o, BH, N, d))
+    return FA_ERR_CUDA;
+  fa::FwdParams p;
+  p.lse = lse;
+  p.block_mask = block_mask;
+  p.N = N;
+  p.nb = N / 128;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = kWaitLimitNs;
+  return from_cuda(fa::launch_fwd(d, tq, tk, tv, to, p, (int)BH, static_cast<cudaStream_t>(stream)));
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (check_common(B, H, N, d, 1.0f) != FA_OK) return 0;
+  return layout(nullptr, B, H, N, d).bytes;
+}
+
+fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int N, int d,
+                            float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!o || !dO || !lse) return FA_ERR_INVALID;
+  if (!aligned16(o) || !aligned16(dO) || !aligned16(lse)) return FA_ERR_INVALID;
+  fa_status st = check_common(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!workspace || !aligned16(workspace)) return FA_ERR_WORKSPACE;
+  Workspace w = layout(workspace, B, H, N, d);
+  if (workspace_bytes < w.bytes) return FA_ERR_WORKSPACE;
+  fa::BwdPreParams p;
+  p.o = static_cast<const uint16_t*>(o);
+  p.dout = static_cast<const uint16_t*>(dO);
+  p.lse = lse;
+  p.delta = w.delta;
+  p.lse2 = w.lse2;
+  p.dq_acc = w.dq_acc;
+  p.rows = (long long)B * H * N;
+  p.N = N;
+  p.Np = (N + 127) / 128 * 128;
+  p.D = d;
+  return from_cuda(fa::launch_bwd_pre(p, static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B,
+                      int H, int N, int d, float scale, int causal, const uint8_t* block_mask, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !dO || !dk || !dv) return FA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_INVALID;
+  fa_status st = check_common(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!workspace || !aligned16(workspace)) return FA_ERR_WORKSPACE;
+  Workspace w = layout(workspace, B, H, N, d);
+  if (workspace_bytes < w.bytes) return FA_ERR_WORKSPACE;
+  if (!get_encoder()) return FA_ERR_CUDA;
+  const long long BH = (long long)B * H;
+  alignas(64) CUtensorMap tq, tk, tv, tdo, tdk, tdv;
+  if (!encode_bhnd(&tq, q, BH, N, d) || !encode_bhnd(&tk, k, BH, N, d) || !encode_bhnd(&tv, v, BH, N, d) ||
+      !encode_bhnd(&tdo, dO, BH, N, d) || !encode_bhnd(&tdk, dk, BH, N, d) || !encode_bhnd(&tdv, dv, BH, N, d))
+    return FA_ERR_CUDA;
+  fa::BwdParams p;
+  p.delta = w.delta;
+  p.lse2 = w.lse2;
+  p.dq_acc = w.dq_acc;
+  p.block_mask = block_mask;
+  p.N = N;
+  p.Np = (N + 127) / 128 * 128;
+  p.nb = N / 128;
+  p.causal = causal ? 1 : 0;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = kWaitLimitNs;
+  return from_cuda(fa::launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, p, (int)BH, static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_bwd_dq_finish(void* dq, int B, int H, int N, int d, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (!dq || !aligned16(dq)) return FA_ERR_INVALID;
+  fa_status st = check_common(B, H, N, d, 1.0f);
+  if (st != FA_OK) return st;
+  if (!workspace || !aligned16(workspace)) return FA_ERR_WORKSPACE;
+  Workspace w = layout(workspace, B, H, N, d);
+  if (workspace_bytes < w.bytes) return FA_ERR_WORKSPACE;
+  fa::DqFinishParams p;
+  p.dq_acc = w.dq_acc;
+  p.dq = static_cast<uint16_t*>(dq);
+  p.rows = (long long)B * H * N;
+  p.N = N;
+  p.Np = (N + 127) / 128 * 128;
+  p.D = d;
+  p.scale = 1.0f;  // the scale is applied to dQ inside fa_bwd_main before accumulation
+  return from_cuda(fa::launch_dq_finish(p, static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                 const uint8_t* block_mask, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID;
+  fa_status st = fa_bwd_preprocess(o, dO, lse, B, H, N, d, scale, workspace, workspace_bytes, stream);
+  if (st != FA_OK) return st;
+  st = fa_bwd_main(q, k, v, dO, dk, dv, B, H, N, d, scale, causal, block_mask, workspace, workspace_bytes, stream);
+  if (st != FA_OK) return st;
+  return fa_bwd_dq_finish(dq, B, H, N, d, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_last_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return FA_ERR_CUDA;
+  int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, fa::g_fa_device_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemcpyToSymbol(fa::g_fa_device_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+}  // extern "C"

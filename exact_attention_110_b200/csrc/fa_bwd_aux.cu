@@ -1,0 +1,107 @@
+// Memory-bound helper kernels of the backward pass.
+//
+//  * bwd_pre: D_i = sum_t dO_it * O_it for every query row (the row sums the softmax
+//    Jacobian produces: sum_j P_ij dP_ij = dO_i . O_i; FlashAttention V1 lecture summary,
+//    spark.aweffr.cn, §4.1), LSE2_i = LSE_i * log2(e) for the exp2-domain recomputation of P,
+//    and a zero-fill of the fp32 dQ accumulator that fa_bwd_main adds into.
+//  * dq_finish: dq = bf16(dq_acc), the combine step after every key block has added its dQ
+//    share ("FlashAttention-2 的前世今生" overview, jishu.shishitao.com, §主要操作, backward:
+//    dQ is the one quantity shared across column blocks and is combined with atomic adds).
+//
+// Both are pure HBM streams: 16-byte vector loads/stores, grid-stride loops sized to the SM
+// count, one row handled by D/8 consecutive threads (8 bf16 = 16 bytes each).
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace fa {
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdPreParams p) {
+  constexpr int TPR = D / 8;  // threads per row
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long nthreads = (long long)gridDim.x * blockDim.x;
+  const int lane = threadIdx.x & 31, sub = lane % TPR;
+  // Rows: dot products of O and dO. A warp covers 32/TPR rows per step; the trip count is
+  // warp-uniform so the full-mask shuffles below always see all 32 lanes.
+  constexpr int RPW = 32 / TPR;
+  const long long warp_g = tid >> 5, nwarps = nthreads >> 5;
+  for (long long r0 = warp_g * RPW; r0 < p.rows; r0 += nwarps * RPW) {
+    const long long row = r0 + lane / TPR;
+    float acc = 0.f;
+    if (row < p.rows) {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(p.o + row * D) + sub);
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(p.dout + row * D) + sub);
+      acc = bf16lo(a.x) * bf16lo(b.x) + bf16hi(a.x) * bf16hi(b.x);
+      acc += bf16lo(a.y) * bf16lo(b.y) + bf16hi(a.y) * bf16hi(b.y);
+      acc += bf16lo(a.z) * bf16lo(b.z) + bf16hi(a.z) * bf16hi(b.z);
+      acc += bf16lo(a.w) * bf16lo(b.w) + bf16hi(a.w) * bf16hi(b.w);
+    }
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, TPR);
+    if (sub == 0 && row < p.rows) {
+      const long long bh = row / p.N, i = row % p.N;
+      const long long out = bh * p.Np + i;
+      p.delta[out] = acc;
+      p.lse2[out] = p.lse[row] * 1.4426950408889634f;
+    }
+  }
+  // Zero the dQ accumulator (float4 stores).
+  const long long nvec = (p.rows / p.N) * (long long)p.Np * D / 4;
+  float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);
+  for (long long e = tid; e < nvec; e += nthreads) acc4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) fa_dq_finish_kernel(const DqFinishParams p) {
+  constexpr int TPR = D / 8;
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long nthreads = (long long)gridDim.x * blockDim.x;
+  const long long total = p.rows * TPR;
+  for (long long e = tid; e < total; e += nthreads) {
+    const long long row = e / TPR;
+    const int sub = (int)(e % TPR);
+    const long long bh = row / p.N, i = row % p.N;
+    const float4* src = reinterpret_cast<const float4*>(p.dq_acc + (bh * p.Np + i) * D) + 2 * sub;
+    const float4 a = src[0], b = src[1];
+    uint4 w;
+    w.x = pack_bf16(a.x * p.scale, a.y * p.scale);
+    w.y = pack_bf16(a.z * p.scale, a.w * p.scale);
+    w.z = pack_bf16(b.x * p.scale, b.y * p.scale);
+    w.w = pack_bf16(b.z * p.scale, b.w * p.scale);
+    reinterpret_cast<uint4*>(p.dq + row * D)[sub] = w;
+  }
+}
+
+static int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream) {
+  const int grid = sm_count() * 8;  // 8 resident 256-thread blocks per SM
+  if (p.D == 64)
+    fa_bwd_pre_kernel<64><<<grid, 256, 0, stream>>>(p);
+  else
+    fa_bwd_pre_kernel<128><<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dq_finish(const DqFinishParams& p, cudaStream_t stream) {
+  const int grid = sm_count() * 8;
+  if (p.D == 64)
+    fa_dq_finish_kernel<64><<<grid, 256, 0, stream>>>(p);
+  else
+    fa_dq_finish_kernel<128><<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

@@ -1,0 +1,415 @@
+// Forward kernel: exact attention with online softmax, S and P kept in tensor memory.
+//
+// Method (sources cited by page and section):
+//   [P1] "FlashAttention-2 的前世今生" overview, jishu.shishitao.com/detail/60083.html
+//   [P2] "Attention 为什么慢" explainer, ds6.com.cn/news/67428.html
+//   [P3] FlashAttention V1 lecture summary, spark.aweffr.cn/summary/0684ec99-...
+//  * Tiling: Q, K, V are cut into 128-row blocks; each (Q block, K/V block) pair is processed
+//    on chip and S = Q K^T, P = softmax(S) never reach HBM ([P3] §3.1, §3.3; [P1] §主要操作).
+//  * FA2 loop order: a thread block owns query row-blocks and loops over K/V column-blocks,
+//    no communication between thread blocks ([P1] §主要操作, forward pass).
+//  * Online softmax: running row max m, running sum l, output rescaled when m grows
+//    ([P2] §时间复杂度, the online normaliser; [P3] §3.2 recurrence, §3.4). The output is kept
+//    unnormalised and divided by l once at the end, which removes per-step non-matmul work
+//    ([P1] §主要操作: "reduce non-matmul FLOPs").
+//  * Saved statistic: LSE = m + ln l per row, the only value the backward needs ([P1]
+//    §主要操作, backward pass).
+//
+// sm_100a design (ours, not the pages'):
+//  * CTA = 256 query rows of one (b, h) as two 128-row tiles t = 0, 1 that ping-pong: the
+//    tensor core computes S for one tile while the other tile's softmax runs.
+//  * Warp 0: TMA producer. Q tiles once; K_j and V_j through separate NS-deep shared-memory
+//    rings guarded by full/empty mbarriers. No cluster multicast: neighbouring CTAs that read
+//    the same K/V tiles are served from L2.
+//  * Warp 1: allocates 512 TMEM columns and issues every tcgen05.mma from one thread:
+//    S_t = Q_t K_j^T (128x128, fp32 in TMEM), then O_t += P_t V_j with P_t read straight
+//    from TMEM (the .kind::f16 "A in tensor memory" form).
+//  * Warps 4-7 and 8-11: one softmax warpgroup per tile; thread r owns row r (TMEM lane r),
+//    so row max and row sum need no shuffles. Scores are scaled into the log2 domain
+//    (x * scale * log2 e) and exponentiated with ex2. P (bf16) is written back over S.
+//  * Lazy rescale: the reference max m_ref moves only when a row's max exceeds it by more
+//    than 8 (a factor 256 in P). Using a stale reference is exact in real arithmetic because
+//    O and l are scaled by the same exp2(-m_ref); it keeps O rescales off the common path.
+//  * Epilogue: O / l -> bf16 into the (now unused) Q tile buffer in the TMA layout, one TMA
+//    store per 64-column panel; LSE = (m_ref + log2 l) * ln 2.
+//
+// TMEM columns: S/P tile 0 [0,128), S/P tile 1 [128,256), O tile 0 [256,256+D),
+// O tile 1 [256+D, 256+2D).
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace fa {
+
+template <int D>
+struct FwdCfg {
+  static constexpr int THREADS = 384;
+  static constexpr int NS = (D == 128) ? 2 : 4;        // K ring and V ring depth
+  static constexpr int PANEL_BYTES = 128 * 128;        // 128 rows x 64 bf16 (one swizzle panel)
+  static constexpr int PANELS = D / 64;
+  static constexpr int TILE_BYTES = PANELS * PANEL_BYTES;  // 128 x D bf16
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NS * TILE_BYTES;
+  static constexpr int NBAR = 2 + 4 * NS + 2 + 2 + 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ bool fwd_tile_active(const FwdParams& p, int qb, int j) {
+  if (qb >= p.nb) return false;
+  if (p.causal && j > qb) return false;
+  if (p.block_mask != nullptr && p.block_mask[qb * p.nb + j] == 0) return false;
+  return true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const FwdParams p) {
+  using C = FwdCfg<D>;
+  constexpr int NS = C::NS;
+  extern __shared__ __align__(1024) uint8_t smem[];
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  if ((smem_u32(smem) & 1023u) != 0) {  // swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) atomicCAS(&g_fa_device_status, 0, WAIT_SMEM_ALIGN);
+    return;
+  }
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* bar_q = bars;            // [2]  Q tile t landed
+  uint64_t* bar_kf = bars + 2;       // [NS] K stage full
+  uint64_t* bar_ke = bar_kf + NS;    // [NS] K stage free
+  uint64_t* bar_vf = bar_ke + NS;    // [NS] V stage full
+  uint64_t* bar_ve = bar_vf + NS;    // [NS] V stage free
+  uint64_t* bar_s = bar_ve + NS;     // [2]  S_t ready in TMEM
+  uint64_t* bar_p = bar_s + 2;       // [2]  P_t written (and O_t rescaled)
+  uint64_t* bar_o = bar_p + 2;       // [2]  all MMAs of tile t complete
+  uint64_t* bar_done = bar_o + 2;    // [1]  every MMA of the CTA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  AbortState* ab = reinterpret_cast<AbortState*>(smem + C::OFF_MISC + 4);
+
+  const int bh = blockIdx.y;
+  const int pair = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;  // heavy first
+  const int qb0 = 2 * pair;  // 128-row tile index of tile 0
+  const int j_end = p.causal ? min(p.nb, qb0 + 2) : p.nb;
+  const uint64_t lim = p.timeout_ns;
+
+  if (warp == 0 && lane == 0) {
+    mbar_init(&bar_q[0], 1);
+    mbar_init(&bar_q[1], 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bar_kf[s], 1);
+      mbar_init(&bar_ke[s], 1);
+      mbar_init(&bar_vf[s], 1);
+      mbar_init(&bar_ve[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bar_s[t], 1);
+      mbar_init(&bar_p[t], 4);  // one arrive per softmax warp
+      mbar_init(&bar_o[t], 1);
+    }
+    mbar_init(bar_done, 1);
+    ab->flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+  const uint32_t sK = smem_u32(smem + C::OFF_K);
+  const uint32_t sV = smem_u32(smem + C::OFF_V);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmO);
+      for (int t = 0; t < 2; ++t) {
+        if (qb0 + t < p.nb) {
+          mbar_arrive_expect_tx(&bar_q[t], C::TILE_BYTES);
+          for (int pn = 0; pn < C::PANELS; ++pn)
+            tma_load_3d(smem + C::OFF_Q + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &bar_q[t], pn * 64,
+                        (qb0 + t) * 128, bh);
+        }
+      }
+      int it = 0;
+      int issued_k[NS], issued_v[NS];
+      for (int s = 0; s < NS; ++s) issued_k[s] = issued_v[s] = -1;
+      bool ok = true;
+      for (int j = 0; j < j_end && ok; ++j) {
+        if (!fwd_tile_active(p, qb0, j) && !fwd_tile_active(p, qb0 + 1, j)) continue;
+        const int s = it % NS;
+        const uint32_t ph = (it / NS) & 1;
+        ok = mbar_wait(&bar_ke[s], ph ^ 1, ab, lim, WAIT_FWD_LOAD + 1);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bar_kf[s], C::TILE_BYTES);
+        for (int pn = 0; pn < C::PANELS; ++pn)
+          tma_load_3d(smem + C::OFF_K + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmK, &bar_kf[s], pn * 64,
+                      j * 128, bh);
+        issued_k[s] = ph;
+        ok = mbar_wait(&bar_ve[s], ph ^ 1, ab, lim, WAIT_FWD_LOAD + 2);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bar_vf[s], C::TILE_BYTES);
+        for (int pn = 0; pn < C::PANELS; ++pn)
+          tma_load_3d(smem + C::OFF_V + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmV, &bar_vf[s], pn * 64,
+                      j * 128, bh);
+        issued_v[s] = ph;
+        ++it;
+      }
+      if (!ok) {
+        // Aborting: let the copies already in flight land before the CTA's memory goes away.
+        AbortState none{0};
+        for (int s = 0; s < NS; ++s) {
+          if (issued_k[s] >= 0) mbar_wait(&bar_kf[s], issued_k[s], &none, lim, WAIT_FWD_LOAD + 3);
+          if (issued_v[s] >= 0) mbar_wait(&bar_vf[s], issued_v[s], &none, lim, WAIT_FWD_LOAD + 3);
+        }
+        for (int t = 0; t < 2; ++t)
+          if (qb0 + t < p.nb) mbar_wait(&bar_q[t], 0, &none, lim, WAIT_FWD_LOAD + 4);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);  // Q, K both K-major
+      constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);    // P (TMEM), V MN-major
+      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
+      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
+      bool ok = true;
+      for (int t = 0; t < 2 && ok; ++t)
+        if (qb0 + t < p.nb) ok = mbar_wait(&bar_q[t], 0, ab, lim, WAIT_FWD_MMA + 1);
+      uint32_t p_phase[2] = {0u, 0u};
+      bool o_started[2] = {false, false};
+      bool prev_act[2] = {false, false};
+      int prev_s = -1;
+      uint32_t prev_ph = 0;
+      int it = 0;
+
+      auto issue_pv = [&](int t, int vs) {
+        const uint32_t vbase = sV + vs * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per MMA
+          const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::PANEL_BYTES, 1024);
+          umma_ts(tO[t], tS[t] + kk * 8, bdesc, IDESC_O, (o_started[t] || kk > 0) ? 1u : 0u);
+        }
+        o_started[t] = true;
+      };
+
+      for (int j = 0; j < j_end && ok; ++j) {
+        const bool act0 = fwd_tile_active(p, qb0, j), act1 = fwd_tile_active(p, qb0 + 1, j);
+        if (!act0 && !act1) continue;
+        const int s = it % NS;
+        const uint32_t ph = (it / NS) & 1;
+        ok = mbar_wait(&bar_kf[s], ph, ab, lim, WAIT_FWD_MMA + 2);
+        if (!ok) break;
+        tc_fence_after();
+        const bool act[2] = {act0, act1};
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (prev_act[t]) {  // O_t += P_t V_{previous}
+            ok = mbar_wait(&bar_vf[prev_s], prev_ph, ab, lim, WAIT_FWD_MMA + 3);
+            if (ok) ok = mbar_wait(&bar_p[t], p_phase[t], ab, lim, WAIT_FWD_MMA + 4);
+            if (!ok) break;
+            p_phase[t] ^= 1u;
+            tc_fence_after();
+            issue_pv(t, prev_s);
+          }
+          if (act[t]) {  // S_t = Q_t K_j^T
+            const uint32_t qbase = sQ + t * C::TILE_BYTES, kbase = sK + s * C::TILE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32;
+              umma_ss(tS[t], sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024), IDESC_S,
+                      kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&bar_s[t]);
+          }
+        }
+        if (!ok) break;
+        umma_commit(&bar_ke[s]);
+        if (prev_s >= 0) umma_commit(&bar_ve[prev_s]);
+        prev_s = s;
+        prev_ph = ph;
+        prev_act[0] = act0;
+        prev_act[1] = act1;
+        ++it;
+      }
+      for (int t = 0; t < 2 && ok; ++t) {  // last PV of each tile
+        if (prev_act[t]) {
+          ok = mbar_wait(&bar_vf[prev_s], prev_ph, ab, lim, WAIT_FWD_MMA + 5);
+          if (ok) ok = mbar_wait(&bar_p[t], p_phase[t], ab, lim, WAIT_FWD_MMA + 6);
+          if (!ok) break;
+          p_phase[t] ^= 1u;
+          tc_fence_after();
+          issue_pv(t, prev_s);
+        }
+      }
+      if (ok && prev_s >= 0) umma_commit(&bar_ve[prev_s]);
+      umma_commit(&bar_o[0]);
+      umma_commit(&bar_o[1]);
+      umma_commit(bar_done);
+      AbortState none{0};
+      mbar_wait(bar_done, 0, &none, lim, WAIT_FWD_MMA + 7);  // all MMAs retired before TMEM is freed
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int t = (warp - 4) >> 2;
+    const uint32_t wq = warp & 3;      // TMEM lane quarter this warp may touch
+    const int r = wq * 32 + lane;      // row inside the tile
+    const int qb = qb0 + t;
+    const bool tvalid = qb < p.nb;
+    const uint32_t lane_off = (wq * 32u) << 16;
+    const uint32_t tS_row = tmem + lane_off + t * 128u;
+    const uint32_t tO_row = tmem + lane_off + 256u + t * D;
+    const float sl2 = p.scale_log2;
+    float m_ref = -INFINITY;  // reference max, log2 domain, scale folded in
+    float l = 0.f;            // running sum of exp2(x - m_ref)
+    uint32_t s_phase = 0;
+    bool o_started = false;
+    bool ok = true;
+
+    if (tvalid) {
+      for (int j = 0; j < j_end; ++j) {
+        if (!fwd_tile_active(p, qb, j)) continue;
+        ok = warp_wait(&bar_s[t], s_phase, ab, lim, WAIT_FWD_SOFTMAX + 1);
+        if (!ok) break;
+        s_phase ^= 1u;
+        tc_fence_after();
+
+        float sv[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t u[32];
+          tmem_ld32(tS_row + c * 32, u);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(u[i]);
+        }
+        if (p.causal && j == qb) {  // diagonal tile: key 128j+c is visible to row 128qb+r iff c <= r
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > r) sv[c] = -INFINITY;
+        }
+        float mx = sv[0];
+#pragma unroll
+        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, sv[c]);
+        const float cand = mx * sl2;
+        float alpha = 1.f;
+        if (cand > m_ref + 8.f) {  // also taken on the first visible tile (m_ref = -inf)
+          alpha = ex2(m_ref - cand);
+          m_ref = cand;
+        }
+        if (o_started && __any_sync(0xffffffffu, alpha != 1.f)) {
+          // O_t already holds every earlier PV (S_t's commit retired them): rescale in place.
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t u[32];
+            tmem_ld32(tO_row + c * 32, u);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+            tmem_st32(tO_row + c * 32, u);
+          }
+        }
+        l *= alpha;
+        const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
+        uint32_t pk[64];
+        float lsum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float p0 = ex2(fmaf(sv[2 * i], sl2, mneg));
+          const float p1 = ex2(fmaf(sv[2 * i + 1], sl2, mneg));
+          lsum += p0 + p1;
+          pk[i] = pack_bf16(p0, p1);
+        }
+        l += lsum;
+        {
+          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(&pk[0]);
+          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t (*)[32]>(&pk[32]);
+          tmem_st32(tS_row, lo);
+          tmem_st32(tS_row + 32, hi);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_p[t]);
+        o_started = true;
+      }
+
+      // ---------------------------------------------------------------- epilogue
+      if (ok) ok = warp_wait(&bar_o[t], 0, ab, lim, WAIT_FWD_EPILOGUE + 1);
+      uint8_t* stage = smem + C::OFF_Q + t * C::TILE_BYTES;  // Q_t is no longer read
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const uint32_t sstage = smem_u32(stage);
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t u[32];
+          if (o_started) {
+            tmem_ld32(tO_row + c * 32, u);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = 0u;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
+          const int col0 = c * 32;                   // first column of this chunk
+          const uint32_t panel = sstage + (col0 >> 6) * C::PANEL_BYTES;
+          const uint32_t chunk0 = (col0 & 63) >> 3;  // 16-byte chunk inside the 128-byte row
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            st_shared_v4(panel + sw128_offset(r, chunk0 + q), w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        }
+        fence_proxy_async_smem();
+        const int row = qb * 128 + r;
+        p.lse[(size_t)bh * p.N + row] = (l > 0.f) ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      }
+      // Every thread of the warpgroup reaches this barrier (tvalid is uniform per warpgroup).
+      named_bar_sync(1 + t, 128);
+      if (wq == 0 && lane == 0 && *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
+        for (int pn = 0; pn < C::PANELS; ++pn) tma_store_3d(&tmO, stage + pn * C::PANEL_BYTES, pn * 64, qb * 128, bh);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D>
+static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  dim3 grid((p.nb + 1) / 2, BH);
+  fa_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream) {
+  if (D == 64) return launch_fwd_t<64>(tq, tk, tv, to, p, BH, stream);
+  return launch_fwd_t<128>(tq, tk, tv, to, p, BH, stream);
+}
+
+}  // namespace fa

@@ -1,0 +1,76 @@
+// Kernel parameter blocks and launchers shared by the host API (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+// Where a device-side bounded wait gave up (stored in the device status word).
+enum WaitSite : int {
+  WAIT_NONE = 0,
+  WAIT_SMEM_ALIGN = 1,
+  WAIT_FWD_LOAD = 0x100,
+  WAIT_FWD_MMA = 0x200,
+  WAIT_FWD_SOFTMAX = 0x300,
+  WAIT_FWD_EPILOGUE = 0x400,
+  WAIT_BWD_LOAD = 0x1100,
+  WAIT_BWD_MMA = 0x1200,
+  WAIT_BWD_COMPUTE = 0x1300,
+  WAIT_BWD_DQ = 0x1400,
+  WAIT_BWD_EPILOGUE = 0x1500,
+  WAIT_SELFTEST = 0x7700,
+};
+
+struct FwdParams {
+  float* lse;                  // [BH][N]
+  const uint8_t* block_mask;   // [nb][nb] or null
+  int N;                       // keys = queries per head (multiple of 128)
+  int nb;                      // N / 128
+  int causal;
+  float scale_log2;            // scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+struct BwdPreParams {
+  const uint16_t* o;     // bf16 [BH][N][D]
+  const uint16_t* dout;  // bf16 [BH][N][D]
+  const float* lse;      // [BH][N]
+  float* delta;          // [BH][Np]
+  float* lse2;           // [BH][Np]  = LSE * log2(e)
+  float* dq_acc;         // [BH][Np][D], zeroed here
+  long long rows;        // BH * N
+  int N, Np, D;
+};
+
+struct BwdParams {
+  const float* delta;    // [BH][Np]
+  const float* lse2;     // [BH][Np]
+  float* dq_acc;         // [BH][Np][D]
+  const uint8_t* block_mask;
+  int N, Np, nb;
+  int causal;
+  float scale;           // scale (for dK)
+  float scale_log2;      // scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+struct DqFinishParams {
+  const float* dq_acc;   // [BH][Np][D]
+  uint16_t* dq;          // bf16 [BH][N][D]
+  long long rows;        // BH * N
+  int N, Np, D;
+  float scale;
+};
+
+// Launchers (return the launch error, if any).
+cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream);
+cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream);
+cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
+                            const BwdParams& p, int BH, cudaStream_t stream);
+cudaError_t launch_dq_finish(const DqFinishParams& p, cudaStream_t stream);
+
+}  // namespace fa

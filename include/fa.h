@@ -1,0 +1,121 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact softmax attention on NVIDIA B200 (sm_100a).
+ *
+ * The library computes O = softmax(scale * Q K^T) V with the N x N score and probability
+ * matrices never written to memory (tiling + online softmax), saves one log-sum-exp per
+ * query row, and computes dQ, dK, dV by recomputing the probabilities from that
+ * statistic.
+ *
+ * Sources (cited by page and section):
+ *   [P1] "FlashAttention-2 的前世今生" overview, jishu.shishitao.com/detail/60083.html
+ *   [P2] "Attention 为什么慢" / Flash Attention explainer, ds6.com.cn/news/67428.html
+ *   [P3] FlashAttention V1 lecture summary, spark.aweffr.cn/summary/0684ec99-...
+ *
+ * Conventions shared by every call:
+ *  - Tensors q, k, v, o, dO, dq, dk, dv are bf16, contiguous [B][H][N][d], d fastest.
+ *    The problem statement of [P3] §2.1/§2.2 (Q, K, V of N x d per head), batched over B
+ *    and H as in [P1] §主要操作 ("parallelise over batch and heads").
+ *  - lse is fp32 [B][H][N]: LSE_i = ln sum_j exp(scale * q_i . k_j) over the allowed keys,
+ *    natural log, scale included -- the single per-row statistic FA2 keeps for the
+ *    backward ([P1] §主要操作, backward pass). A row with no allowed key gets -inf and O=0.
+ *  - causal != 0 allows key j for query i only if j <= i (top-left aligned; [P1] benchmark
+ *    setting "with or without causal mask").
+ *  - block_mask (nullable) is a device array of ceil(N/128) x ceil(N/128) uint8, row-major,
+ *    shared by all (b, h); block (I, J) != 0 lets queries 128I..128I+127 see keys
+ *    128J..128J+127 ([P1] §Block-Sparse FlashAttention). Tiles that are off are never
+ *    loaded or computed. causal and block_mask combine (AND).
+ *  - All pointers are device memory owned by the caller. The library allocates no device
+ *    memory apart from one static device status word.
+ *  - Every pointer must be 16-byte aligned. d must be 64 or 128. N must be a positive
+ *    multiple of 128 (other N: FA_ERR_UNSUPPORTED).
+ *  - stream is a cudaStream_t (NULL = legacy default stream). All calls are asynchronous
+ *    on it; argument errors are reported synchronously, before anything is enqueued.
+ *  - Not re-entrant on the same output buffers; distinct calls on distinct buffers may run
+ *    concurrently on different streams.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID = 1,     /* null/misaligned pointer, non-positive size, non-finite scale */
+  FA_ERR_UNSUPPORTED = 2, /* valid but not implemented: d not in {64,128}, N % 128 != 0 */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call or a kernel launch failed */
+  FA_ERR_TIMEOUT = 4,     /* a device-side bounded wait gave up (see fa_last_device_status) */
+  FA_ERR_WORKSPACE = 5    /* workspace pointer null or smaller than fa_bwd_workspace_bytes */
+} fa_status;
+
+/*
+ * Forward pass ([P3] §3.1-§3.3 tiling + online softmax; FA2 loop order of [P1] §主要操作:
+ * each thread block owns query row-blocks and loops over key/value column-blocks).
+ *   in : q, k, v       bf16 [B][H][N][d]
+ *   out: o             bf16 [B][H][N][d]
+ *        lse           fp32 [B][H][N]
+ *   scale: multiplies q.k (typically 1/sqrt(d)); must be finite.
+ * One kernel launch.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, float scale, int causal, const uint8_t* block_mask, void* stream);
+
+/*
+ * Bytes of caller-provided device workspace fa_bwd needs: fp32 D [B][H][Np], fp32 scaled
+ * LSE [B][H][Np] and the fp32 dQ accumulator [B][H][Np][d] (Np = N rounded up to 128),
+ * each 256-byte aligned. Returns 0 for sizes fa_bwd would reject.
+ */
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward pass by recomputation ([P3] §4.2; [P1] §主要操作, backward: only the LSE is
+ * kept; column-block workers; dQ combined across thread blocks).
+ *   in : q, k, v, o, dO  bf16 [B][H][N][d];  lse fp32 [B][H][N] from fa_fwd
+ *   out: dq, dk, dv      bf16 [B][H][N][d]
+ *   workspace: device buffer of at least fa_bwd_workspace_bytes(B,H,N,d) bytes; its
+ *              contents on entry are ignored and on exit unspecified.
+ * Equivalent to fa_bwd_preprocess + fa_bwd_main + fa_bwd_dq_finish on the same workspace.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 float scale, int causal, const uint8_t* block_mask, void* workspace,
+                 size_t workspace_bytes, void* stream);
+
+/*
+ * The three stages of fa_bwd, exposed so each kernel can be launched (and timed) alone.
+ * fa_bwd_preprocess: D_i = sum_t dO_it * O_it (the row sums of dP o P, from the softmax
+ *   Jacobian [P3] §4.1), the scaled LSE, and zeroes the fp32 dQ accumulator. HBM-bound.
+ * fa_bwd_main: per key tile, recompute S and P, accumulate dK and dV on chip, write dk and
+ *   dv (bf16), and add each tile's dQ contribution into the fp32 accumulator.
+ * fa_bwd_dq_finish: dq = bf16(accumulator).
+ * They must be called in this order on one stream with the same workspace and sizes.
+ */
+fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int N,
+                            int d, float scale, void* workspace, size_t workspace_bytes,
+                            void* stream);
+fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk,
+                      void* dv, int B, int H, int N, int d, float scale, int causal,
+                      const uint8_t* block_mask, void* workspace, size_t workspace_bytes,
+                      void* stream);
+fa_status fa_bwd_dq_finish(void* dq, int B, int H, int N, int d, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reports and clears the device status word: FA_ERR_TIMEOUT if
+ * any kernel since the last call gave up on a bounded wait (its outputs are then invalid),
+ * FA_ERR_CUDA if the stream reports an error, FA_OK otherwise.
+ */
+fa_status fa_last_device_status(void* stream);
+
+/* Static, human-readable name of a status code. Never NULL. */
+const char* fa_status_string(fa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

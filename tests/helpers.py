@@ -1,0 +1,57 @@
+"""Shared helpers for the parity tests: seeded inputs as torch bf16 + fp64 numpy, and the
+parity bars (absolute/mean error on O, absolute on LSE, relative Frobenius on gradients)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import synth
+
+# Parity bars for bf16 inputs drawn from N(0, 1).
+O_MAX_ABS = 1e-2
+O_MEAN_ABS = 1e-3
+LSE_MAX_ABS = 1e-3
+GRAD_REL_FRO = 2e-2
+
+
+def bits_to_torch(bits: np.ndarray, device) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.to(device)
+
+
+def bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return synth.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def make_case(B, H, N, d, seed=synth.BASE_SEED, device="cuda", with_do=True):
+    bits = synth.attention_inputs(B, H, N, d, seed, with_do=with_do)
+    gpu = {k: bits_to_torch(v, device) for k, v in bits.items()}
+    f64 = {k: bits_to_f64(v) for k, v in bits.items()}
+    return gpu, f64
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def assert_fwd_close(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
+    err = np.abs(o_gpu - o_ref)
+    assert err.max() <= O_MAX_ABS, f"{what} O max|err| {err.max():.3e}"
+    assert err.mean() <= O_MEAN_ABS, f"{what} O mean|err| {err.mean():.3e}"
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(lse_gpu), fin), f"{what} LSE finiteness differs"
+    if fin.any():
+        lerr = np.abs(lse_gpu[fin] - lse_ref[fin]).max()
+        assert lerr <= LSE_MAX_ABS, f"{what} LSE max|err| {lerr:.3e}"
+
+
+def rel_fro(a, b):
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
+
+
+def assert_grads_close(gpu, ref, what=""):
+    for name, a, b in zip(("dQ", "dK", "dV"), gpu, ref):
+        assert np.all(np.isfinite(a)), f"{what} {name} has non-finite values"
+        e = rel_fro(a, b)
+        assert e <= GRAD_REL_FRO, f"{what} {name} relative Frobenius error {e:.3e}"

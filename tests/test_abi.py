@@ -1,0 +1,86 @@
+"""The C-ABI library loads without a GPU, exports every entry point include/fa.h declares,
+and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import math
+import re
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parent.parent
+HEADER = ROOT / "include" / "fa.h"
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_attention_110_b200 import build
+    build.build()
+    import exact_attention_110_b200 as fa
+    return fa.library()
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert {"fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_last_device_status", "fa_status_string"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"libfa.so does not export {n}"
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.fa_status_string(s).decode().startswith("FA_")
+    assert lib.fa_status_string(99) == b"unknown fa_status"
+
+
+FAKE = 0x10000  # 16-byte-aligned fake device address: argument checks must reject before use
+
+
+def fwd(lib, q=FAKE, B=1, H=1, N=128, d=64, scale=0.125, lse=FAKE):
+    return lib.fa_fwd(q, FAKE, FAKE, FAKE, lse, B, H, N, d, scale, 0, None, None)
+
+
+def test_fwd_argument_checks(lib):
+    assert fwd(lib, q=None) == 1                 # null pointer -> INVALID
+    assert fwd(lib, q=FAKE + 2) == 1             # misaligned -> INVALID
+    assert fwd(lib, lse=FAKE + 4) == 1
+    assert fwd(lib, B=0) == 1 and fwd(lib, H=-1) == 1 and fwd(lib, N=0) == 1
+    assert fwd(lib, scale=math.nan) == 1 and fwd(lib, scale=math.inf) == 1
+    assert fwd(lib, d=96) == 2                   # unsupported head dim
+    assert fwd(lib, d=256) == 2
+    assert fwd(lib, N=100) == 2                  # N not a multiple of 128
+
+
+def test_workspace_size_and_checks(lib):
+    # D, scaled LSE (fp32 each) and the fp32 dQ accumulator, each 256-byte aligned.
+    B, H, N, d = 2, 3, 256, 64
+    vec = (B * H * N * 4 + 255) // 256 * 256
+    acc = (B * H * N * d * 4 + 255) // 256 * 256
+    assert lib.fa_bwd_workspace_bytes(B, H, N, d) == 2 * vec + acc
+    assert lib.fa_bwd_workspace_bytes(1, 1, 100, 64) == 0
+    assert lib.fa_bwd_workspace_bytes(1, 1, 128, 80) == 0
+    need = lib.fa_bwd_workspace_bytes(1, 1, 128, 64)
+    st = lib.fa_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0, None,
+                    FAKE, need - 1, None)
+    assert st == 5                               # workspace too small
+    st = lib.fa_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0, None,
+                    None, need, None)
+    assert st == 5                               # workspace missing
+    st = lib.fa_bwd(FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0, None,
+                    FAKE, need, None)
+    assert st == 1
+    assert lib.fa_bwd_dq_finish(FAKE + 8, 1, 1, 128, 64, FAKE, need, None) == 1
+    assert lib.fa_bwd_main(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 48, 0.1, 0, None, FAKE, need, None) == 2
+
+
+def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import exact_attention_110_b200 as fa
+    monkeypatch.setattr(fa, "LIB_PATH", tmp_path / "missing.so")
+    monkeypatch.setattr(fa, "_lib", None)
+    with pytest.raises(RuntimeError, match="no fallback"):
+        fa.library()

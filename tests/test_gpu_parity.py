@@ -1,0 +1,169 @@
+"""GPU parity: the CUDA kernels (through the C ABI) against the fp64 oracle on the same
+seeded bf16 inputs, element by element, with the bars in tests/helpers.py."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fa():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    import exact_attention_110_b200 as fa
+    fa.library()
+    return fa
+
+
+def run_fwd(fa, gpu, causal, mask_t, scale):
+    o, lse = fa.forward(gpu["q"], gpu["k"], gpu["v"], causal=causal, block_mask=mask_t, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.last_device_status() == 0
+    return o, lse
+
+
+def run_bwd(fa, gpu, o, lse, causal, mask_t, scale):
+    dq, dk, dv = fa.backward(gpu["q"], gpu["k"], gpu["v"], o, gpu["do"], lse, causal=causal,
+                             block_mask=mask_t, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.last_device_status() == 0
+    return dq, dk, dv
+
+
+def mask_for(kind, N, seed=synth.BASE_SEED):
+    nb = N // 128
+    if kind is None:
+        return None
+    if kind == "bernoulli":
+        return synth.block_mask_for(N, seed)
+    if kind == "ones":
+        return np.ones((nb, nb), np.uint8)
+    if kind == "diag":
+        return np.eye(nb, dtype=np.uint8)
+    raise ValueError(kind)
+
+
+SMALL = [
+    # B, H, N, d, causal, mask
+    (1, 1, 128, 64, False, None),      # tiny config: one tile
+    (1, 2, 384, 64, False, None),      # odd number of 128-row tiles (last CTA has one tile)
+    (1, 2, 384, 128, False, None),
+    (2, 1, 640, 64, True, None),
+    (1, 2, 512, 128, True, None),
+    (1, 2, 512, 64, False, "bernoulli"),
+    (1, 1, 768, 128, True, "bernoulli"),
+    (1, 1, 512, 64, False, "diag"),
+]
+
+
+@pytest.mark.parametrize("B,Hh,N,d,causal,mask", SMALL)
+def test_fwd_bwd_small(fa, oracle_mod, B, Hh, N, d, causal, mask):
+    gpu, ref = H.make_case(B, Hh, N, d, seed=synth.BASE_SEED + N + d)
+    scale = 1.0 / np.sqrt(d)
+    m = mask_for(mask, N)
+    mt = None if m is None else torch.from_numpy(m).cuda()
+    o, lse = run_fwd(fa, gpu, causal, mt, scale)
+    o_ref, lse_ref = oracle_mod.attention_fwd(ref["q"], ref["k"], ref["v"], scale, causal=causal, mask=m)
+    H.assert_fwd_close(H.to_f64(o), H.to_f64(lse), o_ref, lse_ref, f"fwd {B,Hh,N,d,causal,mask}")
+    dq, dk, dv = run_bwd(fa, gpu, o, lse, causal, mt, scale)
+    g_ref = oracle_mod.attention_bwd(ref["q"], ref["k"], ref["v"], ref["do"], scale, causal=causal, mask=m)[:3]
+    H.assert_grads_close([H.to_f64(x) for x in (dq, dk, dv)], g_ref, f"bwd {B,Hh,N,d,causal,mask}")
+
+
+def sampled_heads(B, Hh, n, seed):
+    rng = np.random.default_rng(seed)
+    flat = rng.choice(B * Hh, size=min(n, B * Hh), replace=False)
+    return [(int(f // Hh), int(f % Hh)) for f in sorted(flat)]
+
+
+def check_heads(fa, oracle_mod, B, Hh, N, d, causal, mask, nheads, seed):
+    gpu, ref = H.make_case(B, Hh, N, d, seed=seed)
+    scale = 1.0 / np.sqrt(d)
+    mt = None if mask is None else torch.from_numpy(mask).cuda()
+    o, lse = run_fwd(fa, gpu, causal, mt, scale)
+    dq, dk, dv = run_bwd(fa, gpu, o, lse, causal, mt, scale)
+    outs = [H.to_f64(x) for x in (o, lse, dq, dk, dv)]
+    for (b, h) in sampled_heads(B, Hh, nheads, seed):
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        args = [ref[k][sl] for k in ("q", "k", "v")]
+        o_ref, lse_ref = oracle_mod.attention_fwd(*args, scale, causal=causal, mask=mask)
+        H.assert_fwd_close(outs[0][sl], outs[1][sl], o_ref, lse_ref, f"head {b},{h}")
+        g_ref = oracle_mod.attention_bwd(*args, ref["do"][sl], scale, causal=causal, mask=mask)[:3]
+        H.assert_grads_close([x[sl] for x in outs[2:]], g_ref, f"head {b},{h}")
+
+
+def test_config_bert_large_shape(fa, oracle_mod):
+    # B=16, H=16, N=512, d=64, non-causal (sampled heads checked in full)
+    check_heads(fa, oracle_mod, 16, 16, 512, 64, False, None, nheads=8, seed=synth.BASE_SEED)
+
+
+def test_config_gpt2_shape_causal(fa, oracle_mod):
+    # B=8, H=12, N=1024, d=64, causal
+    check_heads(fa, oracle_mod, 8, 12, 1024, 64, True, None, nheads=4, seed=synth.BASE_SEED)
+
+
+def test_config_block_sparse(fa, oracle_mod):
+    # B=4, H=16, N=4096, d=64, 128x128 blocks: diagonal on, others Bernoulli(0.25)
+    mask = synth.block_mask_for(4096, synth.BASE_SEED)
+    check_heads(fa, oracle_mod, 4, 16, 4096, 64, False, mask, nheads=1, seed=synth.BASE_SEED)
+
+
+@pytest.mark.parametrize("N", [512, 1024, 2048, 4096, 8192, 16384])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_config_seqlen_sweep_forward_rows(fa, oracle_mod, N, d, causal):
+    # 16k tokens, hidden 2048: B = 16384 / N, H = 2048 / d. Forward checked on sampled rows of
+    # sampled heads (the oracle computes those rows one by one).
+    B, Hh = 16384 // N, 2048 // d
+    gpu, ref = H.make_case(B, Hh, N, d, seed=synth.BASE_SEED + 7, with_do=False)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = run_fwd(fa, gpu, causal, None, scale)
+    o64, l64 = H.to_f64(o), H.to_f64(lse)
+    rng = np.random.default_rng(N + d + causal)
+    for (b, h) in sampled_heads(B, Hh, 2, N + d):
+        rows = np.unique(np.concatenate([[0, 127, 128, N - 1], rng.choice(N, 60, replace=False)]))
+        o_ref, l_ref = oracle_mod.attention_fwd_rows(ref["q"][b, h], ref["k"][b, h], ref["v"][b, h], rows, scale,
+                                                     causal=causal)
+        H.assert_fwd_close(o64[b, h, rows], l64[b, h, rows], o_ref, l_ref, f"N={N} d={d} head {b},{h}")
+
+
+def test_masked_blocks_do_not_influence_output(fa):
+    # Keys/values in blocks that are off (or in the causal future) must not change O at all.
+    N, d = 512, 64
+    gpu, _ = H.make_case(1, 2, N, d, seed=11)
+    m = np.array([[1, 0, 0, 0], [1, 1, 0, 0], [0, 1, 1, 0], [1, 0, 0, 1]], np.uint8)
+    mt = torch.from_numpy(m).cuda()
+    o1, l1 = run_fwd(fa, gpu, False, mt, 0.125)
+    k2, v2 = gpu["k"].clone(), gpu["v"].clone()
+    k2[:, :, 128:256] += 3.0   # key block 1 is visible only to query blocks 1, 2
+    v2[:, :, 128:256] -= 5.0
+    gpu2 = dict(gpu, k=k2, v=v2)
+    o2, l2 = run_fwd(fa, gpu2, False, mt, 0.125)
+    assert torch.equal(o1[:, :, :128], o2[:, :, :128]) and torch.equal(o1[:, :, 384:], o2[:, :, 384:])
+    assert torch.equal(l1[:, :, :128], l2[:, :, :128])
+    # causal: perturbing the last key block changes nothing for earlier query blocks
+    o3, _ = run_fwd(fa, gpu, True, None, 0.125)
+    k4 = gpu["k"].clone()
+    k4[:, :, 384:] *= -2.0
+    o4, _ = run_fwd(fa, dict(gpu, k=k4), True, None, 0.125)
+    assert torch.equal(o3[:, :, :384], o4[:, :, :384])
+
+
+def test_fully_masked_query_block(fa, oracle_mod):
+    # Query block 0 sees no key block: O = 0, LSE = -inf, and its dQ is exactly zero.
+    N, d = 384, 64
+    gpu, ref = H.make_case(1, 1, N, d, seed=12)
+    m = np.array([[0, 0, 0], [1, 1, 0], [0, 1, 1]], np.uint8)
+    mt = torch.from_numpy(m).cuda()
+    o, lse = run_fwd(fa, gpu, False, mt, 0.125)
+    assert torch.all(o[:, :, :128] == 0) and torch.all(torch.isneginf(lse[:, :, :128]))
+    o_ref, l_ref = oracle_mod.attention_fwd(ref["q"], ref["k"], ref["v"], 0.125, mask=m)
+    H.assert_fwd_close(H.to_f64(o), H.to_f64(lse), o_ref, l_ref, "fully masked block")
+    dq, dk, dv = run_bwd(fa, gpu, o, lse, False, mt, 0.125)
+    assert torch.all(dq[:, :, :128] == 0)
+    g_ref = oracle_mod.attention_bwd(ref["q"], ref["k"], ref["v"], ref["do"], 0.125, mask=m)[:3]
+    H.assert_grads_close([H.to_f64(x) for x in (dq, dk, dv)], g_ref, "fully masked block")
