@@ -1,0 +1,386 @@
+#!/usr/bin/env python3
+"""Benchmark: exact attention forward + backward on B200 through the fa C ABI.
+
+One step = the whole hot path on one batch: fa_fwd, then fa_bwd's three kernels
+(preprocess, main, dQ finish). Default workload: the sequence-length sweep's
+N=4096 point (16k tokens, hidden 2048 -> B=4, H=16, d=128), non-causal, bf16 N(0,1)
+inputs from the seeded generator. Prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--seqlen N] [--headdim d]
+                    [--causal] [--block-sparse] [--impl reference] [--sweep]
+
+Metric: fwd+bwd TFLOPS with FLOPs counted as 4*B*H*N^2*d for the forward (halved for causal,
+scaled by block density for block-sparse) and 2.5x that for the backward.
+--gpus N (under torchrun): every rank runs the same per-GPU workload on its own (b, h) shard
+(no data-path collective: heads are independent), value = all ranks' FLOPs / max time.
+--impl reference: the fp64 CPU oracle, timed on this host's cores on a bounded sample of
+the same workload (whole heads), reported in the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+TOKENS, HIDDEN = 16384, 2048
+METRIC = "attention fwd / fwd+bwd TFLOPS and % of B200 dense BF16 peak vs seq len"
+UNIT = "TFLOPS"
+
+
+# ----------------------------------------------------------------------------- host logic
+def workload(seqlen: int, headdim: int, causal: bool, block_sparse: bool):
+    if block_sparse:
+        return dict(B=4, H=16, N=4096, d=64, causal=False, block_sparse=True,
+                    name="block-sparse B=4 H=16 N=4096 d=64, 128x128 blocks Bernoulli(0.25), diagonal on")
+    B, H = TOKENS // seqlen, HIDDEN // headdim
+    return dict(B=B, H=H, N=seqlen, d=headdim, causal=causal, block_sparse=False,
+                name=f"seq-len sweep (16k tokens, hidden 2048): N={seqlen} d={headdim} B={B} H={H} "
+                     f"{'causal' if causal else 'non-causal'}")
+
+
+def fwd_flops(B, H, N, d, causal=False, density=1.0) -> float:
+    f = 4.0 * B * H * N * N * d * density
+    return f * 0.5 if causal else f
+
+
+def shard_heads(BH: int, world: int, rank: int):
+    """Contiguous (b, h) shard of a rank. Every head is independent, so no exchange is needed."""
+    per = (BH + world - 1) // world
+    lo = min(BH, rank * per)
+    return lo, min(BH, lo + per)
+
+
+def reduce_max(value: float, dist_on: bool, device=None) -> float:
+    """Max over ranks (timing convention: the slowest rank defines the step time)."""
+    if not dist_on:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return dict(bf16_tflops=float(d["bf16_tflops"]), bf16_tflops_sustained=float(d["bf16_tflops_sustained"]),
+                    hbm_gbs=float(d["hbm_gbs"]), source="measured")
+    return dict(bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, hbm_gbs=6650.0, source="fallback")
+
+
+def physical_gpu(local_rank: int) -> str:
+    """nvidia-smi index (or UUID) of this rank's GPU, honouring CUDA_VISIBLE_DEVICES."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.proc = None
+        self.gpu_index = gpu_index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [ln.split(", ") for ln in (self.out or "").strip().splitlines() if ln.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+def oracle_sample(wl, nheads: int, seed: int):
+    """Times the fp64 oracle (fwd + bwd) on `nheads` whole heads of the workload."""
+    import numpy as np
+    import oracle
+    import synth
+    B, H, N, d = wl["B"], wl["H"], wl["N"], wl["d"]
+    mask = synth.block_mask_for(N) if wl["block_sparse"] else None
+    n = nheads * N * d
+    q, k, v, do = (synth.bf16_bits_to_f32(synth.normal_bf16(seed + i, n)).astype(np.float64).reshape(1, nheads, N, d)
+                   for i in range(4))
+    scale = 1.0 / math.sqrt(d)
+    t0 = time.perf_counter()
+    oracle.attention_fwd(q, k, v, scale, causal=wl["causal"], mask=mask)
+    oracle.attention_bwd(q, k, v, do, scale, causal=wl["causal"], mask=mask)
+    dt = time.perf_counter() - t0
+    density = float(mask.mean()) if mask is not None else 1.0
+    flops = 3.5 * fwd_flops(1, nheads, N, d, wl["causal"], density)
+    return flops, dt, oracle.num_threads()
+
+
+def heads_for_seconds(wl, target_s: float, rate_gflops: float = 20.0) -> int:
+    per_head = 3.5 * fwd_flops(1, 1, wl["N"], wl["d"], wl["causal"], 0.27 if wl["block_sparse"] else 1.0)
+    return max(1, min(wl["B"] * wl["H"], int(target_s * rate_gflops * 1e9 / per_head)))
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return 0
+    nh = heads_for_seconds(wl, 2.0)
+    for _ in range(args.warmup):
+        oracle_sample(wl, nh, 1000)
+    tot_f, tot_t, cores = 0.0, 0.0, 1
+    for s in range(args.steps):
+        f, t, cores = oracle_sample(wl, nh, 2000 + 10 * s)
+        tot_f += f
+        tot_t += t
+    value = tot_f / tot_t / 1e12
+    sample = f"{nh} whole head(s) of {wl['N']}x{wl['d']} per step (fwd+bwd, fp64), of {wl['B'] * wl['H']} heads"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl["name"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_gpu(args, wl, rank, world, local_rank, dist_on):
+    import numpy as np
+    import torch
+    import exact_attention_110_b200 as fa
+    import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    fa.library()
+    B, H, N, d, causal = wl["B"], wl["H"], wl["N"], wl["d"], wl["causal"]
+    shape = (B, H, N, d)
+    seed = synth.BASE_SEED + 97 * rank
+    bits = synth.attention_inputs(B, H, N, d, seed)
+    q, k, v, do = (synth.to_torch_bf16(bits[x], dev) for x in ("q", "k", "v", "do"))
+    mask_np = synth.block_mask_for(N) if wl["block_sparse"] else None
+    mask = None if mask_np is None else torch.from_numpy(mask_np).to(dev)
+    density = float(mask_np.mean()) if mask_np is not None else 1.0
+    scale = 1.0 / math.sqrt(d)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws = torch.empty(fa.bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record()
+        fa.forward(q, k, v, causal=causal, block_mask=mask, scale=scale, out=o, lse=lse)
+        if evs is not None:
+            evs[1].record()
+        fa.bwd_preprocess(o, do, lse, scale=scale, workspace=ws)
+        if evs is not None:
+            evs[2].record()
+        fa.bwd_main(q, k, v, do, ws, causal=causal, block_mask=mask, scale=scale, dk=dk, dv=dv)
+        if evs is not None:
+            evs[3].record()
+        fa.bwd_dq_finish(ws, shape, dev, dq=dq)
+        if evs is not None:
+            evs[4].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if fa.last_device_status(dev) != 0:
+        raise RuntimeError("device wait timed out during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(physical_gpu(local_rank)) as clk:
+        time.sleep(0.3)  # let the sampler start
+        start.record()
+        for s in range(args.steps):
+            step(evs[s])
+        end.record()
+        torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    if fa.last_device_status(dev) != 0:
+        raise RuntimeError("device wait timed out in the timed region")
+    total_ms = reduce_max(start.elapsed_time(end), dist_on, dev)
+    k_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(4)]
+    fwd_ms, pre_ms, main_ms, fin_ms = (reduce_max(x, dist_on, dev) for x in k_ms)
+    ms = total_ms / args.steps
+    f_fwd = fwd_flops(B, H, N, d, causal, density)
+    value = world * 3.5 * f_fwd / (ms * 1e-3) / 1e12
+    peaks = load_peaks()
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+        ho, hdq, hdk, hdv = (torch.empty(shape, dtype=torch.bfloat16).pin_memory() for _ in range(4))
+        hl = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True); do.copy_(hdo, non_blocking=True)
+            fa.forward(q, k, v, causal=causal, block_mask=mask, scale=scale, out=o, lse=lse)
+            fa.backward(q, k, v, o, do, lse, causal=causal, block_mask=mask, scale=scale, workspace=ws,
+                        dq=dq, dk=dk, dv=dv)
+            ho.copy_(o, non_blocking=True); hl.copy_(lse, non_blocking=True)
+            hdq.copy_(dq, non_blocking=True); hdk.copy_(dk, non_blocking=True); hdv.copy_(dv, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist_on:
+            torch.distributed.barrier()
+        e0.record()
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = reduce_max(e0.elapsed_time(e1), dist_on, dev) / args.steps
+        nb = B * H * N * d * 2
+        e2e = {"value": world * 3.5 * f_fwd / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": 4 * nb, "d2h_bytes_per_step": 4 * nb + B * H * N * 4,
+               "ms_per_step": e2e_ms}
+
+    # ---- roofline of the dominant kernel (bwd main: 5 of the 7 matmuls of a step)
+    main_flops = 2.5 * f_fwd
+    achieved = main_flops / (main_ms * 1e-3) / 1e12
+    traffic = None
+    tfile = ROOT / "profiles" / "traffic.json"
+    if tfile.exists():
+        tj = json.loads(tfile.read_text()).get(f"bwd_main N={N} d={d} causal={int(causal)} bs={int(wl['block_sparse'])}")
+        if tj is not None:
+            traffic = tj
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": traffic, "kernel": "fa_bwd_kernel",
+                "peak_kind": f"bf16 dense burst ({peaks['source']})",
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]}
+
+    kernels = {
+        "fwd": {"ms": fwd_ms, "tflops": f_fwd / (fwd_ms * 1e-3) / 1e12},
+        "bwd_preprocess": {"ms": pre_ms, "gbs": (4 * B * H * N * d + 8 * B * H * N + 4 * B * H * N * d + 4 * B * H * N)
+                           / (pre_ms * 1e-3) / 1e9},
+        "bwd_main": {"ms": main_ms, "tflops": achieved},
+        "bwd_dq_finish": {"ms": fin_ms, "gbs": (4 * B * H * N * d + 2 * B * H * N * d) / (fin_ms * 1e-3) / 1e9},
+    }
+    bwd_ms = pre_ms + main_ms + fin_ms
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl["name"], "B": B, "H": H, "N": N, "d": d, "causal": causal,
+                   "block_density": density, "global_batch_heads": world * B * H,
+                   "l2": "no flush: the step's tensors (q,k,v,o,do,dq,dk,dv = 8 x "
+                         f"{B * H * N * d * 2 / 2**20:.0f} MiB) exceed the 126 MB L2",
+                   "parallelism": f"dp{world} over (b,h) shards, no collective"},
+        "fwd_tflops": world * f_fwd / (fwd_ms * 1e-3) / 1e12,
+        "bwd_tflops": world * 2.5 * f_fwd / (bwd_ms * 1e-3) / 1e12,
+        "pct_of_peak_fwd_bwd": 100.0 * value / world / peaks["bf16_tflops"],
+        "pct_of_peak_fwd": 100.0 * f_fwd / (fwd_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+        "kernels": kernels,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nh = heads_for_seconds(wl, 12.0)
+        f, t, cores = oracle_sample(wl, nh, 3000)
+        line["cpu_baseline"] = {"value": f / t / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"{nh} whole head(s) of {N}x{d} (fwd+bwd, fp64) of {B * H} heads; "
+                                          f"{t:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--seqlen", type=int, default=4096)
+    ap.add_argument("--headdim", type=int, default=128)
+    ap.add_argument("--causal", action="store_true")
+    ap.add_argument("--block-sparse", action="store_true")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="one JSON line per sweep point (N x d x causal)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    if args.impl == "reference":
+        wl = workload(args.seqlen, args.headdim, args.causal, args.block_sparse)
+        return run_reference(args, wl, rank, world)
+    if dist_on:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        points = ([(n, dd, c) for dd in (64, 128) for c in (False, True) for n in (512, 1024, 2048, 4096, 8192, 16384)]
+                  if args.sweep else [(args.seqlen, args.headdim, args.causal)])
+        for (n, dd, c) in points:
+            wl = workload(n, dd, c, args.block_sparse)
+            if args.sweep:
+                args.no_cpu_baseline, args.no_e2e = True, True
+            run_gpu(args, wl, rank, world, local_rank, dist_on)
+    finally:
+        if dist_on:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -113,3 +113,11 @@ def attention_inputs(B: int, H: int, N: int, d: int, base_seed: int = BASE_SEED,
 def block_mask_for(N: int, base_seed: int = BASE_SEED, p: float = 0.25, block: int = 128) -> np.ndarray:
     nb = (N + block - 1) // block
     return bernoulli_block_mask(base_seed + SEED_MASK, nb, p)
+
+
+def to_torch_bf16(bits: np.ndarray, device="cpu"):
+    """The bf16 bit patterns as a torch.bfloat16 tensor on `device` (bit-exact)."""
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.to(device)

@@ -2,6 +2,8 @@
 parity bars (absolute/mean error on O, absolute on LSE, relative Frobenius on gradients)."""
 from __future__ import annotations
 
+import functools
+
 import numpy as np
 import torch
 
@@ -15,16 +17,24 @@ GRAD_REL_FRO = 2e-2
 
 
 def bits_to_torch(bits: np.ndarray, device) -> torch.Tensor:
-    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
-    return t.to(device)
+    return synth.to_torch_bf16(bits, device)
 
 
 def bits_to_f64(bits: np.ndarray) -> np.ndarray:
     return synth.bf16_bits_to_f32(bits).astype(np.float64)
 
 
+@functools.lru_cache(maxsize=8)
+def _stream(seed: int, n: int) -> np.ndarray:
+    return synth.normal_bf16(seed, n)
+
+
 def make_case(B, H, N, d, seed=synth.BASE_SEED, device="cuda", with_do=True):
-    bits = synth.attention_inputs(B, H, N, d, seed, with_do=with_do)
+    """Same bytes as synth.attention_inputs (cached: many cases share stream lengths)."""
+    n, shape = B * H * N * d, (B, H, N, d)
+    names = ("q", "k", "v", "do") if with_do else ("q", "k", "v")
+    offs = (synth.SEED_Q, synth.SEED_K, synth.SEED_V, synth.SEED_DO)
+    bits = {k: _stream(seed + o, n).reshape(shape) for k, o in zip(names, offs)}
     gpu = {k: bits_to_torch(v, device) for k, v in bits.items()}
     f64 = {k: bits_to_f64(v) for k, v in bits.items()}
     return gpu, f64
