@@ -4,3 +4,4 @@
 #include "fa_fwd.cu"
 #include "fa_bwd.cu"
 #include "fa_bwd_aux.cu"
+#include "fa_bwd_noalloc.cu"

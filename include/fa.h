@@ -25,7 +25,8 @@
  *    128J..128J+127 ([P1] §Block-Sparse FlashAttention). Tiles that are off are never
  *    loaded or computed. causal and block_mask combine (AND).
  *  - All pointers are device memory owned by the caller. The library allocates no device
- *    memory apart from one static device status word.
+ *    memory apart from one static device status word and the fixed scratch array that
+ *    fa_bwd_noalloc uses.
  *  - Every pointer must be 16-byte aligned. d must be 64 or 128. N must be a positive
  *    multiple of 128 (other N: FA_ERR_UNSUPPORTED).
  *  - stream is a cudaStream_t (NULL = legacy default stream). All calls are asynchronous
@@ -103,6 +104,27 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* d
                       void* stream);
 fa_status fa_bwd_dq_finish(void* dq, int B, int H, int N, int d, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/*
+ * Backward pass without a caller workspace, for callers that cannot allocate device memory
+ * (hosts that own every allocation and forbid allocating from their execution callbacks,
+ * real-time loops that must not allocate once started). The source pages have no
+ * counterpart: this is a deployment convenience, not part of the method.
+ * Same arguments, outputs and numerics as fa_bwd, minus the workspace. The workspace comes
+ * from a fixed array of FA_NOALLOC_SCRATCH_BYTES in the library's device memory, reserved
+ * on every GPU that loads the library until the process exits. Problems whose
+ * fa_bwd_workspace_bytes exceed it return FA_ERR_WORKSPACE (about (d+2)*4 bytes per query
+ * row: B*H*N up to ~129k rows at d = 128, ~254k at d = 64). Allocates nothing.
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current; make that first call before any stream capture. All calls share
+ * the one array: calls whose kernels overlap on the GPU (different streams, no ordering)
+ * race on it and give wrong results. Calls ordered on one stream are safe: each call
+ * re-initialises everything it reads from the array.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                         float scale, int causal, const uint8_t* block_mask, void* stream);
 
 /*
  * Synchronises `stream`, then reports and clears the device status word: FA_ERR_TIMEOUT if
