@@ -34,15 +34,41 @@ def sources():
     return sorted(CSRC.glob("*.cu")) + sorted(CSRC.glob("*.cuh")) + sorted(CSRC.glob("*.h")) + [ROOT / "include" / "fa.h"]
 
 
+# Kernels that re-balance registers with setmaxnreg: the launch allocation ptxas reports must
+# be exactly what their warpgroup split adds up to (see ptx.cuh, reg_alloc/reg_dealloc).
+REG_SPLIT_KERNELS = {"fa_fwd_kernel": 168, "fa_bwd_kernel": 168}
+
+
+def check_register_split(ptxas_log: str) -> None:
+    cur = None
+    for line in ptxas_log.splitlines():
+        if "Compiling entry function" in line:
+            cur = next((k for k in REG_SPLIT_KERNELS if k in line), None)
+        elif cur and "Used" in line and "registers" in line:
+            n = int(line.split("Used")[1].split("registers")[0])
+            if n != REG_SPLIT_KERNELS[cur]:
+                raise RuntimeError(f"{cur}: launch allocation {n} registers/thread, the setmaxnreg split "
+                                   f"assumes {REG_SPLIT_KERNELS[cur]}; refusing to build")
+            cur = None
+
+
 def build(force: bool = False, verbose: bool = False) -> Path:
     newest = max(p.stat().st_mtime for p in sources())
     if not force and LIB.exists() and LIB.stat().st_mtime >= newest:
         return LIB
     tmp = LIB.with_suffix(f".so.tmp{os.getpid()}")
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", str(ROOT / "include"), str(CSRC / "libfa.cu"), "-o", str(tmp)]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
+    cmd = [nvcc(), "-Xptxas=-v", *NVCC_FLAGS, "-I", str(ROOT / "include"), str(CSRC / "libfa.cu"), "-o", str(tmp)]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if verbose or res.returncode != 0:
+        sys.stdout.write(res.stdout)
+        sys.stderr.write(res.stderr)
+    if res.returncode != 0:
+        raise subprocess.CalledProcessError(res.returncode, cmd)
+    try:
+        check_register_split(res.stderr + res.stdout)
+    except RuntimeError:
+        tmp.unlink(missing_ok=True)
+        raise
     os.replace(tmp, LIB)
     return LIB
 

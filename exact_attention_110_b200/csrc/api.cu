@@ -4,7 +4,7 @@
 #include <math.h>
 #include <mutex>
 
-#include "../../include/fa.h"
+#include "fa.h"  // include/ is on the include path
 #include "kernels.h"
 #include "ptx.cuh"
 

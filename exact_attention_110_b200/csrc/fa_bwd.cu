@@ -15,21 +15,33 @@
 //
 // sm_100a design (ours):
 //  * CTA = one 128-key tile j of one (b, h). K_j and V_j stay in shared memory; Q_i, dO_i (and
-//    the 128 LSE2 / D values of tile i) stream through an NS-deep ring.
-//  * Everything is computed transposed so that on-chip results are directly operands:
-//      S^T = K_j Q_i^T, dP^T = V_j dO_i^T           (TMEM, one key per TMEM lane)
-//      P^T = exp2(S^T * scale*log2e - LSE2_i)        (written back over S^T, bf16, in TMEM)
-//      dS^T = P^T o (dP^T - D_i)                    (bf16, 128B-swizzled shared memory)
+//    the 128 values -LSE_i*log2e and -D_i of tile i) stream through an NS-deep ring.
+//  * Everything is computed transposed so on-chip results are directly MMA operands:
+//      S^T = K_j Q_i^T, dP^T = V_j dO_i^T            (TMEM, one key per TMEM lane)
+//      P^T = exp2(S^T * scale*log2e - LSE_i*log2e)     (bf16, written back over S^T in TMEM)
+//      dS^T = P^T o (dP^T - D_i)                      (bf16, 128B-swizzled shared memory)
 //      dV += P^T dO_i   (A = P^T from TMEM)
 //      dK += dS^T Q_i   (A = dS^T, K-major)
-//      dQ_i = dS K_j    (A = the same dS^T buffer read MN-major, B = K_j MN-major)
-//  * Warp 0 TMA producer, warp 1 MMA issuer (single thread), warps 4-7 compute P and dS
-//    (thread = key row), warps 8-11 drain dQ_i from TMEM and add it (times scale) into the
-//    fp32 accumulator with 16-byte red.global.add, then write dK, dV at the end.
-//  * TMEM: S^T/P^T [0,128), dP^T [128,256) (reused for dQ_i once dP^T is consumed),
-//    dV [256,256+D), dK [256+D,256+2D).
+//      dQ_i: d = 128: dQ_i^T = K_j^T dS_i^T (A = K_j MN-major, B = dS^T MN-major), so TMEM lane
+//            = head-dim index and a warp's fp32 adds into the accumulator hit 128 contiguous
+//            bytes (whole L2 sectors); d = 64: dQ_i = dS K_j (lane = query row).
+//  * Roles: warp 0 TMA; warp 1 MMA issuer (one thread; descriptors precomputed, so each MMA
+//    costs only an add); warps 4-7 compute P (P phase) then dS (dS phase), thread = key row;
+//    warps 8-11 drain dQ from TMEM and add scale*dQ into the fp32 accumulator with
+//    red.global.add, then write dK (times scale); warps 4-7 write dV.
+//  * MMA order per query tile i: dV_i as soon as P_i is in TMEM; S_{i+1} (the compute warps
+//    start the next P phase while the tensor core still works on tile i); dQ_i; dK_i (covers
+//    the dQ drain); dP_{i+1}.
+//  * TMEM: S^T/P^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D); dQ: d = 128
+//    reuses the dP^T columns once dP^T has been read, d = 64 has its own [384,448).
 #include "kernels.h"
 #include "ptx.cuh"
+
+#ifndef FA_BWD_REGS_CTRL
+#define FA_BWD_REGS_CTRL 120
+#define FA_BWD_REGS_PDS 216
+#define FA_BWD_REGS_DQ 168
+#endif
 
 namespace fa {
 
@@ -46,13 +58,20 @@ struct BwdCfg {
   static constexpr int OFF_DO = OFF_Q + NS * TILE_BYTES;
   static constexpr int OFF_DS = OFF_DO + NS * TILE_BYTES;  // 128 keys x 128 queries bf16
   static constexpr int DS_BYTES = 2 * PANEL_BYTES;
-  static constexpr int OFF_LSE = OFF_DS + DS_BYTES;        // [NS][128] fp32
-  static constexpr int OFF_DEL = OFF_LSE + NS * 512;       // [NS][128] fp32
+  static constexpr int OFF_LSE = OFF_DS + DS_BYTES;        // [NS][128] fp32: -LSE*log2e
+  static constexpr int OFF_DEL = OFF_LSE + NS * 512;       // [NS][128] fp32: -D
   static constexpr int OFF_BAR = OFF_DEL + NS * 512;
-  static constexpr int NBAR = 1 + 2 * NS + 6 + 1;
+  static constexpr int NBAR = 1 + 2 * NS + 11;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int TMEM_COLS = 512;
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
+  static constexpr bool DQ_T = (D == 128);               // transposed dQ (lane = head dim)
+  static constexpr uint32_t T_DQ = DQ_T ? 128u : 384u;   // d = 128 aliases the dP^T columns
+  // setmaxnreg split of the launch allocation (384 x 168, checked by the build script).
+  // Control warpgroup (TMA, MMA, 2 idle warps), P/dS warpgroup, dQ-drain warpgroup.
+  static constexpr int REGS_CTRL = FA_BWD_REGS_CTRL, REGS_PDS = FA_BWD_REGS_PDS, REGS_DQ = FA_BWD_REGS_DQ;
+  static_assert(128 * (REGS_CTRL + REGS_PDS + REGS_DQ) <= 384 * 168, "setmaxnreg split exceeds the launch");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -60,6 +79,34 @@ __device__ __forceinline__ bool bwd_tile_active(const BwdParams& p, int i, int j
   if (p.causal && i < j) return false;
   if (p.block_mask != nullptr && p.block_mask[i * p.nb + j] == 0) return false;
   return true;
+}
+
+__device__ __forceinline__ void red_add_f32(float* addr, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+}
+
+// Writes one accumulator row (D fp32 columns of TMEM lane `row`, times `mul`) as bf16 into a
+// 128-row tile staged in the TMA store layout (64-column 128B-swizzled panels).
+template <int D>
+__device__ __forceinline__ void stage_row_bf16(uint32_t taddr, uint32_t sstage, int row, float mul, bool zero) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t u[32];
+    if (!zero) {
+      tmem_ld32(taddr + c * 32, u);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) u[e] = 0u;
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) w[e] = pack_bf16(__uint_as_float(u[2 * e]) * mul, __uint_as_float(u[2 * e + 1]) * mul);
+    const uint32_t panel = sstage + ((c * 32) >> 6) * (128 * 128);
+    const uint32_t ch0 = ((c * 32) & 63) >> 3;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      st_shared_v4(panel + sw128_offset(row, ch0 + q), w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+  }
 }
 
 template <int D>
@@ -80,10 +127,12 @@ __global__ void __launch_bounds__(384, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* bar_kv = bars;               // K_j, V_j landed
-  uint64_t* bar_qf = bars + 1;           // [NS] Q_i, dO_i, LSE2_i, D_i landed
+  uint64_t* bar_qf = bars + 1;           // [NS] Q_i, dO_i, -LSE2_i, -D_i landed
   uint64_t* bar_qe = bar_qf + NS;        // [NS] stage free
-  uint64_t* bar_sdp = bar_qe + NS;       // S^T_i and dP^T_i ready in TMEM
-  uint64_t* bar_ds = bar_sdp + 1;        // P^T_i in TMEM, dS^T_i in smem, S/dP fully read
+  uint64_t* bar_s = bar_qe + NS;         // S^T_i ready in TMEM
+  uint64_t* bar_dp = bar_s + 1;          // dP^T_i ready in TMEM
+  uint64_t* bar_p = bar_dp + 1;          // P^T_i written to TMEM (S^T_i fully read)
+  uint64_t* bar_ds = bar_p + 1;          // dS^T_i in smem, dP^T_i fully read
   uint64_t* bar_dsfree = bar_ds + 1;     // MMAs reading dS^T_i done
   uint64_t* bar_dq = bar_dsfree + 1;     // dQ_i ready in TMEM
   uint64_t* bar_dqfree = bar_dq + 1;     // dQ_i read out of TMEM
@@ -103,7 +152,9 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bar_qf[s], 1);
       mbar_init(&bar_qe[s], 1);
     }
-    mbar_init(bar_sdp, 1);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_dp, 1);
+    mbar_init(bar_p, 4);
     mbar_init(bar_ds, 4);
     mbar_init(bar_dsfree, 1);
     mbar_init(bar_dq, 1);
@@ -124,6 +175,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t sK = smem_u32(smem + C::OFF_K), sV = smem_u32(smem + C::OFF_V);
   const uint32_t sQ = smem_u32(smem + C::OFF_Q), sdO = smem_u32(smem + C::OFF_DO);
   const uint32_t sDS = smem_u32(smem + C::OFF_DS);
+  if (warp < 4) reg_dealloc<C::REGS_CTRL>();  // producer, MMA issuer and two idle warps
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -165,30 +217,46 @@ __global__ void __launch_bounds__(384, 1)
         for (int s = 0; s < NS; ++s)
           if (issued[s] >= 0) mbar_wait(&bar_qf[s], issued[s], &none, lim, WAIT_BWD_LOAD + 2);
       }
-      // K/V are always consumed by someone unless the CTA aborts; make sure they landed.
-      mbar_wait(bar_kv, 0, &none, lim, WAIT_BWD_LOAD + 3);
+      mbar_wait(bar_kv, 0, &none, lim, WAIT_BWD_LOAD + 3);  // K/V landed before the CTA can exit
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);  // K/V (A) and Q/dO (B), K-major
       constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, 0, 1);   // dV, dK: B = dO / Q MN-major
-      constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, 1, 1);    // dQ: A = dS MN-major, B = K MN-major
-      const uint32_t tS = tmem + 0u, tDP = tmem + 128u, tDV = tmem + 256u, tDK = tmem + 256u + D;
+      constexpr uint32_t IDESC_Q = C::DQ_T ? idesc_bf16_f32(128, 128, 1, 1)  // dQ^T = K^T dS^T
+                                           : idesc_bf16_f32(128, D, 1, 1);   // dQ = dS K
+      constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
+      const uint32_t tS = tmem + C::T_S, tDP = tmem + C::T_DP, tDV = tmem + C::T_DV, tDK = tmem + C::T_DK;
+      const uint32_t tDQ = tmem + C::T_DQ;
+      const uint64_t dK_k = sdesc_sw128(sK, 16, 1024);               // K as K-major A (S^T)
+      const uint64_t dV_k = sdesc_sw128(sV, 16, 1024);               // V as K-major A (dP^T)
+      const uint64_t dK_mn = sdesc_sw128(sK, C::PANEL_BYTES, 1024);  // K read MN-major (dQ)
+      const uint64_t dQ_k = sdesc_sw128(sQ, 16, 1024);               // Q_i as K-major B (S^T)
+      const uint64_t dQ_mn = sdesc_sw128(sQ, C::PANEL_BYTES, 1024);  // Q_i as MN-major B (dK)
+      const uint64_t dO_k = sdesc_sw128(sdO, 16, 1024);
+      const uint64_t dO_mn = sdesc_sw128(sdO, C::PANEL_BYTES, 1024);
+      const uint64_t dS_k = sdesc_sw128(sDS, 16, 1024);              // dS^T as K-major A (dK)
+      const uint64_t dS_mn = sdesc_sw128(sDS, C::PANEL_BYTES, 1024); // dS^T read MN-major (dQ)
       bool ok = mbar_wait(bar_kv, 0, ab, lim, WAIT_BWD_MMA + 1);
 
-      auto issue_s_dp = [&](int s, bool do_s, bool do_dp) {
-        const uint32_t qb = sQ + s * C::TILE_BYTES, dob = sdO + s * C::TILE_BYTES;
+      auto issue_s = [&](int st) {
+        const uint64_t b = dQ_k + (uint64_t)(st * TILE16);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32;
-          if (do_s) umma_ss(tS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(qb + off, 16, 1024), IDESC_S, kk > 0);
-          if (do_dp)
-            umma_ss(tDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(dob + off, 16, 1024), IDESC_S, kk > 0);
+          const uint32_t off16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
+          umma_ss(tS, dK_k + off16, b + off16, IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_dp = [&](int st) {
+        const uint64_t b = dO_k + (uint64_t)(st * TILE16);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
+          umma_ss(tDP, dV_k + off16, b + off16, IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
 
-      // Find the first active tile.
       int i = i_begin;
       while (i < p.nb && !bwd_tile_active(p, i, j)) ++i;
       int it = 0;
@@ -196,52 +264,70 @@ __global__ void __launch_bounds__(384, 1)
         ok = mbar_wait(&bar_qf[0], 0, ab, lim, WAIT_BWD_MMA + 2);
         if (ok) {
           tc_fence_after();
-          issue_s_dp(0, true, true);
-          umma_commit(bar_sdp);
+          issue_s(0);
+          umma_commit(bar_s);
+          issue_dp(0);
+          umma_commit(bar_dp);
         }
       }
       while (ok && i < p.nb) {
         const int s = it % NS;
         int inext = i + 1;
         while (inext < p.nb && !bwd_tile_active(p, inext, j)) ++inext;
-        ok = mbar_wait(bar_ds, it & 1, ab, lim, WAIT_BWD_MMA + 3);
+        const bool has_next = inext < p.nb;
+        const int sn = (it + 1) % NS;
+        const uint32_t acc = it > 0 ? 1u : 0u;
+        const uint64_t dOs = dO_mn + (uint64_t)(s * TILE16), dQs = dQ_mn + (uint64_t)(s * TILE16);
+
+        // dV += P^T dO_i (reduction over the 128 queries of tile i), A = P^T from TMEM
+        ok = mbar_wait(bar_p, it & 1, ab, lim, WAIT_BWD_MMA + 3);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t qb = sQ + s * C::TILE_BYTES, dob = sdO + s * C::TILE_BYTES;
-        const uint32_t acc = it > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // reduction over the 128 queries of tile i
-          // dV += P^T dO_i
-          umma_ts(tDV, tS + kk * 8, sdesc_sw128(dob + kk * 2048, C::PANEL_BYTES, 1024), IDESC_KV,
-                  (acc || kk > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          // dK += dS^T Q_i
-          const uint32_t aoff = (kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32;
-          umma_ss(tDK, sdesc_sw128(sDS + aoff, 16, 1024), sdesc_sw128(qb + kk * 2048, C::PANEL_BYTES, 1024),
-                  IDESC_KV, (acc || kk > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // reduction over the 128 keys of tile j
-          // dQ_i = dS K_j  (into the dP^T columns, already consumed)
-          umma_ss(tDP, sdesc_sw128(sDS + kk * 2048, C::PANEL_BYTES, 1024),
-                  sdesc_sw128(sK + kk * 2048, C::PANEL_BYTES, 1024), IDESC_Q, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar_dq);
-        umma_commit(bar_dsfree);
-        umma_commit(&bar_qe[s]);
-        if (inext < p.nb) {
-          const int sn = (it + 1) % NS;
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tDV, tS + kk * 8, dOs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV, kk > 0 ? 1u : acc);
+        // S^T_{i+1} over P^T_i (the dV MMAs above read it first: tcgen05.mma runs in order)
+        if (has_next) {
           ok = mbar_wait(&bar_qf[sn], ((it + 1) / NS) & 1, ab, lim, WAIT_BWD_MMA + 4);
           if (!ok) break;
           tc_fence_after();
-          issue_s_dp(sn, true, false);  // S^T_{next}: P^T_i was consumed by the dV MMAs above
-          ok = mbar_wait(bar_dqfree, it & 1, ab, lim, WAIT_BWD_MMA + 5);
+          issue_s(sn);
+          umma_commit(bar_s);
+        }
+        ok = mbar_wait(bar_ds, it & 1, ab, lim, WAIT_BWD_MMA + 5);
+        if (!ok) break;
+        if (!C::DQ_T && it > 0) {  // d = 64: the dQ columns must have been drained
+          ok = mbar_wait(bar_dqfree, (it - 1) & 1, ab, lim, WAIT_BWD_MMA + 6);
           if (!ok) break;
-          tc_fence_after();
-          issue_s_dp(sn, false, true);  // dP^T_{next} once dQ_i has left TMEM
-          umma_commit(bar_sdp);
+        }
+        tc_fence_after();
+        // dQ_i (d = 128: into the dP^T columns, already read by the dS phase)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // reduction over the 128 keys of tile j
+          const uint64_t kdesc = dK_mn + (uint64_t)(kk * (2048 >> 4)), sdesc = dS_mn + (uint64_t)(kk * (2048 >> 4));
+          if (C::DQ_T)
+            umma_ss(tDQ, kdesc, sdesc, IDESC_Q, kk > 0 ? 1u : 0u);
+          else
+            umma_ss(tDQ, sdesc, kdesc, IDESC_Q, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_dq);
+        // dK += dS^T Q_i
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
+          umma_ss(tDK, dS_k + aoff16, dQs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV, kk > 0 ? 1u : acc);
+        }
+        umma_commit(bar_dsfree);
+        umma_commit(&bar_qe[s]);
+        // dP^T_{i+1}
+        if (has_next) {
+          if (C::DQ_T) {  // the dP^T columns hold dQ_i until the drain warps have read it
+            ok = mbar_wait(bar_dqfree, it & 1, ab, lim, WAIT_BWD_MMA + 7);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          issue_dp(sn);
+          umma_commit(bar_dp);
         }
         i = inext;
         ++it;
@@ -249,57 +335,89 @@ __global__ void __launch_bounds__(384, 1)
       umma_commit(bar_acc);
       umma_commit(bar_done);
       AbortState none{0};
-      mbar_wait(bar_done, 0, &none, lim, WAIT_BWD_MMA + 6);
+      mbar_wait(bar_done, 0, &none, lim, WAIT_BWD_MMA + 8);
     }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------------ P and dS (thread = key row)
+    reg_alloc<C::REGS_PDS>();
     const uint32_t wq = warp & 3;
     const int kr = wq * 32 + lane;  // key row inside tile j
     const uint32_t lane_off = (wq * 32u) << 16;
-    const uint32_t tS_row = tmem + lane_off, tDP_row = tmem + lane_off + 128u;
-    const float sl2 = p.scale_log2;
+    const uint32_t tS_row = tmem + lane_off + C::T_S, tDP_row = tmem + lane_off + C::T_DP;
+    const uint64_t sl2_2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     int it = 0;
     for (int i = i_begin; i < p.nb; ++i) {
       if (!bwd_tile_active(p, i, j)) continue;
       const int s = it % NS;
-      ok = warp_wait(bar_sdp, it & 1, ab, lim, WAIT_BWD_COMPUTE + 1);
-      if (ok && it > 0) ok = warp_wait(bar_dsfree, (it - 1) & 1, ab, lim, WAIT_BWD_COMPUTE + 2);
+      const float* nlse2 = reinterpret_cast<const float*>(smem + C::OFF_LSE + s * 512);
+      const float* ndel = reinterpret_cast<const float*>(smem + C::OFF_DEL + s * 512);
+      const bool diag = p.causal && i == j;
+
+      // ---- P phase: P^T = exp2(S^T * scale*log2e - LSE*log2e), back into TMEM as bf16
+      ok = warp_wait(bar_s, it & 1, ab, lim, WAIT_BWD_COMPUTE + 1);
       if (!ok) break;
       tc_fence_after();
-      const float* lse2 = reinterpret_cast<const float*>(smem + C::OFF_LSE + s * 512);
-      const float* del = reinterpret_cast<const float*>(smem + C::OFF_DEL + s * 512);
-      const bool diag = p.causal && i == j;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {  // 32 queries per chunk
-        uint32_t su[32], du[32];
-        tmem_ld32(tS_row + c * 32, su);
-        tmem_ld32(tDP_row + c * 32, du);
-        uint32_t pk[16], dk[16];
+      uint32_t su[128];
+      tmem_ld128(tS_row, su);
+      float pf[128];  // P in fp32, kept for the dS phase
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int q0 = c * 32 + e;
-          float p0 = ex2(fmaf(__uint_as_float(su[e]), sl2, -lse2[q0]));
-          float p1 = ex2(fmaf(__uint_as_float(su[e + 1]), sl2, -lse2[q0 + 1]));
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int q = 32 * c + 2 * e;
+          const float2 nl = *reinterpret_cast<const float2*>(&nlse2[q]);
+          const uint64_t x2 = ffma2(f2_pack(__uint_as_float(su[q]), __uint_as_float(su[q + 1])), sl2_2,
+                                    f2_pack(nl.x, nl.y));
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          float p0 = ex2(x0), p1 = ex2(x1);
           if (diag) {  // key kr is visible to query q iff kr <= q
-            if (q0 < kr) p0 = 0.f;
-            if (q0 + 1 < kr) p1 = 0.f;
+            if (q < kr) p0 = 0.f;
+            if (q + 1 < kr) p1 = 0.f;
           }
-          const float ds0 = p0 * (__uint_as_float(du[e]) - del[q0]);
-          const float ds1 = p1 * (__uint_as_float(du[e + 1]) - del[q0 + 1]);
-          pk[e >> 1] = pack_bf16(p0, p1);
-          dk[e >> 1] = pack_bf16(ds0, ds1);
+          pf[q] = p0;
+          pf[q + 1] = p1;
+          pk[e] = pack_bf16(p0, p1);
         }
-        // P^T chunk over S^T columns [16c, 16c+16): those scores were already read.
-        tmem_st16(tS_row + c * 16, pk);
+        tmem_st16(tS_row + c * 16, pk);  // columns [16c, 16c+16): scores already read
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p);
+
+      // ---- dS phase: dS^T = P^T o (dP^T - D) into the swizzled smem tile
+      ok = warp_wait(bar_dp, it & 1, ab, lim, WAIT_BWD_COMPUTE + 2);
+      if (ok && it > 0) ok = warp_wait(bar_dsfree, (it - 1) & 1, ab, lim, WAIT_BWD_COMPUTE + 3);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t dep = 0;  // chains each chunk's load after the previous chunk's math
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t du[32];
+        tmem_ld32_after(tDP_row + c * 32, du, dep);
+        uint32_t dk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int q = 32 * c + 2 * e;
+          const float2 nd = *reinterpret_cast<const float2*>(&ndel[q]);
+          const uint64_t t2 = fadd2(f2_pack(__uint_as_float(du[2 * e]), __uint_as_float(du[2 * e + 1])),
+                                    f2_pack(nd.x, nd.y));
+          const uint64_t ds2 = fmul2(f2_pack(pf[q], pf[q + 1]), t2);
+          float d0, d1;
+          f2_unpack(ds2, d0, d1);
+          dk[e] = pack_bf16(d0, d1);
+        }
+        dep = dk[15];
         // dS^T row kr, queries 32c..32c+31 -> panel c/2, 16-byte chunks (c%2)*4 .. +3
         const uint32_t panel = sDS + (c >> 1) * C::PANEL_BYTES;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          st_shared_v4(panel + sw128_offset(kr, (c & 1) * 4 + q), dk[4 * q], dk[4 * q + 1], dk[4 * q + 2],
-                       dk[4 * q + 3]);
+        for (int qq = 0; qq < 4; ++qq)
+          st_shared_v4(panel + sw128_offset(kr, (c & 1) * 4 + qq), dk[4 * qq], dk[4 * qq + 1], dk[4 * qq + 2],
+                       dk[4 * qq + 3]);
       }
-      tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -311,25 +429,7 @@ __global__ void __launch_bounds__(384, 1)
     uint8_t* stage = smem + C::OFF_Q;  // Q ring stage 0 is free once every MMA retired
     if (ok) {
       tc_fence_after();
-      const uint32_t sst = smem_u32(stage);
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t u[32];
-        if (it > 0) {
-          tmem_ld32(tmem + lane_off + 256u + c * 32, u);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) u[e] = 0u;
-        }
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) w[e] = pack_bf16(__uint_as_float(u[2 * e]), __uint_as_float(u[2 * e + 1]));
-        const uint32_t panel = sst + ((c * 32) >> 6) * C::PANEL_BYTES;
-        const uint32_t ch0 = ((c * 32) & 63) >> 3;
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          st_shared_v4(panel + sw128_offset(kr, ch0 + q), w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-      }
+      stage_row_bf16<D>(tmem + lane_off + C::T_DV, smem_u32(stage), kr, 1.f, it == 0);
       fence_proxy_async_smem();
     }
     named_bar_sync(1, 128);
@@ -339,11 +439,12 @@ __global__ void __launch_bounds__(384, 1)
       bulk_wait_group_read0();
     }
   } else if (warp >= 8) {
-    // ------------------------------------------------------------------ dQ drain (thread = query row)
+    // ------------------------------------------------------------------ dQ drain
+    reg_alloc<C::REGS_DQ>();
     const uint32_t wq = warp & 3;
-    const int qr = wq * 32 + lane;
+    const int ln = wq * 32 + lane;  // TMEM lane: head-dim index (d = 128) or query row (d = 64)
     const uint32_t lane_off = (wq * 32u) << 16;
-    const uint32_t tDQ_row = tmem + lane_off + 128u;
+    const uint32_t tDQ_row = tmem + lane_off + C::T_DQ;
     const float scale = p.scale;
     bool ok = true;
     int it = 0;
@@ -352,17 +453,29 @@ __global__ void __launch_bounds__(384, 1)
       ok = warp_wait(bar_dq, it & 1, ab, lim, WAIT_BWD_DQ + 1);
       if (!ok) break;
       tc_fence_after();
-      float* dst = p.dq_acc + ((size_t)bh * p.Np + (size_t)i * 128 + qr) * D;
-      uint32_t u[D];
+      float* tile = p.dq_acc + ((size_t)bh * p.Np + (size_t)i * 128) * D;
+      if (C::DQ_T) {
+        uint32_t u[128];  // dQ_i^T row `ln`: column q = query q of tile i
+        tmem_ld128(tDQ_row, u);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_dqfree);
+        // lanes of a warp hold 32 consecutive head-dim entries: each add covers 128 contiguous bytes
+        float* dst = tile + ln;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32(tDQ_row + c * 32, *reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_dqfree);
+        for (int q = 0; q < 128; ++q, dst += D) red_add_f32(dst, __uint_as_float(u[q]) * scale);
+      } else {
+        uint32_t u[64];
+        tmem_ld64(tDQ_row, u);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_dqfree);
+        float* dst = tile + (size_t)ln * D;
 #pragma unroll
-      for (int e = 0; e < D; e += 4)
-        red_add_v4(dst + e, __uint_as_float(u[e]) * scale, __uint_as_float(u[e + 1]) * scale,
-                   __uint_as_float(u[e + 2]) * scale, __uint_as_float(u[e + 3]) * scale);
+        for (int e = 0; e < 64; e += 4)
+          red_add_v4(dst + e, __uint_as_float(u[e]) * scale, __uint_as_float(u[e + 1]) * scale,
+                     __uint_as_float(u[e + 2]) * scale, __uint_as_float(u[e + 3]) * scale);
+      }
       ++it;
     }
     // -------------------------------------------------------------- epilogue: dK (times scale)
@@ -370,26 +483,7 @@ __global__ void __launch_bounds__(384, 1)
     uint8_t* stage = smem + C::OFF_DO;  // dO ring stage 0, free once every MMA retired
     if (ok) {
       tc_fence_after();
-      const uint32_t sst = smem_u32(stage);
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t u[32];
-        if (it > 0) {
-          tmem_ld32(tmem + lane_off + 256u + D + c * 32, u);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) u[e] = 0u;
-        }
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16(__uint_as_float(u[2 * e]) * scale, __uint_as_float(u[2 * e + 1]) * scale);
-        const uint32_t panel = sst + ((c * 32) >> 6) * C::PANEL_BYTES;
-        const uint32_t ch0 = ((c * 32) & 63) >> 3;
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          st_shared_v4(panel + sw128_offset(qr, ch0 + q), w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-      }
+      stage_row_bf16<D>(tmem + lane_off + C::T_DK, smem_u32(stage), ln, scale, it == 0);
       fence_proxy_async_smem();
     }
     named_bar_sync(2, 128);

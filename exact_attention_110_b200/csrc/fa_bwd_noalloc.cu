@@ -13,7 +13,7 @@
 // device with cudaGetSymbolAddress and cached.
 #include <mutex>
 
-#include "../../include/fa.h"
+#include "fa.h"  // include/ is on the include path
 
 static __device__ __align__(256) unsigned char g_fa_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
 

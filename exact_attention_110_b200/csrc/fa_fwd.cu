@@ -38,11 +38,19 @@
 #include "kernels.h"
 #include "ptx.cuh"
 
+#ifndef FA_FWD_EXP_EMU_MASK
+#define FA_FWD_EXP_EMU_MASK 0x0u
+#endif
+
 namespace fa {
 
 template <int D>
 struct FwdCfg {
-  static constexpr int THREADS = 384;
+  static constexpr int THREADS = 384;  // warp 0 TMA, warp 1 MMA, warps 4-11 softmax
+  // setmaxnreg split of the launch allocation (384 x 168, checked by the build script):
+  // the control warpgroup (TMA, MMA, 2 idle warps) keeps 88, the softmax warpgroups get 208.
+  static constexpr int REGS_CTRL = 88, REGS_SOFTMAX = 208;
+  static_assert(128 * REGS_CTRL + 256 * REGS_SOFTMAX <= 384 * 168, "setmaxnreg split exceeds the launch");
   static constexpr int NS = (D == 128) ? 2 : 4;        // K ring and V ring depth
   static constexpr int PANEL_BYTES = 128 * 128;        // 128 rows x 64 bf16 (one swizzle panel)
   static constexpr int PANELS = D / 64;
@@ -55,6 +63,9 @@ struct FwdCfg {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int TMEM_COLS = 512;
+  // Which of the 16 score pairs of each 32-score chunk take 2^x on the FMA pipe (ex2_poly)
+  // instead of the special-function unit: bit i set = pair i emulated.
+  static constexpr uint32_t EXP_EMU_MASK = FA_FWD_EXP_EMU_MASK;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -63,6 +74,46 @@ __device__ __forceinline__ bool fwd_tile_active(const FwdParams& p, int qb, int 
   if (p.causal && j > qb) return false;
   if (p.block_mask != nullptr && p.block_mask[qb * p.nb + j] == 0) return false;
   return true;
+}
+
+// p = 2^(s * scale * log2e - m_ref) for one row's 128 scores; P (bf16) goes back over the
+// scores it came from, 32 scores -> 16 packed columns per chunk, so chunk c only lands on
+// columns already read. Pairs whose bit is set in EMU_MASK (within each chunk of 16 pairs)
+// use the FMA-pipe polynomial, the rest the special-function unit; EMU = false forces the
+// special-function unit everywhere (masked tiles need exact zeros for -inf scores).
+// Returns the row sum of p.
+template <bool EMU, uint32_t EMU_MASK>
+__device__ __forceinline__ float softmax_exp_store(const uint32_t (&su)[128], uint64_t sl2_2, uint64_t mneg_2,
+                                                   uint32_t tS_row, const Ex2PolyConsts& K) {
+  uint64_t ls2[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) ls2[k] = 0ull;  // two +0.0f lanes
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint64_t s2 = f2_pack(__uint_as_float(su[32 * c + 2 * i]), __uint_as_float(su[32 * c + 2 * i + 1]));
+      const uint64_t x2 = ffma2(s2, sl2_2, mneg_2);
+      uint64_t p2;
+      if (EMU && ((EMU_MASK >> i) & 1u)) {
+        p2 = ex2_poly2(x2, K);
+      } else {
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        p2 = f2_pack(ex2(x0), ex2(x1));
+      }
+      ls2[i & 3] = fadd2(ls2[i & 3], p2);
+      float p0, p1;
+      f2_unpack(p2, p0, p1);
+      pk[i] = pack_bf16(p0, p1);
+    }
+    tmem_st16(tS_row + c * 16, pk);
+  }
+  const uint64_t t2 = fadd2(fadd2(ls2[0], ls2[1]), fadd2(ls2[2], ls2[3]));
+  float a, b;
+  f2_unpack(t2, a, b);
+  return a + b;
 }
 
 template <int D>
@@ -129,6 +180,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t sQ = smem_u32(smem + C::OFF_Q);
   const uint32_t sK = smem_u32(smem + C::OFF_K);
   const uint32_t sV = smem_u32(smem + C::OFF_V);
+  if (warp < 4) reg_dealloc<C::REGS_CTRL>();  // producer, MMA issuer and two idle warps
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -182,11 +234,17 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
+    // One thread issues everything. Shared-memory descriptors are built once; each MMA only
+    // adds a compile-time offset (the start-address field is address >> 4), so the issuing
+    // thread spends a few cycles per MMA instead of a dependent chain of 64-bit ALU ops --
+    // the issue rate, not the tensor core, otherwise limits M=128 x N=128 MMAs.
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);  // Q, K both K-major
       constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);    // P (TMEM), V MN-major
-      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
+      constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
+      const uint64_t dq_base = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t dk_base = sdesc_sw128(sK, 16, 1024);
+      const uint64_t dv_base = sdesc_sw128(sV, C::PANEL_BYTES, 1024);
       bool ok = true;
       for (int t = 0; t < 2 && ok; ++t)
         if (qb0 + t < p.nb) ok = mbar_wait(&bar_q[t], 0, ab, lim, WAIT_FWD_MMA + 1);
@@ -197,16 +255,6 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t prev_ph = 0;
       int it = 0;
 
-      auto issue_pv = [&](int t, int vs) {
-        const uint32_t vbase = sV + vs * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // 128 keys, 16 per MMA
-          const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::PANEL_BYTES, 1024);
-          umma_ts(tO[t], tS[t] + kk * 8, bdesc, IDESC_O, (o_started[t] || kk > 0) ? 1u : 0u);
-        }
-        o_started[t] = true;
-      };
-
       for (int j = 0; j < j_end && ok; ++j) {
         const bool act0 = fwd_tile_active(p, qb0, j), act1 = fwd_tile_active(p, qb0 + 1, j);
         if (!act0 && !act1) continue;
@@ -215,23 +263,29 @@ __global__ void __launch_bounds__(384, 1)
         ok = mbar_wait(&bar_kf[s], ph, ab, lim, WAIT_FWD_MMA + 2);
         if (!ok) break;
         tc_fence_after();
-        const bool act[2] = {act0, act1};
-        for (int t = 0; t < 2 && ok; ++t) {
+        const uint64_t dk = dk_base + (uint64_t)(s * TILE16);
+        const uint64_t dv_prev = dv_base + (uint64_t)((prev_s < 0 ? 0 : prev_s) * TILE16);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
           if (prev_act[t]) {  // O_t += P_t V_{previous}
             ok = mbar_wait(&bar_vf[prev_s], prev_ph, ab, lim, WAIT_FWD_MMA + 3);
             if (ok) ok = mbar_wait(&bar_p[t], p_phase[t], ab, lim, WAIT_FWD_MMA + 4);
             if (!ok) break;
             p_phase[t] ^= 1u;
             tc_fence_after();
-            issue_pv(t, prev_s);
+            const uint32_t acc0 = o_started[t] ? 1u : 0u;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per MMA
+              umma_ts(tmem + 256u + t * D, tmem + t * 128u + kk * 8, dv_prev + (uint64_t)(kk * (2048 >> 4)), IDESC_O,
+                      kk > 0 ? 1u : acc0);
+            o_started[t] = true;
           }
-          if (act[t]) {  // S_t = Q_t K_j^T
-            const uint32_t qbase = sQ + t * C::TILE_BYTES, kbase = sK + s * C::TILE_BYTES;
+          if (act0 && t == 0 || act1 && t == 1) {  // S_t = Q_t K_j^T
+            const uint64_t dq = dq_base + (uint64_t)(t * TILE16);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32;
-              umma_ss(tS[t], sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024), IDESC_S,
-                      kk > 0 ? 1u : 0u);
+              const uint32_t off16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
+              umma_ss(tmem + t * 128u, dq + off16, dk + off16, IDESC_S, kk > 0 ? 1u : 0u);
             }
             umma_commit(&bar_s[t]);
           }
@@ -245,14 +299,22 @@ __global__ void __launch_bounds__(384, 1)
         prev_act[1] = act1;
         ++it;
       }
-      for (int t = 0; t < 2 && ok; ++t) {  // last PV of each tile
-        if (prev_act[t]) {
+      const uint64_t dv_last = dv_base + (uint64_t)((prev_s < 0 ? 0 : prev_s) * TILE16);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {  // last PV of each tile
+        if (ok && prev_act[t]) {
           ok = mbar_wait(&bar_vf[prev_s], prev_ph, ab, lim, WAIT_FWD_MMA + 5);
           if (ok) ok = mbar_wait(&bar_p[t], p_phase[t], ab, lim, WAIT_FWD_MMA + 6);
-          if (!ok) break;
-          p_phase[t] ^= 1u;
-          tc_fence_after();
-          issue_pv(t, prev_s);
+          if (ok) {
+            p_phase[t] ^= 1u;
+            tc_fence_after();
+            const uint32_t acc0 = o_started[t] ? 1u : 0u;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_ts(tmem + 256u + t * D, tmem + t * 128u + kk * 8, dv_last + (uint64_t)(kk * (2048 >> 4)), IDESC_O,
+                      kk > 0 ? 1u : acc0);
+            o_started[t] = true;
+          }
         }
       }
       if (ok && prev_s >= 0) umma_commit(&bar_ve[prev_s]);
@@ -264,7 +326,8 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ softmax warpgroups
-    const int t = (warp - 4) >> 2;
+    reg_alloc<C::REGS_SOFTMAX>();
+    const int t = (warp - 4) >> 2;    // warps 4-7: tile 0, warps 8-11: tile 1
     const uint32_t wq = warp & 3;      // TMEM lane quarter this warp may touch
     const int r = wq * 32 + lane;      // row inside the tile
     const int qb = qb0 + t;
@@ -273,6 +336,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tS_row = tmem + lane_off + t * 128u;
     const uint32_t tO_row = tmem + lane_off + 256u + t * D;
     const float sl2 = p.scale_log2;
+    const Ex2PolyConsts ek = ex2_poly_consts();
     float m_ref = -INFINITY;  // reference max, log2 domain, scale folded in
     float l = 0.f;            // running sum of exp2(x - m_ref)
     uint32_t s_phase = 0;
@@ -287,22 +351,23 @@ __global__ void __launch_bounds__(384, 1)
         s_phase ^= 1u;
         tc_fence_after();
 
-        float sv[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t u[32];
-          tmem_ld32(tS_row + c * 32, u);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(u[i]);
-        }
+        uint32_t su[128];  // this row's 128 scores (fp32 bits)
+        tmem_ld128(tS_row, su);
         if (p.causal && j == qb) {  // diagonal tile: key 128j+c is visible to row 128qb+r iff c <= r
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            if (c > r) sv[c] = -INFINITY;
+            if (c > r) su[c] = 0xff800000u;  // -inf
         }
-        float mx = sv[0];
+        // Row max: 8 independent chains of three-input max, then a short tree.
+        float mc[8];
 #pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, sv[c]);
+        for (int k = 0; k < 8; ++k) {
+          float m = fmax3(__uint_as_float(su[k]), __uint_as_float(su[k + 8]), __uint_as_float(su[k + 16]));
+#pragma unroll
+          for (int c = 24; c < 120; c += 16) m = fmax3(m, __uint_as_float(su[c + k]), __uint_as_float(su[c + 8 + k]));
+          mc[k] = fmaxf(m, __uint_as_float(su[120 + k]));
+        }
+        const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
         const float cand = mx * sl2;
         float alpha = 1.f;
         if (cand > m_ref + 8.f) {  // also taken on the first visible tile (m_ref = -inf)
@@ -322,22 +387,11 @@ __global__ void __launch_bounds__(384, 1)
         }
         l *= alpha;
         const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        uint32_t pk[64];
-        float lsum = 0.f;
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p0 = ex2(fmaf(sv[2 * i], sl2, mneg));
-          const float p1 = ex2(fmaf(sv[2 * i + 1], sl2, mneg));
-          lsum += p0 + p1;
-          pk[i] = pack_bf16(p0, p1);
-        }
-        l += lsum;
-        {
-          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t (*)[32]>(&pk[0]);
-          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t (*)[32]>(&pk[32]);
-          tmem_st32(tS_row, lo);
-          tmem_st32(tS_row + 32, hi);
-        }
+        const uint64_t sl2_2 = f2_pack(sl2, sl2), mneg_2 = f2_pack(mneg, mneg);
+        if (p.causal && j == qb)
+          l += softmax_exp_store<false, 0u>(su, sl2_2, mneg_2, tS_row, ek);
+        else
+          l += softmax_exp_store<true, C::EXP_EMU_MASK>(su, sl2_2, mneg_2, tS_row, ek);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();

@@ -37,16 +37,16 @@ struct BwdPreParams {
   const uint16_t* o;     // bf16 [BH][N][D]
   const uint16_t* dout;  // bf16 [BH][N][D]
   const float* lse;      // [BH][N]
-  float* delta;          // [BH][Np]
-  float* lse2;           // [BH][Np]  = LSE * log2(e)
+  float* delta;          // [BH][Np]  = -D = -rowsum(dO o O)
+  float* lse2;           // [BH][Np]  = -LSE * log2(e)
   float* dq_acc;         // [BH][Np][D], zeroed here
   long long rows;        // BH * N
   int N, Np, D;
 };
 
 struct BwdParams {
-  const float* delta;    // [BH][Np]
-  const float* lse2;     // [BH][Np]
+  const float* delta;    // [BH][Np]  -D
+  const float* lse2;     // [BH][Np]  -LSE * log2(e)
   float* dq_acc;         // [BH][Np][D]
   const uint8_t* block_mask;
   int N, Np, nb;
