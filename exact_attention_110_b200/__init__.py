@@ -21,7 +21,7 @@ import torch
 
 __all__ = [
     "FAError", "forward", "backward", "bwd_workspace_bytes", "bwd_preprocess", "bwd_main",
-    "bwd_dq_finish", "last_device_status", "library", "LIB_PATH",
+    "bwd_dq_finish", "last_device_status", "selftest_wait_timeout", "library", "LIB_PATH",
 ]
 
 LIB_PATH = Path(__file__).resolve().with_name("libfa.so")
@@ -64,6 +64,8 @@ def library() -> ctypes.CDLL:
         lib.fa_bwd_dq_finish.argtypes = [vp, i32, i32, i32, i32, vp, sz, vp]
         lib.fa_last_device_status.restype = i32
         lib.fa_last_device_status.argtypes = [vp]
+        lib.fa_selftest_wait_timeout.restype = i32
+        lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
         _lib = lib
     return _lib
 
@@ -171,6 +173,12 @@ def bwd_dq_finish(workspace, shape, device, dq=None):
     _check(library().fa_bwd_dq_finish(_ptr(dq), B, H, N, d, _ptr(workspace), nbytes, _stream(device)),
            "fa_bwd_dq_finish")
     return dq
+
+
+def selftest_wait_timeout(limit_us: int = 20000, device=None) -> None:
+    """Enqueues the failure-detection self-test (a bounded wait that is meant to give up)."""
+    dev = torch.device("cuda") if device is None else device
+    _check(library().fa_selftest_wait_timeout(int(limit_us), _stream(dev)), "fa_selftest_wait_timeout")
 
 
 def last_device_status(device=None) -> int:

@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t dO_mn = sdesc_sw128(sdO, C::PANEL_BYTES, 1024);
       const uint64_t dS_k = sdesc_sw128(sDS, 16, 1024);              // dS^T as K-major A (dK)
       const uint64_t dS_mn = sdesc_sw128(sDS, C::PANEL_BYTES, 1024); // dS^T read MN-major (dQ)
-      bool ok = mbar_wait(bar_kv, 0, ab, lim, WAIT_BWD_MMA + 1);
+      bool ok = mbar_wait_spin(bar_kv, 0, ab, lim, WAIT_BWD_MMA + 1);
 
       auto issue_s = [&](int st) {
         const uint64_t b = dQ_k + (uint64_t)(st * TILE16);
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(384, 1)
       while (i < p.nb && !bwd_tile_active(p, i, j)) ++i;
       int it = 0;
       if (ok && i < p.nb) {
-        ok = mbar_wait(&bar_qf[0], 0, ab, lim, WAIT_BWD_MMA + 2);
+        ok = mbar_wait_spin(&bar_qf[0], 0, ab, lim, WAIT_BWD_MMA + 2);
         if (ok) {
           tc_fence_after();
           issue_s(0);
@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t dOs = dO_mn + (uint64_t)(s * TILE16), dQs = dQ_mn + (uint64_t)(s * TILE16);
 
         // dV += P^T dO_i (reduction over the 128 queries of tile i), A = P^T from TMEM
-        ok = mbar_wait(bar_p, it & 1, ab, lim, WAIT_BWD_MMA + 3);
+        ok = mbar_wait_spin(bar_p, it & 1, ab, lim, WAIT_BWD_MMA + 3);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -288,16 +288,16 @@ __global__ void __launch_bounds__(384, 1)
           umma_ts(tDV, tS + kk * 8, dOs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV, kk > 0 ? 1u : acc);
         // S^T_{i+1} over P^T_i (the dV MMAs above read it first: tcgen05.mma runs in order)
         if (has_next) {
-          ok = mbar_wait(&bar_qf[sn], ((it + 1) / NS) & 1, ab, lim, WAIT_BWD_MMA + 4);
+          ok = mbar_wait_spin(&bar_qf[sn], ((it + 1) / NS) & 1, ab, lim, WAIT_BWD_MMA + 4);
           if (!ok) break;
           tc_fence_after();
           issue_s(sn);
           umma_commit(bar_s);
         }
-        ok = mbar_wait(bar_ds, it & 1, ab, lim, WAIT_BWD_MMA + 5);
+        ok = mbar_wait_spin(bar_ds, it & 1, ab, lim, WAIT_BWD_MMA + 5);
         if (!ok) break;
         if (!C::DQ_T && it > 0) {  // d = 64: the dQ columns must have been drained
-          ok = mbar_wait(bar_dqfree, (it - 1) & 1, ab, lim, WAIT_BWD_MMA + 6);
+          ok = mbar_wait_spin(bar_dqfree, (it - 1) & 1, ab, lim, WAIT_BWD_MMA + 6);
           if (!ok) break;
         }
         tc_fence_after();
@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(384, 1)
         // dP^T_{i+1}
         if (has_next) {
           if (C::DQ_T) {  // the dP^T columns hold dQ_i until the drain warps have read it
-            ok = mbar_wait(bar_dqfree, it & 1, ab, lim, WAIT_BWD_MMA + 7);
+            ok = mbar_wait_spin(bar_dqfree, it & 1, ab, lim, WAIT_BWD_MMA + 7);
             if (!ok) break;
             tc_fence_after();
           }

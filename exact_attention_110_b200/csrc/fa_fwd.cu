@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t dv_base = sdesc_sw128(sV, C::PANEL_BYTES, 1024);
       bool ok = true;
       for (int t = 0; t < 2 && ok; ++t)
-        if (qb0 + t < p.nb) ok = mbar_wait(&bar_q[t], 0, ab, lim, WAIT_FWD_MMA + 1);
+        if (qb0 + t < p.nb) ok = mbar_wait_spin(&bar_q[t], 0, ab, lim, WAIT_FWD_MMA + 1);
       uint32_t p_phase[2] = {0u, 0u};
       bool o_started[2] = {false, false};
       bool prev_act[2] = {false, false};
@@ -260,7 +260,9 @@ __global__ void __launch_bounds__(384, 1)
         if (!act0 && !act1) continue;
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
-        ok = mbar_wait(&bar_kf[s], ph, ab, lim, WAIT_FWD_MMA + 2);
+        ok = mbar_wait_spin(&bar_kf[s], ph, ab, lim, WAIT_FWD_MMA + 2);
+        // V of the previous KV tile (used by this step's PV MMAs of both tiles): waited once
+        if (ok && prev_s >= 0 && (prev_act[0] || prev_act[1])) ok = mbar_wait_spin(&bar_vf[prev_s], prev_ph, ab, lim, WAIT_FWD_MMA + 3);
         if (!ok) break;
         tc_fence_after();
         const uint64_t dk = dk_base + (uint64_t)(s * TILE16);
@@ -268,8 +270,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           if (prev_act[t]) {  // O_t += P_t V_{previous}
-            ok = mbar_wait(&bar_vf[prev_s], prev_ph, ab, lim, WAIT_FWD_MMA + 3);
-            if (ok) ok = mbar_wait(&bar_p[t], p_phase[t], ab, lim, WAIT_FWD_MMA + 4);
+            ok = mbar_wait_spin(&bar_p[t], p_phase[t], ab, lim, WAIT_FWD_MMA + 4);
             if (!ok) break;
             p_phase[t] ^= 1u;
             tc_fence_after();
@@ -303,8 +304,8 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int t = 0; t < 2; ++t) {  // last PV of each tile
         if (ok && prev_act[t]) {
-          ok = mbar_wait(&bar_vf[prev_s], prev_ph, ab, lim, WAIT_FWD_MMA + 5);
-          if (ok) ok = mbar_wait(&bar_p[t], p_phase[t], ab, lim, WAIT_FWD_MMA + 6);
+          ok = mbar_wait_spin(&bar_vf[prev_s], prev_ph, ab, lim, WAIT_FWD_MMA + 5);
+          if (ok) ok = mbar_wait_spin(&bar_p[t], p_phase[t], ab, lim, WAIT_FWD_MMA + 6);
           if (ok) {
             p_phase[t] ^= 1u;
             tc_fence_after();

@@ -5,3 +5,4 @@
 #include "fa_bwd.cu"
 #include "fa_bwd_aux.cu"
 #include "fa_bwd_noalloc.cu"
+#include "selftest.cu"

@@ -46,10 +46,24 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  // The suspend-time hint (ns) lets a waiting warp sleep until the phase completes instead
+  // of re-polling the barrier; polling warps measurably slow the tensor core's issue path.
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(100000u)
+      : "memory");
+  return ok != 0;
+}
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.b32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -78,6 +92,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, AbortS
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
+    if (*reinterpret_cast<volatile int*>(&ab->flag)) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *reinterpret_cast<volatile int*>(&ab->flag) = 1;
+      atomicCAS(&g_fa_device_status, 0, where);
+      return false;
+    }
+  }
+}
+
+// Bounded wait for the single thread that issues tcgen05.mma: spins on the non-blocking
+// test_wait. A blocking try_wait in that thread costs ~90 cycles of tensor-core issue even when
+// the phase has already completed; test_wait does not.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, AbortState* ab, uint64_t limit_ns,
+                                               int where) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_test_wait(bar, parity)) return true;
     if (*reinterpret_cast<volatile int*>(&ab->flag)) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       *reinterpret_cast<volatile int*>(&ab->flag) = 1;

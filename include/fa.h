@@ -133,6 +133,16 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
  */
 fa_status fa_last_device_status(void* stream);
 
+/*
+ * Failure-detection self-test (no counterpart on the pages; it tests the library's own
+ * device-side wait limits). Enqueues one tiny kernel whose single thread waits, bounded by
+ * limit_us microseconds (1 .. 1,000,000), on a barrier that nothing arrives at. The wait
+ * gives up exactly as a stuck attention kernel would: it records a code in the device
+ * status word and returns, leaving the context usable. A following fa_last_device_status
+ * reports FA_ERR_TIMEOUT. Returns FA_ERR_INVALID for an out-of-range limit.
+ */
+fa_status fa_selftest_wait_timeout(unsigned int limit_us, void* stream);
+
 /* Static, human-readable name of a status code. Never NULL. */
 const char* fa_status_string(fa_status status);
 

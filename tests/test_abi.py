@@ -84,3 +84,10 @@ def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(fa, "_lib", None)
     with pytest.raises(RuntimeError, match="no fallback"):
         fa.library()
+
+
+def test_selftest_rejects_out_of_range_limit(lib):
+    lib.fa_selftest_wait_timeout.restype = ctypes.c_int
+    lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, ctypes.c_void_p]
+    assert lib.fa_selftest_wait_timeout(0, None) == 1
+    assert lib.fa_selftest_wait_timeout(2000000, None) == 1

@@ -167,3 +167,15 @@ def test_fully_masked_query_block(fa, oracle_mod):
     assert torch.all(dq[:, :, :128] == 0)
     g_ref = oracle_mod.attention_bwd(ref["q"], ref["k"], ref["v"], ref["do"], 0.125, mask=m)[:3]
     H.assert_grads_close([H.to_f64(x) for x in (dq, dk, dv)], g_ref, "fully masked block")
+
+
+def test_bounded_wait_timeout_is_reported_and_context_survives(fa):
+    # A device-side wait that runs out (on a barrier nothing arrives at) must be reported as
+    # FA_ERR_TIMEOUT by the host and leave the context usable for the next call.
+    assert fa.last_device_status() == 0
+    fa.selftest_wait_timeout(20000)
+    assert fa.last_device_status() == 4  # FA_ERR_TIMEOUT, and the word is cleared
+    assert fa.last_device_status() == 0
+    gpu, _ = H.make_case(1, 1, 256, 64, seed=13)
+    o, lse = run_fwd(fa, gpu, False, None, 0.125)
+    assert torch.isfinite(o.float()).all()
