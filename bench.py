@@ -71,6 +71,25 @@ def reduce_max(value: float, dist_on: bool, device=None) -> float:
     return float(t.item())
 
 
+def kernel_source_hash() -> str:
+    import hashlib
+    m = hashlib.sha256()
+    for f in ("exact_attention_110_b200/csrc/fa_bwd.cu", "exact_attention_110_b200/csrc/ptx.cuh"):
+        m.update((ROOT / f).read_bytes())
+    return m.hexdigest()[:16]
+
+
+def recorded_traffic(key: str):
+    """DRAM bytes per launch from the last ncu capture, or None if the kernel changed since."""
+    tfile = ROOT / "profiles" / "traffic.json"
+    if not tfile.exists():
+        return None
+    rec = json.loads(tfile.read_text()).get(key)
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec["bytes"]
+
+
 def load_peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -296,12 +315,7 @@ def run_gpu(args, wl, rank, world, local_rank, dist_on):
     # ---- roofline of the dominant kernel (bwd main: 5 of the 7 matmuls of a step)
     main_flops = 2.5 * f_fwd
     achieved = main_flops / (main_ms * 1e-3) / 1e12
-    traffic = None
-    tfile = ROOT / "profiles" / "traffic.json"
-    if tfile.exists():
-        tj = json.loads(tfile.read_text()).get(f"bwd_main N={N} d={d} causal={int(causal)} bs={int(wl['block_sparse'])}")
-        if tj is not None:
-            traffic = tj
+    traffic = recorded_traffic(f"bwd_main N={N} d={d} causal={int(causal)} bs={int(wl['block_sparse'])}")
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"], "traffic": traffic, "kernel": "fa_bwd_kernel",
                 "peak_kind": f"bf16 dense burst ({peaks['source']})",
