@@ -26,9 +26,10 @@
 //            = head-dim index and a warp's fp32 adds into the accumulator hit 128 contiguous
 //            bytes (whole L2 sectors); d = 64: dQ_i = dS K_j (lane = query row).
 //  * Roles: warp 0 TMA; warp 1 MMA issuer (one thread; descriptors precomputed, so each MMA
-//    costs only an add); warps 4-7 compute P (P phase) then dS (dS phase), thread = key row;
-//    warps 8-11 drain dQ from TMEM and add scale*dQ into the fp32 accumulator with
-//    red.global.add, then write dK (times scale); warps 4-7 write dV.
+//    costs only an add); warps 4-7 and 8-11 compute P (P phase) then dS (dS phase) for query
+//    columns 0-63 and 64-127 respectively, thread = key row; warps 12-15 drain dQ from TMEM
+//    and add scale*dQ into the fp32 accumulator with red.global.add, then write dK (times
+//    scale); warps 4-11 write dV.
 //  * MMA order per query tile i: dV_i as soon as P_i is in TMEM; S_{i+1} (the compute warps
 //    start the next P phase while the tensor core still works on tile i); dQ_i; dK_i (covers
 //    the dQ drain); dP_{i+1}.
@@ -38,16 +39,16 @@
 #include "ptx.cuh"
 
 #ifndef FA_BWD_REGS_CTRL
-#define FA_BWD_REGS_CTRL 120
-#define FA_BWD_REGS_PDS 216
-#define FA_BWD_REGS_DQ 168
+#define FA_BWD_REGS_CTRL 104
+#define FA_BWD_REGS_PDS 128
+#define FA_BWD_REGS_DQ 152
 #endif
 
 namespace fa {
 
 template <int D>
 struct BwdCfg {
-  static constexpr int THREADS = 384;
+  static constexpr int THREADS = 512;
   static constexpr int NS = (D == 128) ? 2 : 3;  // Q/dO ring depth
   static constexpr int PANEL_BYTES = 128 * 128;
   static constexpr int PANELS = D / 64;
@@ -68,10 +69,10 @@ struct BwdCfg {
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
   static constexpr bool DQ_T = (D == 128);               // transposed dQ (lane = head dim)
   static constexpr uint32_t T_DQ = DQ_T ? 128u : 384u;   // d = 128 aliases the dP^T columns
-  // setmaxnreg split of the launch allocation (384 x 168, checked by the build script).
-  // Control warpgroup (TMA, MMA, 2 idle warps), P/dS warpgroup, dQ-drain warpgroup.
+  // setmaxnreg split of the launch allocation (512 x 128, checked by the build script):
+  // control warpgroup (TMA, MMA, 2 idle warps), two P/dS warpgroups, dQ-drain warpgroup.
   static constexpr int REGS_CTRL = FA_BWD_REGS_CTRL, REGS_PDS = FA_BWD_REGS_PDS, REGS_DQ = FA_BWD_REGS_DQ;
-  static_assert(128 * (REGS_CTRL + REGS_PDS + REGS_DQ) <= 384 * 168, "setmaxnreg split exceeds the launch");
+  static_assert(128 * (REGS_CTRL + 2 * REGS_PDS + REGS_DQ) <= 512 * 128, "setmaxnreg split exceeds the launch");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -110,7 +111,7 @@ __device__ __forceinline__ void stage_row_bf16(uint32_t taddr, uint32_t sstage, 
 }
 
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
@@ -154,8 +155,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(bar_s, 1);
     mbar_init(bar_dp, 1);
-    mbar_init(bar_p, 4);
-    mbar_init(bar_ds, 4);
+    mbar_init(bar_p, 8);   // one arrive per P/dS warp (two warpgroups)
+    mbar_init(bar_ds, 8);
     mbar_init(bar_dsfree, 1);
     mbar_init(bar_dq, 1);
     mbar_init(bar_dqfree, 4);
@@ -285,7 +286,8 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tDV, tS + kk * 8, dOs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV, kk > 0 ? 1u : acc);
+          umma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, dOs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV,
+                  kk > 0 ? 1u : acc);
         // S^T_{i+1} over P^T_i (the dV MMAs above read it first: tcgen05.mma runs in order)
         if (has_next) {
           ok = mbar_wait_spin(&bar_qf[sn], ((it + 1) / NS) & 1, ab, lim, WAIT_BWD_MMA + 4);
@@ -337,86 +339,115 @@ __global__ void __launch_bounds__(384, 1)
       AbortState none{0};
       mbar_wait(bar_done, 0, &none, lim, WAIT_BWD_MMA + 8);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------------ P and dS (thread = key row)
+    // Two warpgroups split the 128 queries of a tile: group h owns query columns [64h, 64h+64)
+    // of S^T and dP^T, writes its P^T into S^T columns [64h, 64h+32) (already read by itself)
+    // and its dS^T into shared-memory panel h. TMEM loads are issued one chunk ahead.
     reg_alloc<C::REGS_PDS>();
+    const int h = (warp - 4) >> 2;
     const uint32_t wq = warp & 3;
     const int kr = wq * 32 + lane;  // key row inside tile j
     const uint32_t lane_off = (wq * 32u) << 16;
-    const uint32_t tS_row = tmem + lane_off + C::T_S, tDP_row = tmem + lane_off + C::T_DP;
+    const uint32_t tS_row = tmem + lane_off + C::T_S + 64u * h, tDP_row = tmem + lane_off + C::T_DP + 64u * h;
     const uint64_t sl2_2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     int it = 0;
     for (int i = i_begin; i < p.nb; ++i) {
       if (!bwd_tile_active(p, i, j)) continue;
       const int s = it % NS;
-      const float* nlse2 = reinterpret_cast<const float*>(smem + C::OFF_LSE + s * 512);
-      const float* ndel = reinterpret_cast<const float*>(smem + C::OFF_DEL + s * 512);
+      const float* nlse2 = reinterpret_cast<const float*>(smem + C::OFF_LSE + s * 512) + 64 * h;
+      const float* ndel = reinterpret_cast<const float*>(smem + C::OFF_DEL + s * 512) + 64 * h;
       const bool diag = p.causal && i == j;
+      const int qoff = 64 * h;  // query index of column 0 of this group
 
       // ---- P phase: P^T = exp2(S^T * scale*log2e - LSE*log2e), back into TMEM as bf16
       ok = warp_wait(bar_s, it & 1, ab, lim, WAIT_BWD_COMPUTE + 1);
       if (!ok) break;
       tc_fence_after();
-      uint32_t su[128];
-      tmem_ld128(tS_row, su);
-      float pf[128];  // P in fp32, kept for the dS phase
+      float pf[64];  // P in fp32, kept for the dS phase
+      {
+        uint32_t sa[32], sb[32];
+        tmem_ld32_async(tS_row, sa);
+        tmem_wait_ld_tied(sa);
+        tmem_ld32_async(tS_row + 32, sb);  // in flight while chunk 0 is processed
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        for (int c = 0; c < 2; ++c) {
+          uint32_t (&su)[32] = c == 0 ? sa : sb;
+          if (c == 1) tmem_wait_ld_tied(sb);
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int q = 32 * c + 2 * e;
-          const float2 nl = *reinterpret_cast<const float2*>(&nlse2[q]);
-          const uint64_t x2 = ffma2(f2_pack(__uint_as_float(su[q]), __uint_as_float(su[q + 1])), sl2_2,
-                                    f2_pack(nl.x, nl.y));
-          float x0, x1;
-          f2_unpack(x2, x0, x1);
-          float p0 = ex2(x0), p1 = ex2(x1);
-          if (diag) {  // key kr is visible to query q iff kr <= q
-            if (q < kr) p0 = 0.f;
-            if (q + 1 < kr) p1 = 0.f;
+          for (int e = 0; e < 16; e += 2) {
+            const int q = 32 * c + 2 * e;  // local query index of this 4-query group
+            const float4 nl = *reinterpret_cast<const float4*>(&nlse2[q]);
+            const uint64_t x01 = ffma2(f2_pack(__uint_as_float(su[2 * e]), __uint_as_float(su[2 * e + 1])), sl2_2,
+                                       f2_pack(nl.x, nl.y));
+            const uint64_t x23 = ffma2(f2_pack(__uint_as_float(su[2 * e + 2]), __uint_as_float(su[2 * e + 3])),
+                                       sl2_2, f2_pack(nl.z, nl.w));
+            float x0, x1, x2, x3;
+            f2_unpack(x01, x0, x1);
+            f2_unpack(x23, x2, x3);
+            float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+            if (diag) {  // key kr is visible to query qoff+q iff kr <= qoff+q
+              const int qq = qoff + q;
+              if (qq < kr) p0 = 0.f;
+              if (qq + 1 < kr) p1 = 0.f;
+              if (qq + 2 < kr) p2 = 0.f;
+              if (qq + 3 < kr) p3 = 0.f;
+            }
+            pf[q] = p0;
+            pf[q + 1] = p1;
+            pf[q + 2] = p2;
+            pf[q + 3] = p3;
+            pk[e] = pack_bf16(p0, p1);
+            pk[e + 1] = pack_bf16(p2, p3);
           }
-          pf[q] = p0;
-          pf[q + 1] = p1;
-          pk[e] = pack_bf16(p0, p1);
+          tmem_st16(tS_row + c * 16, pk);  // columns [64h + 16c, +16): scores already read
         }
-        tmem_st16(tS_row + c * 16, pk);  // columns [16c, 16c+16): scores already read
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_p);
 
-      // ---- dS phase: dS^T = P^T o (dP^T - D) into the swizzled smem tile
+      // ---- dS phase: dS^T = P^T o (dP^T - D) into shared-memory panel h
       ok = warp_wait(bar_dp, it & 1, ab, lim, WAIT_BWD_COMPUTE + 2);
       if (ok && it > 0) ok = warp_wait(bar_dsfree, (it - 1) & 1, ab, lim, WAIT_BWD_COMPUTE + 3);
       if (!ok) break;
       tc_fence_after();
-      uint32_t dep = 0;  // chains each chunk's load after the previous chunk's math
+      {
+        uint32_t da[32], db[32];
+        tmem_ld32_async(tDP_row, da);
+        tmem_wait_ld_tied(da);
+        tmem_ld32_async(tDP_row + 32, db);
+        const uint32_t panel = sDS + h * C::PANEL_BYTES;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t du[32];
-        tmem_ld32_after(tDP_row + c * 32, du, dep);
-        uint32_t dk[16];
+        for (int c = 0; c < 2; ++c) {
+          uint32_t (&du)[32] = c == 0 ? da : db;
+          if (c == 1) tmem_wait_ld_tied(db);
+          uint32_t dk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int q = 32 * c + 2 * e;
-          const float2 nd = *reinterpret_cast<const float2*>(&ndel[q]);
-          const uint64_t t2 = fadd2(f2_pack(__uint_as_float(du[2 * e]), __uint_as_float(du[2 * e + 1])),
-                                    f2_pack(nd.x, nd.y));
-          const uint64_t ds2 = fmul2(f2_pack(pf[q], pf[q + 1]), t2);
-          float d0, d1;
-          f2_unpack(ds2, d0, d1);
-          dk[e] = pack_bf16(d0, d1);
+          for (int e = 0; e < 16; e += 2) {
+            const int q = 32 * c + 2 * e;
+            const float4 nd = *reinterpret_cast<const float4*>(&ndel[q]);
+            const uint64_t t01 = fadd2(f2_pack(__uint_as_float(du[2 * e]), __uint_as_float(du[2 * e + 1])),
+                                       f2_pack(nd.x, nd.y));
+            const uint64_t t23 = fadd2(f2_pack(__uint_as_float(du[2 * e + 2]), __uint_as_float(du[2 * e + 3])),
+                                       f2_pack(nd.z, nd.w));
+            const uint64_t ds01 = fmul2(f2_pack(pf[q], pf[q + 1]), t01);
+            const uint64_t ds23 = fmul2(f2_pack(pf[q + 2], pf[q + 3]), t23);
+            float d0, d1, d2, d3;
+            f2_unpack(ds01, d0, d1);
+            f2_unpack(ds23, d2, d3);
+            dk[e] = pack_bf16(d0, d1);
+            dk[e + 1] = pack_bf16(d2, d3);
+          }
+          // dS^T row kr, local queries 32c..32c+31 -> 16-byte chunks 4c .. 4c+3 of panel h
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq)
+            st_shared_v4(panel + sw128_offset(kr, c * 4 + qq), dk[4 * qq], dk[4 * qq + 1], dk[4 * qq + 2],
+                         dk[4 * qq + 3]);
         }
-        dep = dk[15];
-        // dS^T row kr, queries 32c..32c+31 -> panel c/2, 16-byte chunks (c%2)*4 .. +3
-        const uint32_t panel = sDS + (c >> 1) * C::PANEL_BYTES;
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq)
-          st_shared_v4(panel + sw128_offset(kr, (c & 1) * 4 + qq), dk[4 * qq], dk[4 * qq + 1], dk[4 * qq + 2],
-                       dk[4 * qq + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -424,21 +455,21 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0) mbar_arrive(bar_ds);
       ++it;
     }
-    // -------------------------------------------------------------- epilogue: dV
+    // -------------------------------------------------------------- epilogue: dV (group h: panel h)
     if (ok) ok = warp_wait(bar_acc, 0, ab, lim, WAIT_BWD_EPILOGUE + 1);
     uint8_t* stage = smem + C::OFF_Q;  // Q ring stage 0 is free once every MMA retired
-    if (ok) {
+    if (ok && h < C::PANELS) {
       tc_fence_after();
-      stage_row_bf16<D>(tmem + lane_off + C::T_DV, smem_u32(stage), kr, 1.f, it == 0);
+      stage_row_bf16<64>(tmem + lane_off + C::T_DV + 64u * h, smem_u32(stage + h * C::PANEL_BYTES), kr, 1.f, it == 0);
       fence_proxy_async_smem();
     }
-    named_bar_sync(1, 128);
-    if (wq == 0 && lane == 0 && *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
+    named_bar_sync(1, 256);
+    if (warp == 4 && lane == 0 && *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
       for (int pn = 0; pn < C::PANELS; ++pn) tma_store_3d(&tmdV, stage + pn * C::PANEL_BYTES, pn * 64, j * 128, bh);
       bulk_commit_group();
       bulk_wait_group_read0();
     }
-  } else if (warp >= 8) {
+  } else if (warp >= 12) {
     // ------------------------------------------------------------------ dQ drain
     reg_alloc<C::REGS_DQ>();
     const uint32_t wq = warp & 3;
@@ -456,7 +487,8 @@ __global__ void __launch_bounds__(384, 1)
       float* tile = p.dq_acc + ((size_t)bh * p.Np + (size_t)i * 128) * D;
       if (C::DQ_T) {
         uint32_t u[128];  // dQ_i^T row `ln`: column q = query q of tile i
-        tmem_ld128(tDQ_row, u);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tDQ_row + c * 32, *reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_dqfree);

@@ -304,6 +304,24 @@ __device__ __forceinline__ void tmem_ld32_after(uint32_t taddr, uint32_t (&r)[32
       : "r"(taddr), "r"(dep)
       : "memory");
 }
+// Asynchronous 32-column load: the registers are valid only after tmem_wait_ld_tied(r).
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : FA_R8(0), FA_R8(8), FA_R8(16), FA_R8(24)
+      : "r"(taddr)
+      : "memory");
+}
+#define FA_T8(i) "+r"(r[i + 0]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), \
+                 "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])
+// Waits for this warp's outstanding TMEM loads. `r` is passed through the asm so no use of
+// those registers can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld_tied(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : FA_T8(0), FA_T8(8), FA_T8(16), FA_T8(24)::"memory");
+}
+#undef FA_T8
 // Loads 16 columns and waits.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
