@@ -49,7 +49,14 @@ namespace fa {
 template <int D>
 struct BwdCfg {
   static constexpr int THREADS = 512;
-  static constexpr int NS = (D == 128) ? 2 : 3;  // Q/dO ring depth
+  static constexpr int NS = (D == 128) ? 2 : 3;     // Q ring depth (with -LSE*log2e and -D)
+  // d = 128: dO is single-buffered to make room for the dQ staging buffer. dO_i is last read by
+  // dV_i and next needed by dP_{i+1}, three MMA groups later, which covers the load.
+  static constexpr int NS_DO = (D == 128) ? 1 : NS;
+  static constexpr bool DQ_BULK = (D == 128);       // dQ combined by bulk reductions from smem
+  static constexpr int DQ_ROWS = 16;                // queries per bulk reduction (8 KB at d = 128)
+  static constexpr int DQ_SLOTS = 4;                // staging slots in flight
+  static constexpr int DQ_SLOT_BYTES = DQ_ROWS * D * 4;
   static constexpr int PANEL_BYTES = 128 * 128;
   static constexpr int PANELS = D / 64;
   static constexpr int TILE_BYTES = PANELS * PANEL_BYTES;
@@ -57,12 +64,14 @@ struct BwdCfg {
   static constexpr int OFF_V = OFF_K + TILE_BYTES;
   static constexpr int OFF_Q = OFF_V + TILE_BYTES;
   static constexpr int OFF_DO = OFF_Q + NS * TILE_BYTES;
-  static constexpr int OFF_DS = OFF_DO + NS * TILE_BYTES;  // 128 keys x 128 queries bf16
+  static constexpr int OFF_DS = OFF_DO + NS_DO * TILE_BYTES;  // 128 keys x 128 queries bf16
   static constexpr int DS_BYTES = 2 * PANEL_BYTES;
-  static constexpr int OFF_LSE = OFF_DS + DS_BYTES;        // [NS][128] fp32: -LSE*log2e
-  static constexpr int OFF_DEL = OFF_LSE + NS * 512;       // [NS][128] fp32: -D
+  static constexpr int OFF_DQS = OFF_DS + DS_BYTES;           // dQ staging [DQ_SLOTS][DQ_ROWS][D] fp32
+  static constexpr int DQS_BYTES = DQ_BULK ? DQ_SLOTS * DQ_SLOT_BYTES : 0;
+  static constexpr int OFF_LSE = OFF_DQS + DQS_BYTES;         // [NS][128] fp32: -LSE*log2e
+  static constexpr int OFF_DEL = OFF_LSE + NS * 512;          // [NS][128] fp32: -D
   static constexpr int OFF_BAR = OFF_DEL + NS * 512;
-  static constexpr int NBAR = 1 + 2 * NS + 11;
+  static constexpr int NBAR = 1 + 2 * NS + 2 * NS_DO + 9;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int TMEM_COLS = 512;
@@ -117,7 +126,7 @@ __global__ void __launch_bounds__(512, 1)
                   const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                   const BwdParams p) {
   using C = BwdCfg<D>;
-  constexpr int NS = C::NS;
+  constexpr int NS = C::NS, NS_DO = C::NS_DO;
   extern __shared__ __align__(1024) uint8_t smem[];
 
   const uint32_t warp = warp_id(), lane = lane_id();
@@ -128,9 +137,11 @@ __global__ void __launch_bounds__(512, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* bar_kv = bars;               // K_j, V_j landed
-  uint64_t* bar_qf = bars + 1;           // [NS] Q_i, dO_i, -LSE2_i, -D_i landed
-  uint64_t* bar_qe = bar_qf + NS;        // [NS] stage free
-  uint64_t* bar_s = bar_qe + NS;         // S^T_i ready in TMEM
+  uint64_t* bar_qf = bars + 1;           // [NS] Q_i, -LSE2_i, -D_i landed
+  uint64_t* bar_qe = bar_qf + NS;        // [NS] Q stage free (after dK_i)
+  uint64_t* bar_dof = bar_qe + NS;       // [NS_DO] dO_i landed
+  uint64_t* bar_doe = bar_dof + NS_DO;   // [NS_DO] dO stage free (after dV_i)
+  uint64_t* bar_s = bar_doe + NS_DO;     // S^T_i ready in TMEM
   uint64_t* bar_dp = bar_s + 1;          // dP^T_i ready in TMEM
   uint64_t* bar_p = bar_dp + 1;          // P^T_i written to TMEM (S^T_i fully read)
   uint64_t* bar_ds = bar_p + 1;          // dS^T_i in smem, dP^T_i fully read
@@ -152,6 +163,10 @@ __global__ void __launch_bounds__(512, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(&bar_qf[s], 1);
       mbar_init(&bar_qe[s], 1);
+    }
+    for (int s = 0; s < NS_DO; ++s) {
+      mbar_init(&bar_dof[s], 1);
+      mbar_init(&bar_doe[s], 1);
     }
     mbar_init(bar_s, 1);
     mbar_init(bar_dp, 1);
@@ -191,32 +206,42 @@ __global__ void __launch_bounds__(512, 1)
         tma_load_3d(smem + C::OFF_V + pn * C::PANEL_BYTES, &tmV, bar_kv, pn * 64, j * 128, bh);
       }
       int it = 0;
-      int issued[NS];
+      int issued[NS], issued_do[NS_DO];
       for (int s = 0; s < NS; ++s) issued[s] = -1;
+      for (int s = 0; s < NS_DO; ++s) issued_do[s] = -1;
       bool ok = true;
       for (int i = i_begin; i < p.nb; ++i) {
         if (!bwd_tile_active(p, i, j)) continue;
+        // Q_i first: its stage frees at dK_{i-NS}, before dO_i's stage frees at dV_{i-NS_DO}.
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
         ok = mbar_wait(&bar_qe[s], ph ^ 1, ab, lim, WAIT_BWD_LOAD + 1);
         if (!ok) break;
-        mbar_arrive_expect_tx(&bar_qf[s], 2 * C::TILE_BYTES + 1024);
-        for (int pn = 0; pn < C::PANELS; ++pn) {
+        mbar_arrive_expect_tx(&bar_qf[s], C::TILE_BYTES + 1024);
+        for (int pn = 0; pn < C::PANELS; ++pn)
           tma_load_3d(smem + C::OFF_Q + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &bar_qf[s], pn * 64, i * 128,
                       bh);
-          tma_load_3d(smem + C::OFF_DO + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmdO, &bar_qf[s], pn * 64,
-                      i * 128, bh);
-        }
         const size_t vec = (size_t)bh * p.Np + (size_t)i * 128;
         bulk_load(smem + C::OFF_LSE + s * 512, p.lse2 + vec, 512, &bar_qf[s]);
         bulk_load(smem + C::OFF_DEL + s * 512, p.delta + vec, 512, &bar_qf[s]);
         issued[s] = ph;
+        const int sd = it % NS_DO;
+        const uint32_t phd = (it / NS_DO) & 1;
+        ok = mbar_wait(&bar_doe[sd], phd ^ 1, ab, lim, WAIT_BWD_LOAD + 4);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bar_dof[sd], C::TILE_BYTES);
+        for (int pn = 0; pn < C::PANELS; ++pn)
+          tma_load_3d(smem + C::OFF_DO + sd * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmdO, &bar_dof[sd], pn * 64,
+                      i * 128, bh);
+        issued_do[sd] = phd;
         ++it;
       }
       AbortState none{0};
       if (!ok) {
         for (int s = 0; s < NS; ++s)
           if (issued[s] >= 0) mbar_wait(&bar_qf[s], issued[s], &none, lim, WAIT_BWD_LOAD + 2);
+        for (int s = 0; s < NS_DO; ++s)
+          if (issued_do[s] >= 0) mbar_wait(&bar_dof[s], issued_do[s], &none, lim, WAIT_BWD_LOAD + 5);
       }
       mbar_wait(bar_kv, 0, &none, lim, WAIT_BWD_LOAD + 3);  // K/V landed before the CTA can exit
     }
@@ -267,6 +292,10 @@ __global__ void __launch_bounds__(512, 1)
           tc_fence_after();
           issue_s(0);
           umma_commit(bar_s);
+          ok = mbar_wait_spin(&bar_dof[0], 0, ab, lim, WAIT_BWD_MMA + 9);
+        }
+        if (ok) {
+          tc_fence_after();
           issue_dp(0);
           umma_commit(bar_dp);
         }
@@ -277,8 +306,9 @@ __global__ void __launch_bounds__(512, 1)
         while (inext < p.nb && !bwd_tile_active(p, inext, j)) ++inext;
         const bool has_next = inext < p.nb;
         const int sn = (it + 1) % NS;
+        const int sd = it % NS_DO, sdn = (it + 1) % NS_DO;
         const uint32_t acc = it > 0 ? 1u : 0u;
-        const uint64_t dOs = dO_mn + (uint64_t)(s * TILE16), dQs = dQ_mn + (uint64_t)(s * TILE16);
+        const uint64_t dOs = dO_mn + (uint64_t)(sd * TILE16), dQs = dQ_mn + (uint64_t)(s * TILE16);
 
         // dV += P^T dO_i (reduction over the 128 queries of tile i), A = P^T from TMEM
         ok = mbar_wait_spin(bar_p, it & 1, ab, lim, WAIT_BWD_MMA + 3);
@@ -288,6 +318,7 @@ __global__ void __launch_bounds__(512, 1)
         for (int kk = 0; kk < 8; ++kk)
           umma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, dOs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV,
                   kk > 0 ? 1u : acc);
+        umma_commit(&bar_doe[sd]);  // dO_i read by dP_i and dV_i
         // S^T_{i+1} over P^T_i (the dV MMAs above read it first: tcgen05.mma runs in order)
         if (has_next) {
           ok = mbar_wait_spin(&bar_qf[sn], ((it + 1) / NS) & 1, ab, lim, WAIT_BWD_MMA + 4);
@@ -326,9 +357,11 @@ __global__ void __launch_bounds__(512, 1)
           if (C::DQ_T) {  // the dP^T columns hold dQ_i until the drain warps have read it
             ok = mbar_wait_spin(bar_dqfree, it & 1, ab, lim, WAIT_BWD_MMA + 7);
             if (!ok) break;
-            tc_fence_after();
           }
-          issue_dp(sn);
+          ok = mbar_wait_spin(&bar_dof[sdn], ((it + 1) / NS_DO) & 1, ab, lim, WAIT_BWD_MMA + 10);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dp(sdn);
           umma_commit(bar_dp);
         }
         i = inext;
@@ -477,16 +510,47 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t lane_off = (wq * 32u) << 16;
     const uint32_t tDQ_row = tmem + lane_off + C::T_DQ;
     const float scale = p.scale;
+    const uint32_t sDQS = smem_u32(smem + C::OFF_DQS);
+    const bool issuer = (wq == 0 && lane == 0);  // issues the bulk reductions of the warpgroup
     bool ok = true;
     int it = 0;
+    uint32_t slot = 0;  // bulk reductions issued so far (staging slot = slot % DQ_SLOTS)
     for (int i = i_begin; i < p.nb; ++i) {
       if (!bwd_tile_active(p, i, j)) continue;
       ok = warp_wait(bar_dq, it & 1, ab, lim, WAIT_BWD_DQ + 1);
+      // the four warps must leave together: they meet at named barriers below
+      if (C::DQ_BULK) ok = named_bar_and(3, 128, ok);
       if (!ok) break;
       tc_fence_after();
       float* tile = p.dq_acc + ((size_t)bh * p.Np + (size_t)i * 128) * D;
-      if (C::DQ_T) {
+      if (C::DQ_BULK) {
         uint32_t u[128];  // dQ_i^T row `ln`: column q = query q of tile i
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tDQ_row + c * 32, *reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_dqfree);
+        // Stage scale*dQ_i row-major ([query][head dim], lanes write 128 contiguous bytes) in
+        // DQ_ROWS-query slots; one thread adds each slot to the fp32 accumulator with a bulk
+        // reduction (performed in L2), keeping DQ_SLOTS - 1 of them in flight.
+#pragma unroll
+        for (int g = 0; g < 128 / C::DQ_ROWS; ++g, ++slot) {
+          if (issuer && slot >= C::DQ_SLOTS) bulk_wait_group_read<C::DQ_SLOTS - 1>();
+          named_bar_sync(3, 128);  // the slot's previous reduction has read it
+          const uint32_t sbuf = sDQS + (slot % C::DQ_SLOTS) * C::DQ_SLOT_BYTES + ln * 4;
+#pragma unroll
+          for (int r = 0; r < C::DQ_ROWS; ++r)
+            st_shared_f32(sbuf + r * (D * 4), __uint_as_float(u[g * C::DQ_ROWS + r]) * scale);
+          fence_proxy_async_smem();
+          named_bar_sync(3, 128);  // slot written
+          if (issuer) {
+            bulk_reduce_add_f32(tile + g * C::DQ_ROWS * D, sDQS + (slot % C::DQ_SLOTS) * C::DQ_SLOT_BYTES,
+                                C::DQ_SLOT_BYTES);
+            bulk_commit_group();
+          }
+        }
+      } else if (C::DQ_T) {
+        uint32_t u[128];
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tDQ_row + c * 32, *reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
         tc_fence_before();
@@ -510,6 +574,7 @@ __global__ void __launch_bounds__(512, 1)
       }
       ++it;
     }
+    if (C::DQ_BULK && issuer) bulk_wait_group0();  // every reduction complete before the CTA exits
     // -------------------------------------------------------------- epilogue: dK (times scale)
     if (ok) ok = warp_wait(bar_acc, 0, ab, lim, WAIT_BWD_EPILOGUE + 2);
     uint8_t* stage = smem + C::OFF_DO;  // dO ring stage 0, free once every MMA retired
