@@ -518,18 +518,22 @@ __global__ void __launch_bounds__(512, 1)
     for (int i = i_begin; i < p.nb; ++i) {
       if (!bwd_tile_active(p, i, j)) continue;
       ok = warp_wait(bar_dq, it & 1, ab, lim, WAIT_BWD_DQ + 1);
-      // the four warps must leave together: they meet at named barriers below
-      if (C::DQ_BULK) ok = named_bar_and(3, 128, ok);
-      if (!ok) break;
-      tc_fence_after();
       float* tile = p.dq_acc + ((size_t)bh * p.Np + (size_t)i * 128) * D;
       if (C::DQ_BULK) {
-        uint32_t u[128];  // dQ_i^T row `ln`: column q = query q of tile i
+        // Read dQ_i^T row `ln` (column q = query q of tile i) and release the TMEM columns
+        // before anything else: the next dP^T waits for them. When aborting (!ok) the values
+        // are not used; the columns stay allocated until every role has left.
+        uint32_t u[128];
+        tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tDQ_row + c * 32, *reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
+        for (int c = 0; c < 4; ++c) tmem_ld32_async(tDQ_row + c * 32, *reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_wait_ld_tied(*reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_dqfree);
+        if (lane == 0 && ok) mbar_arrive(bar_dqfree);
+        // the four warps leave together: they meet at named barriers below
+        if (!named_bar_and(3, 128, ok)) break;
         // Stage scale*dQ_i row-major ([query][head dim], lanes write 128 contiguous bytes) in
         // DQ_ROWS-query slots; one thread adds each slot to the fp32 accumulator with a bulk
         // reduction (performed in L2), keeping DQ_SLOTS - 1 of them in flight.
@@ -550,6 +554,8 @@ __global__ void __launch_bounds__(512, 1)
           }
         }
       } else if (C::DQ_T) {
+        if (!ok) break;
+        tc_fence_after();
         uint32_t u[128];
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tDQ_row + c * 32, *reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
@@ -561,6 +567,8 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int q = 0; q < 128; ++q, dst += D) red_add_f32(dst, __uint_as_float(u[q]) * scale);
       } else {
+        if (!ok) break;
+        tc_fence_after();
         uint32_t u[64];
         tmem_ld64(tDQ_row, u);
         tc_fence_before();
