@@ -38,6 +38,19 @@ bool encode_bhnd(CUtensorMap* map, const void* base, long long BH, int N, int D)
   return r == CUDA_SUCCESS;
 }
 
+// The fp32 dQ accumulator [BH*Np][D] as a 2-D tensor {D, BH*Np}; box 32 x 128 (one 128-byte
+// swizzled row per query), the unit of the backward's bulk reductions.
+bool encode_dq_acc(CUtensorMap* map, float* base, long long rows, int D) {
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 4};
+  cuuint32_t box[2] = {32, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 fa_status check_common(int B, int H, int N, int d, float scale) {
@@ -124,6 +137,7 @@ fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int
   if (!aligned16(o) || !aligned16(dO) || !aligned16(lse)) return FA_ERR_INVALID;
   fa_status st = check_common(B, H, N, d, scale);
   if (st != FA_OK) return st;
+  if (!(scale > 0.f)) return FA_ERR_UNSUPPORTED;  // the backward folds log2(scale) into P
   if (!workspace || !aligned16(workspace)) return FA_ERR_WORKSPACE;
   Workspace w = layout(workspace, B, H, N, d);
   if (workspace_bytes < w.bytes) return FA_ERR_WORKSPACE;
@@ -138,6 +152,7 @@ fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int
   p.N = N;
   p.Np = (N + 127) / 128 * 128;
   p.D = d;
+  p.log2_scale = log2f(scale);
   return from_cuda(fa::launch_bwd_pre(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -149,14 +164,17 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* d
     return FA_ERR_INVALID;
   fa_status st = check_common(B, H, N, d, scale);
   if (st != FA_OK) return st;
+  if (!(scale > 0.f)) return FA_ERR_UNSUPPORTED;  // the backward folds log2(scale) into P
+  if ((long long)B * H * ((N + 127) / 128 * 128) > 0x7fffffffll) return FA_ERR_UNSUPPORTED;  // TMA row coordinate
   if (!workspace || !aligned16(workspace)) return FA_ERR_WORKSPACE;
   Workspace w = layout(workspace, B, H, N, d);
   if (workspace_bytes < w.bytes) return FA_ERR_WORKSPACE;
   if (!get_encoder()) return FA_ERR_CUDA;
   const long long BH = (long long)B * H;
-  alignas(64) CUtensorMap tq, tk, tv, tdo, tdk, tdv;
+  alignas(64) CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdqa;
   if (!encode_bhnd(&tq, q, BH, N, d) || !encode_bhnd(&tk, k, BH, N, d) || !encode_bhnd(&tv, v, BH, N, d) ||
-      !encode_bhnd(&tdo, dO, BH, N, d) || !encode_bhnd(&tdk, dk, BH, N, d) || !encode_bhnd(&tdv, dv, BH, N, d))
+      !encode_bhnd(&tdo, dO, BH, N, d) || !encode_bhnd(&tdk, dk, BH, N, d) || !encode_bhnd(&tdv, dv, BH, N, d) ||
+      !encode_dq_acc(&tdqa, w.dq_acc, BH * ((N + 127) / 128 * 128), d))
     return FA_ERR_CUDA;
   fa::BwdParams p;
   p.delta = w.delta;
@@ -167,10 +185,11 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* d
   p.Np = (N + 127) / 128 * 128;
   p.nb = N / 128;
   p.causal = causal ? 1 : 0;
-  p.scale = scale;
+  p.inv_scale = 1.0f / scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
-  return from_cuda(fa::launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, p, (int)BH, static_cast<cudaStream_t>(stream)));
+  return from_cuda(
+      fa::launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, tdqa, p, (int)BH, static_cast<cudaStream_t>(stream)));
 }
 
 fa_status fa_bwd_dq_finish(void* dq, int B, int H, int N, int d, void* workspace, size_t workspace_bytes,
@@ -188,7 +207,7 @@ fa_status fa_bwd_dq_finish(void* dq, int B, int H, int N, int d, void* workspace
   p.N = N;
   p.Np = (N + 127) / 128 * 128;
   p.D = d;
-  p.scale = 1.0f;  // the scale is applied to dQ inside fa_bwd_main before accumulation
+  p.scale = 1.0f;  // the accumulated dQ already carries the scale (fa_bwd_main folds it into P)
   return from_cuda(fa::launch_dq_finish(p, static_cast<cudaStream_t>(stream)));
 }
 

@@ -14,22 +14,26 @@
 //      dK_j += scale dS_ij^T Q_i,  dQ_i += scale dS_ij K_j,  with D_i = rowsum(dO_i o O_i).
 //
 // sm_100a design (ours):
-//  * CTA = one 128-key tile j of one (b, h). K_j and V_j stay in shared memory; Q_i, dO_i (and
-//    the 128 values -LSE_i*log2e and -D_i of tile i) stream through an NS-deep ring.
-//  * Everything is computed transposed so on-chip results are directly MMA operands:
+//  * CTA = one 128-key tile j of one (b, h). K_j and V_j stay in shared memory; Q_i (with the
+//    128 values -LSE_i*log2e + log2(scale) and -D_i of tile i) streams through an NS-deep ring,
+//    dO_i through an NS_DO-deep one.
+//  * The softmax scale rides in the exponent: the recomputed probabilities are
+//    P' = exp2(S * scale*log2e - LSE*log2e + log2(scale)) = scale * P, so dS' = P' o (dP - D)
+//    = scale * dS already carries the factor dK and dQ need, and dV = (1/scale) sum P'^T dO is
+//    corrected once in its epilogue (this needs scale > 0; the host rejects other values).
+//  * Everything but dQ is computed transposed so on-chip results are directly MMA operands:
 //      S^T = K_j Q_i^T, dP^T = V_j dO_i^T            (TMEM, one key per TMEM lane)
-//      P^T = exp2(S^T * scale*log2e - LSE_i*log2e)     (bf16, written back over S^T in TMEM)
-//      dS^T = P^T o (dP^T - D_i)                      (bf16, 128B-swizzled shared memory)
-//      dV += P^T dO_i   (A = P^T from TMEM)
-//      dK += dS^T Q_i   (A = dS^T, K-major)
-//      dQ_i: d = 128: dQ_i^T = K_j^T dS_i^T (A = K_j MN-major, B = dS^T MN-major), so TMEM lane
-//            = head-dim index and a warp's fp32 adds into the accumulator hit 128 contiguous
-//            bytes (whole L2 sectors); d = 64: dQ_i = dS K_j (lane = query row).
+//      P'^T                                           (bf16, written back over S^T in TMEM)
+//      dS'^T = P'^T o (dP^T - D_i)                    (bf16, 128B-swizzled shared memory)
+//      dV += P'^T dO_i  (A = P'^T from TMEM)
+//      dK += dS'^T Q_i  (A = dS'^T, K-major)
+//      dQ_i = dS'_i K_j (A = dS'^T read MN-major, B = K_j MN-major; lane = query row)
 //  * Roles: warp 0 TMA; warp 1 MMA issuer (one thread; descriptors precomputed, so each MMA
 //    costs only an add); warps 4-7 and 8-11 compute P (P phase) then dS (dS phase) for query
 //    columns 0-63 and 64-127 respectively, thread = key row; warps 12-15 drain dQ from TMEM
-//    and add scale*dQ into the fp32 accumulator with red.global.add, then write dK (times
-//    scale); warps 4-11 write dV.
+//    into a 128B-swizzled staging ring and add it to the fp32 accumulator with bulk tensor
+//    reductions (one thread issues them; L2 performs the adds), then write dK; warps 4-11
+//    write dV.
 //  * MMA order per query tile i: dV_i as soon as P_i is in TMEM; S_{i+1} (the compute warps
 //    start the next P phase while the tensor core still works on tile i); dQ_i; dK_i (covers
 //    the dQ drain); dP_{i+1}.
@@ -37,6 +41,12 @@
 //    reuses the dP^T columns once dP^T has been read, d = 64 has its own [384,448).
 #include "kernels.h"
 #include "ptx.cuh"
+
+// Which of the 16 score pairs of each 32-score chunk of the P phase take 2^x on the FMA pipe
+// (ex2_poly2) instead of the special-function unit: bit i set = pair i emulated.
+#ifndef FA_BWD_EXP_EMU_MASK
+#define FA_BWD_EXP_EMU_MASK 0x0u
+#endif
 
 #ifndef FA_BWD_REGS_CTRL
 #define FA_BWD_REGS_CTRL 104
@@ -53,10 +63,9 @@ struct BwdCfg {
   // d = 128: dO is single-buffered to make room for the dQ staging buffer. dO_i is last read by
   // dV_i and next needed by dP_{i+1}, three MMA groups later, which covers the load.
   static constexpr int NS_DO = (D == 128) ? 1 : NS;
-  static constexpr bool DQ_BULK = (D == 128);       // dQ combined by bulk reductions from smem
-  static constexpr int DQ_ROWS = 16;                // queries per bulk reduction (8 KB at d = 128)
-  static constexpr int DQ_SLOTS = 4;                // staging slots in flight
-  static constexpr int DQ_SLOT_BYTES = DQ_ROWS * D * 4;
+  static constexpr int DQ_CHUNKS = D / 32;         // 32-column dQ chunks per query tile
+  static constexpr int DQ_SLOTS = 2;                // staging slots: one filling, one being reduced
+  static constexpr int DQ_SLOT_BYTES = 128 * 32 * 4;
   static constexpr int PANEL_BYTES = 128 * 128;
   static constexpr int PANELS = D / 64;
   static constexpr int TILE_BYTES = PANELS * PANEL_BYTES;
@@ -66,8 +75,8 @@ struct BwdCfg {
   static constexpr int OFF_DO = OFF_Q + NS * TILE_BYTES;
   static constexpr int OFF_DS = OFF_DO + NS_DO * TILE_BYTES;  // 128 keys x 128 queries bf16
   static constexpr int DS_BYTES = 2 * PANEL_BYTES;
-  static constexpr int OFF_DQS = OFF_DS + DS_BYTES;           // dQ staging [DQ_SLOTS][DQ_ROWS][D] fp32
-  static constexpr int DQS_BYTES = DQ_BULK ? DQ_SLOTS * DQ_SLOT_BYTES : 0;
+  static constexpr int OFF_DQS = OFF_DS + DS_BYTES;           // dQ staging [DQ_SLOTS][128][32] fp32
+  static constexpr int DQS_BYTES = DQ_SLOTS * DQ_SLOT_BYTES;
   static constexpr int OFF_LSE = OFF_DQS + DQS_BYTES;         // [NS][128] fp32: -LSE*log2e
   static constexpr int OFF_DEL = OFF_LSE + NS * 512;          // [NS][128] fp32: -D
   static constexpr int OFF_BAR = OFF_DEL + NS * 512;
@@ -76,8 +85,8 @@ struct BwdCfg {
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
-  static constexpr bool DQ_T = (D == 128);               // transposed dQ (lane = head dim)
-  static constexpr uint32_t T_DQ = DQ_T ? 128u : 384u;   // d = 128 aliases the dP^T columns
+  static constexpr bool DQ_ALIAS = (D == 128);           // dQ reuses the dP^T columns
+  static constexpr uint32_t T_DQ = DQ_ALIAS ? T_DP : 384u;
   // setmaxnreg split of the launch allocation (512 x 128, checked by the build script):
   // control warpgroup (TMA, MMA, 2 idle warps), two P/dS warpgroups, dQ-drain warpgroup.
   static constexpr int REGS_CTRL = FA_BWD_REGS_CTRL, REGS_PDS = FA_BWD_REGS_PDS, REGS_DQ = FA_BWD_REGS_DQ;
@@ -89,10 +98,6 @@ __device__ __forceinline__ bool bwd_tile_active(const BwdParams& p, int i, int j
   if (p.causal && i < j) return false;
   if (p.block_mask != nullptr && p.block_mask[i * p.nb + j] == 0) return false;
   return true;
-}
-
-__device__ __forceinline__ void red_add_f32(float* addr, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
 
 // Writes one accumulator row (D fp32 columns of TMEM lane `row`, times `mul`) as bf16 into a
@@ -124,7 +129,7 @@ __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmdQa, const BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int NS = C::NS, NS_DO = C::NS_DO;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -250,8 +255,7 @@ __global__ void __launch_bounds__(512, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);  // K/V (A) and Q/dO (B), K-major
       constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, 0, 1);   // dV, dK: B = dO / Q MN-major
-      constexpr uint32_t IDESC_Q = C::DQ_T ? idesc_bf16_f32(128, 128, 1, 1)  // dQ^T = K^T dS^T
-                                           : idesc_bf16_f32(128, D, 1, 1);   // dQ = dS K
+      constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, 1, 1);    // dQ = dS K: A = dS^T, B = K, MN-major
       constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
       const uint32_t tS = tmem + C::T_S, tDP = tmem + C::T_DP, tDV = tmem + C::T_DV, tDK = tmem + C::T_DK;
       const uint32_t tDQ = tmem + C::T_DQ;
@@ -329,7 +333,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         ok = mbar_wait_spin(bar_ds, it & 1, ab, lim, WAIT_BWD_MMA + 5);
         if (!ok) break;
-        if (!C::DQ_T && it > 0) {  // d = 64: the dQ columns must have been drained
+        if (!C::DQ_ALIAS && it > 0) {  // d = 64: the dQ columns must have been drained
           ok = mbar_wait_spin(bar_dqfree, (it - 1) & 1, ab, lim, WAIT_BWD_MMA + 6);
           if (!ok) break;
         }
@@ -338,10 +342,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // reduction over the 128 keys of tile j
           const uint64_t kdesc = dK_mn + (uint64_t)(kk * (2048 >> 4)), sdesc = dS_mn + (uint64_t)(kk * (2048 >> 4));
-          if (C::DQ_T)
-            umma_ss(tDQ, kdesc, sdesc, IDESC_Q, kk > 0 ? 1u : 0u);
-          else
-            umma_ss(tDQ, sdesc, kdesc, IDESC_Q, kk > 0 ? 1u : 0u);
+          umma_ss(tDQ, sdesc, kdesc, IDESC_Q, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar_dq);
         // dK += dS^T Q_i
@@ -354,7 +355,7 @@ __global__ void __launch_bounds__(512, 1)
         umma_commit(&bar_qe[s]);
         // dP^T_{i+1}
         if (has_next) {
-          if (C::DQ_T) {  // the dP^T columns hold dQ_i until the drain warps have read it
+          if (C::DQ_ALIAS) {  // the dP^T columns hold dQ_i until the drain warps have read it
             ok = mbar_wait_spin(bar_dqfree, it & 1, ab, lim, WAIT_BWD_MMA + 7);
             if (!ok) break;
           }
@@ -384,6 +385,8 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t lane_off = (wq * 32u) << 16;
     const uint32_t tS_row = tmem + lane_off + C::T_S + 64u * h, tDP_row = tmem + lane_off + C::T_DP + 64u * h;
     const uint64_t sl2_2 = f2_pack(p.scale_log2, p.scale_log2);
+    constexpr uint32_t EMU = FA_BWD_EXP_EMU_MASK;
+    const Ex2PolyConsts ek = ex2_poly_consts();
     bool ok = true;
     int it = 0;
     for (int i = i_begin; i < p.nb; ++i) {
@@ -417,10 +420,23 @@ __global__ void __launch_bounds__(512, 1)
                                        f2_pack(nl.x, nl.y));
             const uint64_t x23 = ffma2(f2_pack(__uint_as_float(su[2 * e + 2]), __uint_as_float(su[2 * e + 3])),
                                        sl2_2, f2_pack(nl.z, nl.w));
-            float x0, x1, x2, x3;
-            f2_unpack(x01, x0, x1);
-            f2_unpack(x23, x2, x3);
-            float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+            float p0, p1, p2, p3;
+            if ((EMU >> e) & 1u) {
+              f2_unpack(ex2_poly2(x01, ek), p0, p1);
+            } else {
+              float x0, x1;
+              f2_unpack(x01, x0, x1);
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            if ((EMU >> (e + 1)) & 1u) {
+              f2_unpack(ex2_poly2(x23, ek), p2, p3);
+            } else {
+              float x2, x3;
+              f2_unpack(x23, x2, x3);
+              p2 = ex2(x2);
+              p3 = ex2(x3);
+            }
             if (diag) {  // key kr is visible to query qoff+q iff kr <= qoff+q
               const int qq = qoff + q;
               if (qq < kr) p0 = 0.f;
@@ -493,7 +509,8 @@ __global__ void __launch_bounds__(512, 1)
     uint8_t* stage = smem + C::OFF_Q;  // Q ring stage 0 is free once every MMA retired
     if (ok && h < C::PANELS) {
       tc_fence_after();
-      stage_row_bf16<64>(tmem + lane_off + C::T_DV + 64u * h, smem_u32(stage + h * C::PANEL_BYTES), kr, 1.f, it == 0);
+      stage_row_bf16<64>(tmem + lane_off + C::T_DV + 64u * h, smem_u32(stage + h * C::PANEL_BYTES), kr, p.inv_scale,
+                         it == 0);
       fence_proxy_async_smem();
     }
     named_bar_sync(1, 256);
@@ -504,91 +521,68 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp >= 12) {
     // ------------------------------------------------------------------ dQ drain
+    // Thread = query row of dQ_i (TMEM lane). The tile goes back to memory in 32-column
+    // chunks: each chunk is staged as 128 rows of 128 bytes (the tensor map's 128-byte
+    // swizzle, so the 16-byte stores of a warp are conflict-free) and added to the fp32
+    // accumulator by one thread with a bulk tensor reduction performed in L2.
     reg_alloc<C::REGS_DQ>();
     const uint32_t wq = warp & 3;
-    const int ln = wq * 32 + lane;  // TMEM lane: head-dim index (d = 128) or query row (d = 64)
+    const int ln = wq * 32 + lane;
     const uint32_t lane_off = (wq * 32u) << 16;
     const uint32_t tDQ_row = tmem + lane_off + C::T_DQ;
-    const float scale = p.scale;
     const uint32_t sDQS = smem_u32(smem + C::OFF_DQS);
     const bool issuer = (wq == 0 && lane == 0);  // issues the bulk reductions of the warpgroup
+    if (issuer) tma_prefetch_desc(&tmdQa);
     bool ok = true;
     int it = 0;
-    uint32_t slot = 0;  // bulk reductions issued so far (staging slot = slot % DQ_SLOTS)
+    uint32_t nred = 0;  // bulk reductions issued so far (staging slot = nred % DQ_SLOTS)
     for (int i = i_begin; i < p.nb; ++i) {
       if (!bwd_tile_active(p, i, j)) continue;
       ok = warp_wait(bar_dq, it & 1, ab, lim, WAIT_BWD_DQ + 1);
-      float* tile = p.dq_acc + ((size_t)bh * p.Np + (size_t)i * 128) * D;
-      if (C::DQ_BULK) {
-        // Read dQ_i^T row `ln` (column q = query q of tile i) and release the TMEM columns
-        // before anything else: the next dP^T waits for them. When aborting (!ok) the values
-        // are not used; the columns stay allocated until every role has left.
-        uint32_t u[128];
-        tc_fence_after();
+      // Read the whole row and release the TMEM columns before anything else (at d = 128 the
+      // next dP^T is written there). When aborting (!ok) the values are not used; the columns
+      // stay allocated until every role has left.
+      uint32_t u[D];
+      tc_fence_after();
+      if constexpr (D == 128) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32_async(tDQ_row + c * 32, *reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_wait_ld_tied(*reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0 && ok) mbar_arrive(bar_dqfree);
-        // the four warps leave together: they meet at named barriers below
-        if (!named_bar_and(3, 128, ok)) break;
-        // Stage scale*dQ_i row-major ([query][head dim], lanes write 128 contiguous bytes) in
-        // DQ_ROWS-query slots; one thread adds each slot to the fp32 accumulator with a bulk
-        // reduction (performed in L2), keeping DQ_SLOTS - 1 of them in flight.
-#pragma unroll
-        for (int g = 0; g < 128 / C::DQ_ROWS; ++g, ++slot) {
-          if (issuer && slot >= C::DQ_SLOTS) bulk_wait_group_read<C::DQ_SLOTS - 1>();
-          named_bar_sync(3, 128);  // the slot's previous reduction has read it
-          const uint32_t sbuf = sDQS + (slot % C::DQ_SLOTS) * C::DQ_SLOT_BYTES + ln * 4;
-#pragma unroll
-          for (int r = 0; r < C::DQ_ROWS; ++r)
-            st_shared_f32(sbuf + r * (D * 4), __uint_as_float(u[g * C::DQ_ROWS + r]) * scale);
-          fence_proxy_async_smem();
-          named_bar_sync(3, 128);  // slot written
-          if (issuer) {
-            bulk_reduce_add_f32(tile + g * C::DQ_ROWS * D, sDQS + (slot % C::DQ_SLOTS) * C::DQ_SLOT_BYTES,
-                                C::DQ_SLOT_BYTES);
-            bulk_commit_group();
-          }
-        }
-      } else if (C::DQ_T) {
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t u[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tDQ_row + c * 32, *reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_dqfree);
-        // lanes of a warp hold 32 consecutive head-dim entries: each add covers 128 contiguous bytes
-        float* dst = tile + ln;
-#pragma unroll
-        for (int q = 0; q < 128; ++q, dst += D) red_add_f32(dst, __uint_as_float(u[q]) * scale);
       } else {
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t u[64];
         tmem_ld64(tDQ_row, u);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_dqfree);
-        float* dst = tile + (size_t)ln * D;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0 && ok) mbar_arrive(bar_dqfree);
+      // the four warps leave together: they meet at named barriers below
+      if (!named_bar_and(3, 128, ok)) break;
+      const int row0 = bh * p.Np + i * 128;
 #pragma unroll
-        for (int e = 0; e < 64; e += 4)
-          red_add_v4(dst + e, __uint_as_float(u[e]) * scale, __uint_as_float(u[e + 1]) * scale,
-                     __uint_as_float(u[e + 2]) * scale, __uint_as_float(u[e + 3]) * scale);
+      for (int c = 0; c < C::DQ_CHUNKS; ++c, ++nred) {
+        if (issuer && nred >= C::DQ_SLOTS) bulk_wait_group_read<C::DQ_SLOTS - 1>();
+        named_bar_sync(3, 128);  // the slot's previous reduction has read it
+        const uint32_t slot = sDQS + (nred % C::DQ_SLOTS) * C::DQ_SLOT_BYTES;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // 16-byte chunk k of row ln: columns 32c + 4k .. +3
+          st_shared_v4(slot + sw128_offset(ln, k), u[32 * c + 4 * k], u[32 * c + 4 * k + 1], u[32 * c + 4 * k + 2],
+                       u[32 * c + 4 * k + 3]);
+        fence_proxy_async_smem();
+        named_bar_sync(3, 128);  // slot written
+        if (issuer) {
+          tma_reduce_add_2d(&tmdQa, slot, 32 * c, row0);
+          bulk_commit_group();
+        }
       }
       ++it;
     }
-    if (C::DQ_BULK && issuer) bulk_wait_group0();  // every reduction complete before the CTA exits
-    // -------------------------------------------------------------- epilogue: dK (times scale)
+    if (issuer) bulk_wait_group0();  // every reduction complete before the CTA exits
+    // -------------------------------------------------------------- epilogue: dK (dS carries the scale)
     if (ok) ok = warp_wait(bar_acc, 0, ab, lim, WAIT_BWD_EPILOGUE + 2);
     uint8_t* stage = smem + C::OFF_DO;  // dO ring stage 0, free once every MMA retired
     if (ok) {
       tc_fence_after();
-      stage_row_bf16<D>(tmem + lane_off + C::T_DK, smem_u32(stage), ln, scale, it == 0);
+      stage_row_bf16<D>(tmem + lane_off + C::T_DK, smem_u32(stage), ln, 1.f, it == 0);
       fence_proxy_async_smem();
     }
     named_bar_sync(2, 128);
@@ -611,20 +605,20 @@ __global__ void __launch_bounds__(512, 1)
 template <int D>
 static cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
-                                const BwdParams& p, int BH, cudaStream_t stream) {
+                                const CUtensorMap& tdqa, const BwdParams& p, int BH, cudaStream_t stream) {
   using C = BwdCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(fa_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(p.nb, BH);
-  fa_bwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdk, tdv, p);
+  fa_bwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdk, tdv, tdqa, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
-                            const BwdParams& p, int BH, cudaStream_t stream) {
-  if (D == 64) return launch_bwd_t<64>(tq, tk, tv, tdo, tdk, tdv, p, BH, stream);
-  return launch_bwd_t<128>(tq, tk, tv, tdo, tdk, tdv, p, BH, stream);
+                            const CUtensorMap& tdqa, const BwdParams& p, int BH, cudaStream_t stream) {
+  if (D == 64) return launch_bwd_t<64>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+  return launch_bwd_t<128>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
 }
 
 }  // namespace fa

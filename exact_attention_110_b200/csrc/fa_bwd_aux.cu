@@ -3,8 +3,9 @@
 //  * bwd_pre: D_i = sum_t dO_it * O_it for every query row (the row sums the softmax
 //    Jacobian produces: sum_j P_ij dP_ij = dO_i . O_i; FlashAttention V1 lecture summary,
 //    spark.aweffr.cn, §4.1) and LSE_i * log2(e) for the exp2-domain recomputation of P, both
-//    stored negated (the backward's inner loops then need only fused multiply-adds), and a
-//    zero-fill of the fp32 dQ accumulator that fa_bwd_main adds into.
+//    stored negated (the backward's inner loops then need only fused multiply-adds; the
+//    exponent offset also carries log2(scale), so the recomputed P comes out as scale * P),
+//    and a zero-fill of the fp32 dQ accumulator that fa_bwd_main adds into.
 //  * dq_finish: dq = bf16(dq_acc), the combine step after every key block has added its dQ
 //    share ("FlashAttention-2 的前世今生" overview, jishu.shishitao.com, §主要操作, backward:
 //    dQ is the one quantity shared across column blocks and is combined with atomic adds).
@@ -46,7 +47,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdPreParams p) {
       const long long bh = row / p.N, i = row % p.N;
       const long long out = bh * p.Np + i;
       p.delta[out] = -acc;                               // stored negated: the backward adds it
-      p.lse2[out] = -p.lse[row] * 1.4426950408889634f;  // -LSE in log2 units
+      p.lse2[out] = p.log2_scale - p.lse[row] * 1.4426950408889634f;  // log2(scale) - LSE*log2(e)
     }
   }
   // Zero the dQ accumulator (float4 stores).

@@ -38,20 +38,21 @@ struct BwdPreParams {
   const uint16_t* dout;  // bf16 [BH][N][D]
   const float* lse;      // [BH][N]
   float* delta;          // [BH][Np]  = -D = -rowsum(dO o O)
-  float* lse2;           // [BH][Np]  = -LSE * log2(e)
+  float* lse2;           // [BH][Np]  = -LSE * log2(e) + log2(scale)
   float* dq_acc;         // [BH][Np][D], zeroed here
   long long rows;        // BH * N
   int N, Np, D;
+  float log2_scale;      // log2(scale), scale > 0: folds the softmax scale into P (see fa_bwd.cu)
 };
 
 struct BwdParams {
   const float* delta;    // [BH][Np]  -D
-  const float* lse2;     // [BH][Np]  -LSE * log2(e)
+  const float* lse2;     // [BH][Np]  -LSE * log2(e) + log2(scale)
   float* dq_acc;         // [BH][Np][D]
   const uint8_t* block_mask;
   int N, Np, nb;
   int causal;
-  float scale;           // scale (for dK)
+  float inv_scale;       // 1 / scale (dV epilogue: P carries the scale)
   float scale_log2;      // scale * log2(e)
   unsigned long long timeout_ns;
 };
@@ -70,7 +71,7 @@ cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, cons
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
-                            const BwdParams& p, int BH, cudaStream_t stream);
+                            const CUtensorMap& tdqa, const BwdParams& p, int BH, cudaStream_t stream);
 cudaError_t launch_dq_finish(const DqFinishParams& p, cudaStream_t stream);
 
 }  // namespace fa

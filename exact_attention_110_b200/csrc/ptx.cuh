@@ -196,12 +196,13 @@ template <int N>
 __device__ __forceinline__ void bulk_wait_group_read() {
   asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
-// Untiled bulk reduction shared -> global: dst[k] += src[k] for bytes/4 fp32 values, performed
-// in L2. Both addresses 16-byte aligned, bytes % 16 == 0; completion is tracked by bulk groups.
-__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src, uint32_t bytes) {
-  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-                   reinterpret_cast<uint64_t>(dst)),
-               "r"(src), "r"(bytes)
+// 2-D tiled bulk reduction shared -> global: the box at (x, y) of the map's tensor += the
+// staged tile, performed in L2 (fp32 add). x * element size must be a multiple of 16 bytes and
+// neither coordinate may be negative; completion is tracked by bulk groups.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
                : "memory");
 }
 
@@ -482,11 +483,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
-// Fire-and-forget vector fp32 add into global memory (sm_90+).
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
 
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128-byte-swizzled panel
 // of 128-byte rows (the layout TMA writes with CU_TENSOR_MAP_SWIZZLE_128B and the tensor

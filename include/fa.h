@@ -79,6 +79,8 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
  *   out: dq, dk, dv      bf16 [B][H][N][d]
  *   workspace: device buffer of at least fa_bwd_workspace_bytes(B,H,N,d) bytes; its
  *              contents on entry are ignored and on exit unspecified.
+ *   scale: as passed to fa_fwd, and > 0: the kernels fold log2(scale) into the recomputed
+ *          probabilities (FA_ERR_UNSUPPORTED otherwise).
  * Equivalent to fa_bwd_preprocess + fa_bwd_main + fa_bwd_dq_finish on the same workspace.
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
@@ -93,7 +95,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  * fa_bwd_main: per key tile, recompute S and P, accumulate dK and dV on chip, write dk and
  *   dv (bf16), and add each tile's dQ contribution into the fp32 accumulator.
  * fa_bwd_dq_finish: dq = bf16(accumulator).
- * They must be called in this order on one stream with the same workspace and sizes.
+ * They must be called in this order on one stream with the same workspace, sizes and scale.
  */
 fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int N,
                             int d, float scale, void* workspace, size_t workspace_bytes,

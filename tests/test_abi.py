@@ -78,6 +78,17 @@ def test_workspace_size_and_checks(lib):
     assert lib.fa_bwd_main(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 48, 0.1, 0, None, FAKE, need, None) == 2
 
 
+@pytest.mark.parametrize("scale", [0.0, -0.125])
+def test_backward_needs_positive_scale(lib, scale):
+    # The backward folds log2(scale) into the recomputed probabilities: scale <= 0 is refused
+    # up front (the forward accepts any finite scale).
+    need = lib.fa_bwd_workspace_bytes(1, 1, 128, 64)
+    assert lib.fa_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, scale, 0, None,
+                      FAKE, need, None) == 2
+    assert lib.fa_bwd_preprocess(FAKE, FAKE, FAKE, 1, 1, 128, 64, scale, FAKE, need, None) == 2
+    assert lib.fa_bwd_main(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, scale, 0, None, FAKE, need, None) == 2
+
+
 def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     import exact_attention_110_b200 as fa
     monkeypatch.setattr(fa, "LIB_PATH", tmp_path / "missing.so")
