@@ -59,7 +59,7 @@ struct FwdCfg {
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + NS * TILE_BYTES;
-  static constexpr int NBAR = 2 + 4 * NS + 2 + 2 + 2 + 1;
+  static constexpr int NBAR = 2 + 4 * NS + 2 + 4 + 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int TMEM_COLS = 512;
@@ -81,10 +81,12 @@ __device__ __forceinline__ bool fwd_tile_active(const FwdParams& p, int qb, int 
 // columns already read. Pairs whose bit is set in EMU_MASK (within each chunk of 16 pairs)
 // use the FMA-pipe polynomial, the rest the special-function unit; EMU = false forces the
 // special-function unit everywhere (masked tiles need exact zeros for -inf scores).
-// Returns the row sum of p.
+// After the first two chunks (keys 0-63) the warp arrives on `half0`, so the tensor core can
+// start O += P V on those keys while the second half is computed; the caller signals the
+// second half. Returns the row sum of p.
 template <bool EMU, uint32_t EMU_MASK>
 __device__ __forceinline__ float softmax_exp_store(const uint32_t (&su)[128], uint64_t sl2_2, uint64_t mneg_2,
-                                                   uint32_t tS_row, const Ex2PolyConsts& K) {
+                                                   uint32_t tS_row, const Ex2PolyConsts& K, uint64_t* half0) {
   uint64_t ls2[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) ls2[k] = 0ull;  // two +0.0f lanes
@@ -109,6 +111,12 @@ __device__ __forceinline__ float softmax_exp_store(const uint32_t (&su)[128], ui
       pk[i] = pack_bf16(p0, p1);
     }
     tmem_st16(tS_row + c * 16, pk);
+    if (c == 1) {
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane_id() == 0) mbar_arrive(half0);
+    }
   }
   const uint64_t t2 = fadd2(fadd2(ls2[0], ls2[1]), fadd2(ls2[2], ls2[3]));
   float a, b;
@@ -138,8 +146,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* bar_vf = bar_ke + NS;    // [NS] V stage full
   uint64_t* bar_ve = bar_vf + NS;    // [NS] V stage free
   uint64_t* bar_s = bar_ve + NS;     // [2]  S_t ready in TMEM
-  uint64_t* bar_p = bar_s + 2;       // [2]  P_t written (and O_t rescaled)
-  uint64_t* bar_o = bar_p + 2;       // [2]  all MMAs of tile t complete
+  uint64_t* bar_p = bar_s + 2;       // [2][2] P_t keys 0-63 / 64-127 written (O_t rescaled before)
+  uint64_t* bar_o = bar_p + 4;       // [2]  all MMAs of tile t complete
   uint64_t* bar_done = bar_o + 2;    // [1]  every MMA of the CTA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   AbortState* ab = reinterpret_cast<AbortState*>(smem + C::OFF_MISC + 4);
@@ -161,7 +169,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar_s[t], 1);
-      mbar_init(&bar_p[t], 4);  // one arrive per softmax warp
+      mbar_init(&bar_p[2 * t], 4);  // one arrive per softmax warp
+      mbar_init(&bar_p[2 * t + 1], 4);
       mbar_init(&bar_o[t], 1);
     }
     mbar_init(bar_done, 1);
@@ -269,16 +278,20 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t dv_prev = dv_base + (uint64_t)((prev_s < 0 ? 0 : prev_s) * TILE16);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (prev_act[t]) {  // O_t += P_t V_{previous}
-            ok = mbar_wait_spin(&bar_p[t], p_phase[t], ab, lim, WAIT_FWD_MMA + 4);
-            if (!ok) break;
-            p_phase[t] ^= 1u;
-            tc_fence_after();
+          if (prev_act[t]) {  // O_t += P_t V_{previous}, 16 keys per MMA, in two halves of P
             const uint32_t acc0 = o_started[t] ? 1u : 0u;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per MMA
-              umma_ts(tmem + 256u + t * D, tmem + t * 128u + kk * 8, dv_prev + (uint64_t)(kk * (2048 >> 4)), IDESC_O,
-                      kk > 0 ? 1u : acc0);
+            for (int hf = 0; hf < 2; ++hf) {
+              ok = mbar_wait_spin(&bar_p[2 * t + hf], p_phase[t], ab, lim, WAIT_FWD_MMA + 4);
+              if (!ok) break;
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
+                umma_ts(tmem + 256u + t * D, tmem + t * 128u + kk * 8, dv_prev + (uint64_t)(kk * (2048 >> 4)),
+                        IDESC_O, kk > 0 ? 1u : acc0);
+            }
+            if (!ok) break;
+            p_phase[t] ^= 1u;
             o_started[t] = true;
           }
           if (act0 && t == 0 || act1 && t == 1) {  // S_t = Q_t K_j^T
@@ -305,15 +318,20 @@ __global__ void __launch_bounds__(384, 1)
       for (int t = 0; t < 2; ++t) {  // last PV of each tile
         if (ok && prev_act[t]) {
           ok = mbar_wait_spin(&bar_vf[prev_s], prev_ph, ab, lim, WAIT_FWD_MMA + 5);
-          if (ok) ok = mbar_wait_spin(&bar_p[t], p_phase[t], ab, lim, WAIT_FWD_MMA + 6);
+          const uint32_t acc0 = o_started[t] ? 1u : 0u;
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            if (ok) ok = mbar_wait_spin(&bar_p[2 * t + hf], p_phase[t], ab, lim, WAIT_FWD_MMA + 6);
+            if (ok) {
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
+                umma_ts(tmem + 256u + t * D, tmem + t * 128u + kk * 8, dv_last + (uint64_t)(kk * (2048 >> 4)),
+                        IDESC_O, kk > 0 ? 1u : acc0);
+            }
+          }
           if (ok) {
             p_phase[t] ^= 1u;
-            tc_fence_after();
-            const uint32_t acc0 = o_started[t] ? 1u : 0u;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              umma_ts(tmem + 256u + t * D, tmem + t * 128u + kk * 8, dv_last + (uint64_t)(kk * (2048 >> 4)), IDESC_O,
-                      kk > 0 ? 1u : acc0);
             o_started[t] = true;
           }
         }
@@ -390,13 +408,13 @@ __global__ void __launch_bounds__(384, 1)
         const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
         const uint64_t sl2_2 = f2_pack(sl2, sl2), mneg_2 = f2_pack(mneg, mneg);
         if (p.causal && j == qb)
-          l += softmax_exp_store<false, 0u>(su, sl2_2, mneg_2, tS_row, ek);
+          l += softmax_exp_store<false, 0u>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[2 * t]);
         else
-          l += softmax_exp_store<true, C::EXP_EMU_MASK>(su, sl2_2, mneg_2, tS_row, ek);
+          l += softmax_exp_store<true, C::EXP_EMU_MASK>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[2 * t]);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_p[t]);
+        if (lane == 0) mbar_arrive(&bar_p[2 * t + 1]);
         o_started = true;
       }
 
