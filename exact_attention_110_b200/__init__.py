@@ -8,7 +8,7 @@ the library is missing, every call raises -- there is no fallback implementation
     o, lse = forward(q, k, v, causal=False, block_mask=None, scale=None)
     dq, dk, dv = backward(q, k, v, o, do, lse, causal=False, block_mask=None, scale=None)
 
-q, k, v, o, do: bf16 CUDA tensors [B, H, N, d], contiguous, d in {64, 128}, N % 128 == 0.
+q, k, v, o, do: bf16 CUDA tensors [B, H, N, d], contiguous, d in {64, 128}, any N >= 1.
 lse: fp32 [B, H, N]. block_mask: uint8 CUDA tensor [ceil(N/128), ceil(N/128)] or None.
 """
 from __future__ import annotations

@@ -56,7 +56,6 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 fa_status check_common(int B, int H, int N, int d, float scale) {
   if (B <= 0 || H <= 0 || N <= 0 || !isfinite(scale)) return FA_ERR_INVALID;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (N % 128 != 0) return FA_ERR_UNSUPPORTED;
   const long long BH = (long long)B * H;
   if (BH > 65535) return FA_ERR_UNSUPPORTED;               // grid.y limit
   if ((long long)N * d > (1ll << 31) / 2) return FA_ERR_UNSUPPORTED;  // per-head elements
@@ -119,7 +118,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.lse = lse;
   p.block_mask = block_mask;
   p.N = N;
-  p.nb = N / 128;
+  p.nb = (N + 127) / 128;  // the last tile may be partial: TMA zero-fills rows >= N
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
@@ -183,7 +182,7 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* d
   p.block_mask = block_mask;
   p.N = N;
   p.Np = (N + 127) / 128 * 128;
-  p.nb = N / 128;
+  p.nb = (N + 127) / 128;
   p.causal = causal ? 1 : 0;
   p.inv_scale = 1.0f / scale;
   p.scale_log2 = scale * 1.4426950408889634f;

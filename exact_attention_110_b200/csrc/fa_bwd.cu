@@ -395,6 +395,9 @@ __global__ void __launch_bounds__(512, 1)
       const float* nlse2 = reinterpret_cast<const float*>(smem + C::OFF_LSE + s * 512) + 64 * h;
       const float* ndel = reinterpret_cast<const float*>(smem + C::OFF_DEL + s * 512) + 64 * h;
       const bool diag = p.causal && i == j;
+      // Keys of a partial last tile beyond N (zero rows from TMA) take no part: P = 0 there, so
+      // nothing non-finite can reach dQ through them.
+      const bool kpad = 128 * j + kr >= p.N;
       const int qoff = 64 * h;  // query index of column 0 of this group
 
       // ---- P phase: P^T = exp2(S^T * scale*log2e - LSE*log2e), back into TMEM as bf16
@@ -444,6 +447,7 @@ __global__ void __launch_bounds__(512, 1)
               if (qq + 2 < kr) p2 = 0.f;
               if (qq + 3 < kr) p3 = 0.f;
             }
+            if (kpad) p0 = p1 = p2 = p3 = 0.f;
             pf[q] = p0;
             pf[q + 1] = p1;
             pf[q + 2] = p2;

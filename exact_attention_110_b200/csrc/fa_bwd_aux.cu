@@ -50,6 +50,13 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdPreParams p) {
       p.lse2[out] = p.log2_scale - p.lse[row] * 1.4426950408889634f;  // log2(scale) - LSE*log2(e)
     }
   }
+  // Rows of a partial last query tile beyond N: -inf exponent offset (P = 0 there) and D = 0.
+  const long long BH = p.rows / p.N, pad = p.Np - p.N;
+  for (long long e = tid; e < BH * pad; e += nthreads) {
+    const long long out = (e / pad) * p.Np + p.N + e % pad;
+    p.delta[out] = 0.f;
+    p.lse2[out] = -INFINITY;
+  }
   // Zero the dQ accumulator (float4 stores).
   const long long nvec = (p.rows / p.N) * (long long)p.Np * D / 4;
   float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);

@@ -372,10 +372,14 @@ __global__ void __launch_bounds__(384, 1)
 
         uint32_t su[128];  // this row's 128 scores (fp32 bits)
         tmem_ld128(tS_row, su);
-        if (p.causal && j == qb) {  // diagonal tile: key 128j+c is visible to row 128qb+r iff c <= r
+        // Elementwise mask: on the causal diagonal key 128j+c is visible to row 128qb+r iff
+        // c <= r; in a partial last key tile keys 128j+c >= N do not exist (TMA filled zeros).
+        const bool masked = (p.causal && j == qb) || (128 * j + 128 > p.N);
+        if (masked) {
+          const int lim = min((p.causal && j == qb) ? r + 1 : 128, p.N - 128 * j);
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            if (c > r) su[c] = 0xff800000u;  // -inf
+            if (c >= lim) su[c] = 0xff800000u;  // -inf
         }
         // Row max: 8 independent chains of three-input max, then a short tree.
         float mc[8];
@@ -407,7 +411,7 @@ __global__ void __launch_bounds__(384, 1)
         l *= alpha;
         const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
         const uint64_t sl2_2 = f2_pack(sl2, sl2), mneg_2 = f2_pack(mneg, mneg);
-        if (p.causal && j == qb)
+        if (masked)
           l += softmax_exp_store<false, 0u>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[2 * t]);
         else
           l += softmax_exp_store<true, C::EXP_EMU_MASK>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[2 * t]);
@@ -447,7 +451,8 @@ __global__ void __launch_bounds__(384, 1)
         }
         fence_proxy_async_smem();
         const int row = qb * 128 + r;
-        p.lse[(size_t)bh * p.N + row] = (l > 0.f) ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (row < p.N)  // rows of a partial last tile beyond N are not stored (the O store clips them)
+          p.lse[(size_t)bh * p.N + row] = (l > 0.f) ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       }
       // Every thread of the warpgroup reaches this barrier (tvalid is uniform per warpgroup).
       named_bar_sync(1 + t, 128);

@@ -27,8 +27,9 @@
  *  - All pointers are device memory owned by the caller. The library allocates no device
  *    memory apart from one static device status word and the fixed scratch array that
  *    fa_bwd_noalloc uses.
- *  - Every pointer must be 16-byte aligned. d must be 64 or 128. N must be a positive
- *    multiple of 128 (other N: FA_ERR_UNSUPPORTED).
+ *  - Every pointer must be 16-byte aligned. d must be 64 or 128. N is any positive length;
+ *    a partial last 128-row tile is handled inside the kernels (rows and keys beyond N take no
+ *    part and are never written).
  *  - stream is a cudaStream_t (NULL = legacy default stream). All calls are asynchronous
  *    on it; argument errors are reported synchronously, before anything is enqueued.
  *  - Not re-entrant on the same output buffers; distinct calls on distinct buffers may run
@@ -47,7 +48,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID = 1,     /* null/misaligned pointer, non-positive size, non-finite scale */
-  FA_ERR_UNSUPPORTED = 2, /* valid but not implemented: d not in {64,128}, N % 128 != 0 */
+  FA_ERR_UNSUPPORTED = 2, /* valid but not implemented: d not in {64,128}; backward scale <= 0 */
   FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call or a kernel launch failed */
   FA_ERR_TIMEOUT = 4,     /* a device-side bounded wait gave up (see fa_last_device_status) */
   FA_ERR_WORKSPACE = 5    /* workspace pointer null or smaller than fa_bwd_workspace_bytes */

@@ -53,7 +53,7 @@ def test_fwd_argument_checks(lib):
     assert fwd(lib, scale=math.nan) == 1 and fwd(lib, scale=math.inf) == 1
     assert fwd(lib, d=96) == 2                   # unsupported head dim
     assert fwd(lib, d=256) == 2
-    assert fwd(lib, N=100) == 2                  # N not a multiple of 128
+    assert fwd(lib, N=0) == 1                    # empty sequence -> INVALID
 
 
 def test_workspace_size_and_checks(lib):
@@ -62,7 +62,9 @@ def test_workspace_size_and_checks(lib):
     vec = (B * H * N * 4 + 255) // 256 * 256
     acc = (B * H * N * d * 4 + 255) // 256 * 256
     assert lib.fa_bwd_workspace_bytes(B, H, N, d) == 2 * vec + acc
-    assert lib.fa_bwd_workspace_bytes(1, 1, 100, 64) == 0
+    # any N: the vectors and the accumulator are padded to whole 128-row tiles
+    assert lib.fa_bwd_workspace_bytes(1, 1, 100, 64) == 2 * 512 + 128 * 64 * 4
+    assert lib.fa_bwd_workspace_bytes(1, 1, 0, 64) == 0
     assert lib.fa_bwd_workspace_bytes(1, 1, 128, 80) == 0
     need = lib.fa_bwd_workspace_bytes(1, 1, 128, 64)
     st = lib.fa_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0, None,

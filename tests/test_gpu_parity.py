@@ -35,7 +35,7 @@ def run_bwd(fa, gpu, o, lse, causal, mask_t, scale):
 
 
 def mask_for(kind, N, seed=synth.BASE_SEED):
-    nb = N // 128
+    nb = (N + 127) // 128
     if kind is None:
         return None
     if kind == "bernoulli":
@@ -57,6 +57,14 @@ SMALL = [
     (1, 2, 512, 64, False, "bernoulli"),
     (1, 1, 768, 128, True, "bernoulli"),
     (1, 1, 512, 64, False, "diag"),
+    # ragged sequence lengths: a partial last tile of queries and keys
+    (1, 1, 1, 64, False, None),        # a single query and key
+    (1, 2, 77, 64, True, None),        # one partial tile
+    (2, 1, 130, 64, False, "bernoulli"),
+    (1, 2, 200, 128, False, None),
+    (1, 1, 333, 128, True, None),
+    (1, 1, 641, 64, True, "bernoulli"),
+    (1, 1, 1000, 128, False, None),
 ]
 
 
