@@ -7,7 +7,7 @@ N=4096 point (16k tokens, hidden 2048 -> B=4, H=16, d=128), non-causal, bf16 N(0
 inputs from the seeded generator. Prints ONE JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--seqlen N] [--headdim d]
-                    [--causal] [--block-sparse] [--impl reference] [--sweep]
+                    [--causal] [--block-sparse] [--dtype bf16|f16] [--impl reference] [--sweep]
 
 Metric: fwd+bwd TFLOPS with FLOPs counted as 4*B*H*N^2*d for the forward (halved for causal,
 scaled by block density for block-sparse) and 2.5x that for the backward.
@@ -151,7 +151,7 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- CPU oracle arm
-def oracle_sample(wl, nheads: int, seed: int):
+def oracle_sample(wl, nheads: int, seed: int, dtype: str = "bf16"):
     """Times the fp64 oracle (fwd + bwd) on `nheads` whole heads of the workload."""
     import numpy as np
     import oracle
@@ -159,8 +159,8 @@ def oracle_sample(wl, nheads: int, seed: int):
     B, H, N, d = wl["B"], wl["H"], wl["N"], wl["d"]
     mask = synth.block_mask_for(N) if wl["block_sparse"] else None
     n = nheads * N * d
-    q, k, v, do = (synth.bf16_bits_to_f32(synth.normal_bf16(seed + i, n)).astype(np.float64).reshape(1, nheads, N, d)
-                   for i in range(4))
+    q, k, v, do = (synth.bits_to_f32(synth.normal_bits(seed + i, n, dtype), dtype).astype(np.float64)
+                   .reshape(1, nheads, N, d) for i in range(4))
     scale = 1.0 / math.sqrt(d)
     t0 = time.perf_counter()
     oracle.attention_fwd(q, k, v, scale, causal=wl["causal"], mask=mask)
@@ -181,10 +181,10 @@ def run_reference(args, wl, rank, world):
         return 0
     nh = heads_for_seconds(wl, 2.0)
     for _ in range(args.warmup):
-        oracle_sample(wl, nh, 1000)
+        oracle_sample(wl, nh, 1000, args.dtype)
     tot_f, tot_t, cores = 0.0, 0.0, 1
     for s in range(args.steps):
-        f, t, cores = oracle_sample(wl, nh, 2000 + 10 * s)
+        f, t, cores = oracle_sample(wl, nh, 2000 + 10 * s, args.dtype)
         tot_f += f
         tot_t += t
     value = tot_f / tot_t / 1e12
@@ -203,11 +203,11 @@ def run_reference(args, wl, rank, world):
 
 # ----------------------------------------------------------------------------- GPU arm
 @functools.lru_cache(maxsize=4)
-def _stream(seed: int, n: int):
-    """Seeded N(0,1) bf16 bits (same bytes as synth.attention_inputs); every sweep point has
-    the same element count, so the streams are generated once."""
+def _stream(seed: int, n: int, dtype: str = "bf16"):
+    """Seeded N(0,1) bf16 (or fp16) bits (same bytes as synth.attention_inputs); every sweep
+    point has the same element count, so the streams are generated once."""
     import synth
-    return synth.normal_bf16(seed, n)
+    return synth.normal_bits(seed, n, dtype)
 
 
 def run_gpu(args, wl, rank, world, local_rank, dist_on):
@@ -223,7 +223,8 @@ def run_gpu(args, wl, rank, world, local_rank, dist_on):
     shape = (B, H, N, d)
     seed = synth.BASE_SEED + 97 * rank
     offs = (synth.SEED_Q, synth.SEED_K, synth.SEED_V, synth.SEED_DO)
-    q, k, v, do = (synth.to_torch_bf16(_stream(seed + o, B * H * N * d).reshape(B, H, N, d), dev) for o in offs)
+    q, k, v, do = (synth.to_torch(_stream(seed + o, B * H * N * d, args.dtype).reshape(B, H, N, d), args.dtype, dev)
+                   for o in offs)
     mask_np = synth.block_mask_for(N) if wl["block_sparse"] else None
     mask = None if mask_np is None else torch.from_numpy(mask_np).to(dev)
     density = float(mask_np.mean()) if mask_np is not None else 1.0
@@ -283,7 +284,7 @@ def run_gpu(args, wl, rank, world, local_rank, dist_on):
     e2e = None
     if not args.no_e2e:
         hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
-        ho, hdq, hdk, hdv = (torch.empty(shape, dtype=torch.bfloat16).pin_memory() for _ in range(4))
+        ho, hdq, hdk, hdv = (torch.empty(shape, dtype=q.dtype).pin_memory() for _ in range(4))
         hl = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
 
         def e2e_step():
@@ -315,10 +316,12 @@ def run_gpu(args, wl, rank, world, local_rank, dist_on):
     # ---- roofline of the dominant kernel (bwd main: 5 of the 7 matmuls of a step)
     main_flops = 2.5 * f_fwd
     achieved = main_flops / (main_ms * 1e-3) / 1e12
-    traffic = recorded_traffic(f"bwd_main N={N} d={d} causal={int(causal)} bs={int(wl['block_sparse'])}")
+    traffic = recorded_traffic(f"bwd_main N={N} d={d} causal={int(causal)} bs={int(wl['block_sparse'])}"
+                               + ("" if args.dtype == "bf16" else f" {args.dtype}"))
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"], "traffic": traffic, "kernel": "fa_bwd_kernel",
-                "peak_kind": f"bf16 dense burst ({peaks['source']})",
+                "peak_kind": f"bf16 dense burst ({peaks['source']})" + (
+                    "; fp16 has the same nominal dense rate (ratio 1)" if args.dtype == "f16" else ""),
                 "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]}
 
     kernels = {
@@ -331,7 +334,7 @@ def run_gpu(args, wl, rank, world, local_rank, dist_on):
     bwd_ms = pre_ms + main_ms + fin_ms
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": args.dtype,
         "data": "synthetic",
         "config": {"workload": wl["name"], "B": B, "H": H, "N": N, "d": d, "causal": causal,
                    "block_density": density, "global_batch_heads": world * B * H,
@@ -350,7 +353,7 @@ def run_gpu(args, wl, rank, world, local_rank, dist_on):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         nh = heads_for_seconds(wl, 12.0)
-        f, t, cores = oracle_sample(wl, nh, 3000)
+        f, t, cores = oracle_sample(wl, nh, 3000, args.dtype)
         line["cpu_baseline"] = {"value": f / t / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": f"{nh} whole head(s) of {N}x{d} (fwd+bwd, fp64) of {B * H} heads; "
                                           f"{t:.1f} s"}
@@ -372,6 +375,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="one JSON line per sweep point (N x d x causal)")
+    ap.add_argument("--dtype", choices=["bf16", "f16"], default="bf16",
+                    help="element type of q, k, v, o, dO and the gradients (fp32 accumulation either way)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -8,7 +8,8 @@ the library is missing, every call raises -- there is no fallback implementation
     o, lse = forward(q, k, v, causal=False, block_mask=None, scale=None)
     dq, dk, dv = backward(q, k, v, o, do, lse, causal=False, block_mask=None, scale=None)
 
-q, k, v, o, do: bf16 CUDA tensors [B, H, N, d], contiguous, d in {64, 128}, any N >= 1.
+q, k, v, o, do: bf16 (or fp16) CUDA tensors [B, H, N, d] of one type, contiguous, d in {64, 128},
+any N >= 1.
 lse: fp32 [B, H, N]. block_mask: uint8 CUDA tensor [ceil(N/128), ceil(N/128)] or None.
 """
 from __future__ import annotations
@@ -27,6 +28,7 @@ __all__ = [
 LIB_PATH = Path(__file__).resolve().with_name("libfa.so")
 
 FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+FA_DTYPE_BF16, FA_DTYPE_F16 = 0, 1
 
 _lib = None
 
@@ -62,6 +64,12 @@ def library() -> ctypes.CDLL:
         lib.fa_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, vp, vp, sz, vp]
         lib.fa_bwd_dq_finish.restype = i32
         lib.fa_bwd_dq_finish.argtypes = [vp, i32, i32, i32, i32, vp, sz, vp]
+        for name, base in (("fa_fwd_typed", lib.fa_fwd), ("fa_bwd_typed", lib.fa_bwd),
+                           ("fa_bwd_preprocess_typed", lib.fa_bwd_preprocess),
+                           ("fa_bwd_main_typed", lib.fa_bwd_main), ("fa_bwd_dq_finish_typed", lib.fa_bwd_dq_finish)):
+            f = getattr(lib, name)
+            f.restype = i32
+            f.argtypes = [i32] + list(base.argtypes)
         lib.fa_last_device_status.restype = i32
         lib.fa_last_device_status.argtypes = [vp]
         lib.fa_selftest_wait_timeout.restype = i32
@@ -83,13 +91,18 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+_DTYPES = {torch.bfloat16: FA_DTYPE_BF16, torch.float16: FA_DTYPE_F16}
+
+
 def _check_qkv(*ts):
     q = ts[0]
     if q.dim() != 4:
         raise ValueError("expected [B, H, N, d] tensors")
+    if q.dtype not in _DTYPES:
+        raise ValueError("q, k, v (o, do) must be bf16 or fp16")
     for t in ts:
-        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != q.shape:
-            raise ValueError("q, k, v (o, do) must be contiguous bf16 CUDA tensors of one shape")
+        if not t.is_cuda or t.dtype != q.dtype or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError("q, k, v (o, do) must be contiguous CUDA tensors of one shape and type")
         if t.device != q.device:
             raise ValueError("all tensors must be on one device")
     return q.shape
@@ -115,8 +128,8 @@ def forward(q, k, v, causal: bool = False, block_mask=None, scale=None, out=None
     mask = _check_mask(block_mask, N, q.device)
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
-    _check(library().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, N, d, _scale(scale, d),
-                            int(bool(causal)), _ptr(mask), _stream(q.device)), "fa_fwd")
+    _check(library().fa_fwd_typed(_DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, N, d,
+                                  _scale(scale, d), int(bool(causal)), _ptr(mask), _stream(q.device)), "fa_fwd")
     return o, l
 
 
@@ -140,17 +153,18 @@ def backward(q, k, v, o, do, lse, causal: bool = False, block_mask=None, scale=N
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     ws, nbytes = _workspace(B, H, N, d, q.device, workspace)
-    _check(library().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
-                            _ptr(dv), B, H, N, d, _scale(scale, d), int(bool(causal)), _ptr(mask), _ptr(ws),
-                            nbytes, _stream(q.device)), "fa_bwd")
+    _check(library().fa_bwd_typed(_DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                                  _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, _scale(scale, d), int(bool(causal)),
+                                  _ptr(mask), _ptr(ws), nbytes, _stream(q.device)), "fa_bwd")
     return dq, dk, dv
 
 
 def bwd_preprocess(o, do, lse, scale=None, workspace=None):
     B, H, N, d = _check_qkv(o, do)
     ws, nbytes = _workspace(B, H, N, d, o.device, workspace)
-    _check(library().fa_bwd_preprocess(_ptr(o), _ptr(do), _ptr(lse), B, H, N, d, _scale(scale, d), _ptr(ws),
-                                       nbytes, _stream(o.device)), "fa_bwd_preprocess")
+    _check(library().fa_bwd_preprocess_typed(_DTYPES[o.dtype], _ptr(o), _ptr(do), _ptr(lse), B, H, N, d,
+                                             _scale(scale, d), _ptr(ws), nbytes, _stream(o.device)),
+           "fa_bwd_preprocess")
     return ws
 
 
@@ -160,18 +174,20 @@ def bwd_main(q, k, v, do, workspace, causal=False, block_mask=None, scale=None, 
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     nbytes = workspace.numel() * workspace.element_size()
-    _check(library().fa_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dk), _ptr(dv), B, H, N, d,
-                                 _scale(scale, d), int(bool(causal)), _ptr(mask), _ptr(workspace), nbytes,
-                                 _stream(q.device)), "fa_bwd_main")
+    _check(library().fa_bwd_main_typed(_DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dk), _ptr(dv),
+                                       B, H, N, d, _scale(scale, d), int(bool(causal)), _ptr(mask), _ptr(workspace),
+                                       nbytes, _stream(q.device)), "fa_bwd_main")
     return dk, dv
 
 
-def bwd_dq_finish(workspace, shape, device, dq=None):
+def bwd_dq_finish(workspace, shape, device, dq=None, dtype=torch.bfloat16):
     B, H, N, d = shape
-    dq = torch.empty(shape, dtype=torch.bfloat16, device=device) if dq is None else dq
+    dq = torch.empty(shape, dtype=dtype, device=device) if dq is None else dq
+    if dq.dtype not in _DTYPES:
+        raise ValueError("dq must be bf16 or fp16")
     nbytes = workspace.numel() * workspace.element_size()
-    _check(library().fa_bwd_dq_finish(_ptr(dq), B, H, N, d, _ptr(workspace), nbytes, _stream(device)),
-           "fa_bwd_dq_finish")
+    _check(library().fa_bwd_dq_finish_typed(_DTYPES[dq.dtype], _ptr(dq), B, H, N, d, _ptr(workspace), nbytes,
+                                            _stream(device)), "fa_bwd_dq_finish")
     return dq
 
 

@@ -26,13 +26,14 @@ bool get_encoder() {
   return g_encode != nullptr;
 }
 
-// [BH][N][D] bf16 viewed as a 3-D tensor {D, N, BH}; box 64 x 128 x 1, 128-byte swizzle.
-bool encode_bhnd(CUtensorMap* map, const void* base, long long BH, int N, int D) {
+// [BH][N][D] bf16 (or fp16) viewed as a 3-D tensor {D, N, BH}; box 64 x 128 x 1, 128-byte swizzle.
+bool encode_bhnd(CUtensorMap* map, const void* base, long long BH, int N, int D, int f16) {
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+  const CUtensorMapDataType dt = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = g_encode(map, dt, 3, const_cast<void*>(base), dims, strides, box,
                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -50,6 +51,8 @@ bool encode_dq_acc(CUtensorMap* map, float* base, long long rows, int D) {
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+bool valid_dtype(int dt) { return dt == FA_DTYPE_BF16 || dt == FA_DTYPE_F16; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -102,8 +105,10 @@ const char* fa_status_string(fa_status s) {
   return "unknown fa_status";
 }
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-                 float scale, int causal, const uint8_t* block_mask, void* stream) {
+fa_status fa_fwd_typed(int dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                       int N, int d, float scale, int causal, const uint8_t* block_mask, void* stream) {
+  if (!valid_dtype(dtype)) return FA_ERR_INVALID;
+  const int f16 = dtype == FA_DTYPE_F16;
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID;
   fa_status st = check_common(B, H, N, d, scale);
@@ -111,8 +116,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   if (!get_encoder()) return FA_ERR_CUDA;
   const long long BH = (long long)B * H;
   alignas(64) CUtensorMap tq, tk, tv, to;
-  if (!encode_bhnd(&tq, q, BH, N, d) || !encode_bhnd(&tk, k, BH, N, d) || !encode_bhnd(&tv, v, BH, N, d) ||
-      !encode_bhnd(&to, o, BH, N, d))
+  if (!encode_bhnd(&tq, q, BH, N, d, f16) || !encode_bhnd(&tk, k, BH, N, d, f16) ||
+      !encode_bhnd(&tv, v, BH, N, d, f16) || !encode_bhnd(&to, o, BH, N, d, f16))
     return FA_ERR_CUDA;
   fa::FwdParams p;
   p.lse = lse;
@@ -122,7 +127,13 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
+  p.f16 = f16;
   return from_cuda(fa::launch_fwd(d, tq, tk, tv, to, p, (int)BH, static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                 float scale, int causal, const uint8_t* block_mask, void* stream) {
+  return fa_fwd_typed(FA_DTYPE_BF16, q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
@@ -130,8 +141,9 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   return layout(nullptr, B, H, N, d).bytes;
 }
 
-fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int N, int d,
-                            float scale, void* workspace, size_t workspace_bytes, void* stream) {
+fa_status fa_bwd_preprocess_typed(int dtype, const void* o, const void* dO, const float* lse, int B, int H, int N,
+                                  int d, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!valid_dtype(dtype)) return FA_ERR_INVALID;
   if (!o || !dO || !lse) return FA_ERR_INVALID;
   if (!aligned16(o) || !aligned16(dO) || !aligned16(lse)) return FA_ERR_INVALID;
   fa_status st = check_common(B, H, N, d, scale);
@@ -152,12 +164,20 @@ fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int
   p.Np = (N + 127) / 128 * 128;
   p.D = d;
   p.log2_scale = log2f(scale);
+  p.f16 = dtype == FA_DTYPE_F16;
   return from_cuda(fa::launch_bwd_pre(p, static_cast<cudaStream_t>(stream)));
 }
 
-fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B,
-                      int H, int N, int d, float scale, int causal, const uint8_t* block_mask, void* workspace,
-                      size_t workspace_bytes, void* stream) {
+fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int N, int d,
+                            float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  return fa_bwd_preprocess_typed(FA_DTYPE_BF16, o, dO, lse, B, H, N, d, scale, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_main_typed(int dtype, const void* q, const void* k, const void* v, const void* dO, void* dk,
+                            void* dv, int B, int H, int N, int d, float scale, int causal,
+                            const uint8_t* block_mask, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!valid_dtype(dtype)) return FA_ERR_INVALID;
+  const int f16 = dtype == FA_DTYPE_F16;
   if (!q || !k || !v || !dO || !dk || !dv) return FA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) || !aligned16(dv))
     return FA_ERR_INVALID;
@@ -171,8 +191,9 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* d
   if (!get_encoder()) return FA_ERR_CUDA;
   const long long BH = (long long)B * H;
   alignas(64) CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdqa;
-  if (!encode_bhnd(&tq, q, BH, N, d) || !encode_bhnd(&tk, k, BH, N, d) || !encode_bhnd(&tv, v, BH, N, d) ||
-      !encode_bhnd(&tdo, dO, BH, N, d) || !encode_bhnd(&tdk, dk, BH, N, d) || !encode_bhnd(&tdv, dv, BH, N, d) ||
+  if (!encode_bhnd(&tq, q, BH, N, d, f16) || !encode_bhnd(&tk, k, BH, N, d, f16) ||
+      !encode_bhnd(&tv, v, BH, N, d, f16) || !encode_bhnd(&tdo, dO, BH, N, d, f16) ||
+      !encode_bhnd(&tdk, dk, BH, N, d, f16) || !encode_bhnd(&tdv, dv, BH, N, d, f16) ||
       !encode_dq_acc(&tdqa, w.dq_acc, BH * ((N + 127) / 128 * 128), d))
     return FA_ERR_CUDA;
   fa::BwdParams p;
@@ -187,12 +208,21 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* d
   p.inv_scale = 1.0f / scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
+  p.f16 = f16;
   return from_cuda(
       fa::launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, tdqa, p, (int)BH, static_cast<cudaStream_t>(stream)));
 }
 
-fa_status fa_bwd_dq_finish(void* dq, int B, int H, int N, int d, void* workspace, size_t workspace_bytes,
-                           void* stream) {
+fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B,
+                      int H, int N, int d, float scale, int causal, const uint8_t* block_mask, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  return fa_bwd_main_typed(FA_DTYPE_BF16, q, k, v, dO, dk, dv, B, H, N, d, scale, causal, block_mask, workspace,
+                           workspace_bytes, stream);
+}
+
+fa_status fa_bwd_dq_finish_typed(int dtype, void* dq, int B, int H, int N, int d, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (!valid_dtype(dtype)) return FA_ERR_INVALID;
   if (!dq || !aligned16(dq)) return FA_ERR_INVALID;
   fa_status st = check_common(B, H, N, d, 1.0f);
   if (st != FA_OK) return st;
@@ -207,18 +237,35 @@ fa_status fa_bwd_dq_finish(void* dq, int B, int H, int N, int d, void* workspace
   p.Np = (N + 127) / 128 * 128;
   p.D = d;
   p.scale = 1.0f;  // the accumulated dQ already carries the scale (fa_bwd_main folds it into P)
+  p.f16 = dtype == FA_DTYPE_F16;
   return from_cuda(fa::launch_dq_finish(p, static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_bwd_dq_finish(void* dq, int B, int H, int N, int d, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  return fa_bwd_dq_finish_typed(FA_DTYPE_BF16, dq, B, H, N, d, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_typed(int dtype, const void* q, const void* k, const void* v, const void* o, const void* dO,
+                       const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+                       int causal, const uint8_t* block_mask, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  if (!valid_dtype(dtype)) return FA_ERR_INVALID;
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID;
+  fa_status st =
+      fa_bwd_preprocess_typed(dtype, o, dO, lse, B, H, N, d, scale, workspace, workspace_bytes, stream);
+  if (st != FA_OK) return st;
+  st = fa_bwd_main_typed(dtype, q, k, v, dO, dk, dv, B, H, N, d, scale, causal, block_mask, workspace,
+                         workspace_bytes, stream);
+  if (st != FA_OK) return st;
+  return fa_bwd_dq_finish_typed(dtype, dq, B, H, N, d, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                  void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
                  const uint8_t* block_mask, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID;
-  fa_status st = fa_bwd_preprocess(o, dO, lse, B, H, N, d, scale, workspace, workspace_bytes, stream);
-  if (st != FA_OK) return st;
-  st = fa_bwd_main(q, k, v, dO, dk, dv, B, H, N, d, scale, causal, block_mask, workspace, workspace_bytes, stream);
-  if (st != FA_OK) return st;
-  return fa_bwd_dq_finish(dq, B, H, N, d, workspace, workspace_bytes, stream);
+  return fa_bwd_typed(FA_DTYPE_BF16, q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, block_mask,
+                      workspace, workspace_bytes, stream);
 }
 
 fa_status fa_last_device_status(void* stream) {

@@ -102,8 +102,8 @@ __device__ __forceinline__ bool bwd_tile_active(const BwdParams& p, int i, int j
 
 // Writes one accumulator row (D fp32 columns of TMEM lane `row`, times `mul`) as bf16 into a
 // 128-row tile staged in the TMA store layout (64-column 128B-swizzled panels).
-template <int D>
-__device__ __forceinline__ void stage_row_bf16(uint32_t taddr, uint32_t sstage, int row, float mul, bool zero) {
+template <int D, bool F16>
+__device__ __forceinline__ void stage_row16(uint32_t taddr, uint32_t sstage, int row, float mul, bool zero) {
 #pragma unroll 1
   for (int c = 0; c < D / 32; ++c) {
     uint32_t u[32];
@@ -115,7 +115,7 @@ __device__ __forceinline__ void stage_row_bf16(uint32_t taddr, uint32_t sstage, 
     }
     uint32_t w[16];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) w[e] = pack_bf16(__uint_as_float(u[2 * e]) * mul, __uint_as_float(u[2 * e + 1]) * mul);
+    for (int e = 0; e < 16; ++e) w[e] = pack16<F16>(__uint_as_float(u[2 * e]) * mul, __uint_as_float(u[2 * e + 1]) * mul);
     const uint32_t panel = sstage + ((c * 32) >> 6) * (128 * 128);
     const uint32_t ch0 = ((c * 32) & 63) >> 3;
 #pragma unroll
@@ -124,7 +124,7 @@ __device__ __forceinline__ void stage_row_bf16(uint32_t taddr, uint32_t sstage, 
   }
 }
 
-template <int D>
+template <int D, bool F16>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -253,9 +253,9 @@ __global__ void __launch_bounds__(512, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);  // K/V (A) and Q/dO (B), K-major
-      constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, 0, 1);   // dV, dK: B = dO / Q MN-major
-      constexpr uint32_t IDESC_Q = idesc_bf16_f32(128, D, 1, 1);    // dQ = dS K: A = dS^T, B = K, MN-major
+      constexpr uint32_t IDESC_S = idesc_f32acc(128, 128, 0, 0, F16);  // K/V (A) and Q/dO (B), K-major
+      constexpr uint32_t IDESC_KV = idesc_f32acc(128, D, 0, 1, F16);   // dV, dK: B = dO / Q MN-major
+      constexpr uint32_t IDESC_Q = idesc_f32acc(128, D, 1, 1, F16);    // dQ = dS K: A = dS^T, B = K, MN-major
       constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
       const uint32_t tS = tmem + C::T_S, tDP = tmem + C::T_DP, tDV = tmem + C::T_DV, tDK = tmem + C::T_DK;
       const uint32_t tDQ = tmem + C::T_DQ;
@@ -452,8 +452,8 @@ __global__ void __launch_bounds__(512, 1)
             pf[q + 1] = p1;
             pf[q + 2] = p2;
             pf[q + 3] = p3;
-            pk[e] = pack_bf16(p0, p1);
-            pk[e + 1] = pack_bf16(p2, p3);
+            pk[e] = pack16<F16>(p0, p1);
+            pk[e + 1] = pack16<F16>(p2, p3);
           }
           tmem_st16(tS_row + c * 16, pk);  // columns [64h + 16c, +16): scores already read
         }
@@ -492,8 +492,8 @@ __global__ void __launch_bounds__(512, 1)
             float d0, d1, d2, d3;
             f2_unpack(ds01, d0, d1);
             f2_unpack(ds23, d2, d3);
-            dk[e] = pack_bf16(d0, d1);
-            dk[e + 1] = pack_bf16(d2, d3);
+            dk[e] = pack16<F16>(d0, d1);
+            dk[e + 1] = pack16<F16>(d2, d3);
           }
           // dS^T row kr, local queries 32c..32c+31 -> 16-byte chunks 4c .. 4c+3 of panel h
 #pragma unroll
@@ -513,7 +513,7 @@ __global__ void __launch_bounds__(512, 1)
     uint8_t* stage = smem + C::OFF_Q;  // Q ring stage 0 is free once every MMA retired
     if (ok && h < C::PANELS) {
       tc_fence_after();
-      stage_row_bf16<64>(tmem + lane_off + C::T_DV + 64u * h, smem_u32(stage + h * C::PANEL_BYTES), kr, p.inv_scale,
+      stage_row16<64, F16>(tmem + lane_off + C::T_DV + 64u * h, smem_u32(stage + h * C::PANEL_BYTES), kr, p.inv_scale,
                          it == 0);
       fence_proxy_async_smem();
     }
@@ -586,7 +586,7 @@ __global__ void __launch_bounds__(512, 1)
     uint8_t* stage = smem + C::OFF_DO;  // dO ring stage 0, free once every MMA retired
     if (ok) {
       tc_fence_after();
-      stage_row_bf16<D>(tmem + lane_off + C::T_DK, smem_u32(stage), ln, 1.f, it == 0);
+      stage_row16<D, F16>(tmem + lane_off + C::T_DK, smem_u32(stage), ln, 1.f, it == 0);
       fence_proxy_async_smem();
     }
     named_bar_sync(2, 128);
@@ -606,23 +606,28 @@ __global__ void __launch_bounds__(512, 1)
   }
 }
 
-template <int D>
+template <int D, bool F16>
 static cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
                                 const CUtensorMap& tdqa, const BwdParams& p, int BH, cudaStream_t stream) {
   using C = BwdCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(fa_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  cudaError_t e =
+      cudaFuncSetAttribute(fa_bwd_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid(p.nb, BH);
-  fa_bwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdk, tdv, tdqa, p);
+  fa_bwd_kernel<D, F16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdk, tdv, tdqa, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
                             const CUtensorMap& tdqa, const BwdParams& p, int BH, cudaStream_t stream) {
-  if (D == 64) return launch_bwd_t<64>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
-  return launch_bwd_t<128>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+  if (p.f16) {
+    if (D == 64) return launch_bwd_t<64, true>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+    return launch_bwd_t<128, true>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+  }
+  if (D == 64) return launch_bwd_t<64, false>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+  return launch_bwd_t<128, false>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
 }
 
 }  // namespace fa

@@ -17,10 +17,7 @@
 
 namespace fa {
 
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-template <int D>
+template <int D, bool F16>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdPreParams p) {
   constexpr int TPR = D / 8;  // threads per row
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -36,10 +33,10 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdPreParams p) {
     if (row < p.rows) {
       const uint4 a = __ldg(reinterpret_cast<const uint4*>(p.o + row * D) + sub);
       const uint4 b = __ldg(reinterpret_cast<const uint4*>(p.dout + row * D) + sub);
-      acc = bf16lo(a.x) * bf16lo(b.x) + bf16hi(a.x) * bf16hi(b.x);
-      acc += bf16lo(a.y) * bf16lo(b.y) + bf16hi(a.y) * bf16hi(b.y);
-      acc += bf16lo(a.z) * bf16lo(b.z) + bf16hi(a.z) * bf16hi(b.z);
-      acc += bf16lo(a.w) * bf16lo(b.w) + bf16hi(a.w) * bf16hi(b.w);
+      acc = unpack16_lo<F16>(a.x) * unpack16_lo<F16>(b.x) + unpack16_hi<F16>(a.x) * unpack16_hi<F16>(b.x);
+      acc += unpack16_lo<F16>(a.y) * unpack16_lo<F16>(b.y) + unpack16_hi<F16>(a.y) * unpack16_hi<F16>(b.y);
+      acc += unpack16_lo<F16>(a.z) * unpack16_lo<F16>(b.z) + unpack16_hi<F16>(a.z) * unpack16_hi<F16>(b.z);
+      acc += unpack16_lo<F16>(a.w) * unpack16_lo<F16>(b.w) + unpack16_hi<F16>(a.w) * unpack16_hi<F16>(b.w);
     }
 #pragma unroll
     for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, TPR);
@@ -63,7 +60,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdPreParams p) {
   for (long long e = tid; e < nvec; e += nthreads) acc4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-template <int D>
+template <int D, bool F16>
 __global__ void __launch_bounds__(256) fa_dq_finish_kernel(const DqFinishParams p) {
   constexpr int TPR = D / 8;
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -76,10 +73,10 @@ __global__ void __launch_bounds__(256) fa_dq_finish_kernel(const DqFinishParams 
     const float4* src = reinterpret_cast<const float4*>(p.dq_acc + (bh * p.Np + i) * D) + 2 * sub;
     const float4 a = src[0], b = src[1];
     uint4 w;
-    w.x = pack_bf16(a.x * p.scale, a.y * p.scale);
-    w.y = pack_bf16(a.z * p.scale, a.w * p.scale);
-    w.z = pack_bf16(b.x * p.scale, b.y * p.scale);
-    w.w = pack_bf16(b.z * p.scale, b.w * p.scale);
+    w.x = pack16<F16>(a.x * p.scale, a.y * p.scale);
+    w.y = pack16<F16>(a.z * p.scale, a.w * p.scale);
+    w.z = pack16<F16>(b.x * p.scale, b.y * p.scale);
+    w.w = pack16<F16>(b.z * p.scale, b.w * p.scale);
     reinterpret_cast<uint4*>(p.dq + row * D)[sub] = w;
   }
 }
@@ -98,18 +95,21 @@ static int sm_count() {
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream) {
   const int grid = sm_count() * 8;  // 8 resident 256-thread blocks per SM
   if (p.D == 64)
-    fa_bwd_pre_kernel<64><<<grid, 256, 0, stream>>>(p);
+    p.f16 ? fa_bwd_pre_kernel<64, true><<<grid, 256, 0, stream>>>(p) : fa_bwd_pre_kernel<64, false><<<grid, 256, 0, stream>>>(p);
   else
-    fa_bwd_pre_kernel<128><<<grid, 256, 0, stream>>>(p);
+    p.f16 ? fa_bwd_pre_kernel<128, true><<<grid, 256, 0, stream>>>(p)
+          : fa_bwd_pre_kernel<128, false><<<grid, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dq_finish(const DqFinishParams& p, cudaStream_t stream) {
   const int grid = sm_count() * 8;
   if (p.D == 64)
-    fa_dq_finish_kernel<64><<<grid, 256, 0, stream>>>(p);
+    p.f16 ? fa_dq_finish_kernel<64, true><<<grid, 256, 0, stream>>>(p)
+          : fa_dq_finish_kernel<64, false><<<grid, 256, 0, stream>>>(p);
   else
-    fa_dq_finish_kernel<128><<<grid, 256, 0, stream>>>(p);
+    p.f16 ? fa_dq_finish_kernel<128, true><<<grid, 256, 0, stream>>>(p)
+          : fa_dq_finish_kernel<128, false><<<grid, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

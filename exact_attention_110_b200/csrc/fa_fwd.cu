@@ -84,7 +84,7 @@ __device__ __forceinline__ bool fwd_tile_active(const FwdParams& p, int qb, int 
 // After the first two chunks (keys 0-63) the warp arrives on `half0`, so the tensor core can
 // start O += P V on those keys while the second half is computed; the caller signals the
 // second half. Returns the row sum of p.
-template <bool EMU, uint32_t EMU_MASK>
+template <bool F16, bool EMU, uint32_t EMU_MASK>
 __device__ __forceinline__ float softmax_exp_store(const uint32_t (&su)[128], uint64_t sl2_2, uint64_t mneg_2,
                                                    uint32_t tS_row, const Ex2PolyConsts& K, uint64_t* half0) {
   uint64_t ls2[4];
@@ -108,7 +108,7 @@ __device__ __forceinline__ float softmax_exp_store(const uint32_t (&su)[128], ui
       ls2[i & 3] = fadd2(ls2[i & 3], p2);
       float p0, p1;
       f2_unpack(p2, p0, p1);
-      pk[i] = pack_bf16(p0, p1);
+      pk[i] = pack16<F16>(p0, p1);
     }
     tmem_st16(tS_row + c * 16, pk);
     if (c == 1) {
@@ -124,7 +124,7 @@ __device__ __forceinline__ float softmax_exp_store(const uint32_t (&su)[128], ui
   return a + b;
 }
 
-template <int D>
+template <int D, bool F16>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -248,8 +248,8 @@ __global__ void __launch_bounds__(384, 1)
     // thread spends a few cycles per MMA instead of a dependent chain of 64-bit ALU ops --
     // the issue rate, not the tensor core, otherwise limits M=128 x N=128 MMAs.
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);  // Q, K both K-major
-      constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);    // P (TMEM), V MN-major
+      constexpr uint32_t IDESC_S = idesc_f32acc(128, 128, 0, 0, F16);  // Q, K both K-major
+      constexpr uint32_t IDESC_O = idesc_f32acc(128, D, 0, 1, F16);    // P (TMEM), V MN-major
       constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
       const uint64_t dq_base = sdesc_sw128(sQ, 16, 1024);
       const uint64_t dk_base = sdesc_sw128(sK, 16, 1024);
@@ -412,9 +412,9 @@ __global__ void __launch_bounds__(384, 1)
         const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
         const uint64_t sl2_2 = f2_pack(sl2, sl2), mneg_2 = f2_pack(mneg, mneg);
         if (masked)
-          l += softmax_exp_store<false, 0u>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[2 * t]);
+          l += softmax_exp_store<F16, false, 0u>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[2 * t]);
         else
-          l += softmax_exp_store<true, C::EXP_EMU_MASK>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[2 * t]);
+          l += softmax_exp_store<F16, true, C::EXP_EMU_MASK>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[2 * t]);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -441,7 +441,7 @@ __global__ void __launch_bounds__(384, 1)
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            w[i] = pack_bf16(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
+            w[i] = pack16<F16>(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
           const int col0 = c * 32;                   // first column of this chunk
           const uint32_t panel = sstage + (col0 >> 6) * C::PANEL_BYTES;
           const uint32_t chunk0 = (col0 & 63) >> 3;  // 16-byte chunk inside the 128-byte row
@@ -473,21 +473,26 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <int D>
+template <int D, bool F16>
 static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream) {
   using C = FwdCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  cudaError_t e =
+      cudaFuncSetAttribute(fa_fwd_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid((p.nb + 1) / 2, BH);
-  fa_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
+  fa_fwd_kernel<D, F16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream) {
-  if (D == 64) return launch_fwd_t<64>(tq, tk, tv, to, p, BH, stream);
-  return launch_fwd_t<128>(tq, tk, tv, to, p, BH, stream);
+  if (p.f16) {
+    if (D == 64) return launch_fwd_t<64, true>(tq, tk, tv, to, p, BH, stream);
+    return launch_fwd_t<128, true>(tq, tk, tv, to, p, BH, stream);
+  }
+  if (D == 64) return launch_fwd_t<64, false>(tq, tk, tv, to, p, BH, stream);
+  return launch_fwd_t<128, false>(tq, tk, tv, to, p, BH, stream);
 }
 
 }  // namespace fa

@@ -31,6 +31,7 @@ struct FwdParams {
   int causal;
   float scale_log2;            // scale * log2(e)
   unsigned long long timeout_ns;
+  int f16;                     // element type: fp16 if non-zero, bf16 otherwise
 };
 
 struct BwdPreParams {
@@ -43,6 +44,7 @@ struct BwdPreParams {
   long long rows;        // BH * N
   int N, Np, D;
   float log2_scale;      // log2(scale), scale > 0: folds the softmax scale into P (see fa_bwd.cu)
+  int f16;               // element type: fp16 if non-zero, bf16 otherwise
 };
 
 struct BwdParams {
@@ -55,6 +57,7 @@ struct BwdParams {
   float inv_scale;       // 1 / scale (dV epilogue: P carries the scale)
   float scale_log2;      // scale * log2(e)
   unsigned long long timeout_ns;
+  int f16;               // element type: fp16 if non-zero, bf16 otherwise
 };
 
 struct DqFinishParams {
@@ -63,6 +66,7 @@ struct DqFinishParams {
   long long rows;        // BH * N
   int N, Np, D;
   float scale;
+  int f16;               // element type: fp16 if non-zero, bf16 otherwise
 };
 
 // Launchers (return the launch error, if any).

@@ -253,10 +253,10 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major, int b_mn_major) {
-  return (1u << 4)     // D: f32
-         | (1u << 7)   // A: bf16
-         | (1u << 10)  // B: bf16
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, int a_mn_major, int b_mn_major, bool f16) {
+  return (1u << 4)                          // D: f32
+         | ((f16 ? 0u : 1u) << 7)           // A: f16 (0) or bf16 (1)
+         | ((f16 ? 0u : 1u) << 10)          // B: same type as A
          | (static_cast<uint32_t>(a_mn_major) << 15) | (static_cast<uint32_t>(b_mn_major) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
@@ -481,6 +481,40 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+// The same into IEEE fp16x2.
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// 16-bit element type of the kernels: fp16 when F16, bf16 otherwise.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack16(float lo, float hi) {
+  if constexpr (F16)
+    return pack_f16(lo, hi);
+  else
+    return pack_bf16(lo, hi);
+}
+template <bool F16>
+__device__ __forceinline__ float unpack16_lo(uint32_t w) {
+  if constexpr (F16) {
+    float r;
+    asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n cvt.f32.f16 %0, lo;\n}" : "=f"(r) : "r"(w));
+    return r;
+  } else {
+    return __uint_as_float(w << 16);
+  }
+}
+template <bool F16>
+__device__ __forceinline__ float unpack16_hi(uint32_t w) {
+  if constexpr (F16) {
+    float r;
+    asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n cvt.f32.f16 %0, hi;\n}" : "=f"(r) : "r"(w));
+    return r;
+  } else {
+    return __uint_as_float(w & 0xFFFF0000u);
+  }
 }
 
 

@@ -69,8 +69,17 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
-def normal_bf16(seed: int, n: int) -> np.ndarray:
-    """n standard-normal draws as bf16 bit patterns (uint16)."""
+def f32_to_f16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp32 values to IEEE fp16 (round to nearest, ties to even) as bit patterns."""
+    return np.ascontiguousarray(x, dtype=np.float32).astype(np.float16).view(np.uint16)
+
+
+def f16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Widen fp16 bit patterns to fp32 (exact)."""
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float32)
+
+
+def _normal_bits(seed: int, n: int, to_bits) -> np.ndarray:
     out = np.empty(n, dtype=np.uint16)
     npairs_total = (n + 1) // 2
     for lo in range(0, npairs_total, _CHUNK):
@@ -83,8 +92,26 @@ def normal_bf16(seed: int, n: int) -> np.ndarray:
         z[0::2] = r * np.cos(theta)
         z[1::2] = r * np.sin(theta)
         m = min(n - 2 * lo, z.size)
-        out[2 * lo:2 * lo + m] = f32_to_bf16_bits(z[:m].astype(np.float32))
+        out[2 * lo:2 * lo + m] = to_bits(z[:m].astype(np.float32))
     return out
+
+
+def normal_bf16(seed: int, n: int) -> np.ndarray:
+    """n standard-normal draws as bf16 bit patterns (uint16)."""
+    return _normal_bits(seed, n, f32_to_bf16_bits)
+
+
+def normal_f16(seed: int, n: int) -> np.ndarray:
+    """The same n standard-normal draws as fp16 bit patterns (uint16)."""
+    return _normal_bits(seed, n, f32_to_f16_bits)
+
+
+def normal_bits(seed: int, n: int, dtype: str = "bf16") -> np.ndarray:
+    return normal_f16(seed, n) if dtype == "f16" else normal_bf16(seed, n)
+
+
+def bits_to_f32(bits: np.ndarray, dtype: str = "bf16") -> np.ndarray:
+    return f16_bits_to_f32(bits) if dtype == "f16" else bf16_bits_to_f32(bits)
 
 
 def bernoulli_block_mask(seed: int, nb: int, p: float = 0.25, force_diagonal: bool = True) -> np.ndarray:
@@ -96,17 +123,18 @@ def bernoulli_block_mask(seed: int, nb: int, p: float = 0.25, force_diagonal: bo
     return m
 
 
-def attention_inputs(B: int, H: int, N: int, d: int, base_seed: int = BASE_SEED, with_do: bool = True):
-    """Q, K, V (and dO) for a [B, H, N, d] problem as bf16 bit arrays of that shape."""
+def attention_inputs(B: int, H: int, N: int, d: int, base_seed: int = BASE_SEED, with_do: bool = True,
+                     dtype: str = "bf16"):
+    """Q, K, V (and dO) for a [B, H, N, d] problem as bf16 (or fp16) bit arrays of that shape."""
     shape = (B, H, N, d)
     n = B * H * N * d
     out = {
-        "q": normal_bf16(base_seed + SEED_Q, n).reshape(shape),
-        "k": normal_bf16(base_seed + SEED_K, n).reshape(shape),
-        "v": normal_bf16(base_seed + SEED_V, n).reshape(shape),
+        "q": normal_bits(base_seed + SEED_Q, n, dtype).reshape(shape),
+        "k": normal_bits(base_seed + SEED_K, n, dtype).reshape(shape),
+        "v": normal_bits(base_seed + SEED_V, n, dtype).reshape(shape),
     }
     if with_do:
-        out["do"] = normal_bf16(base_seed + SEED_DO, n).reshape(shape)
+        out["do"] = normal_bits(base_seed + SEED_DO, n, dtype).reshape(shape)
     return out
 
 
@@ -120,4 +148,13 @@ def to_torch_bf16(bits: np.ndarray, device="cpu"):
     import torch
 
     t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.to(device)
+
+
+def to_torch(bits: np.ndarray, dtype: str = "bf16", device="cpu"):
+    """bf16 or fp16 bit patterns as a torch tensor of that type on `device` (bit-exact)."""
+    import torch
+
+    tdt = torch.float16 if dtype == "f16" else torch.bfloat16
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(tdt)
     return t.to(device)

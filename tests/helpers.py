@@ -9,34 +9,27 @@ import torch
 
 import synth
 
-# Parity bars for bf16 inputs drawn from N(0, 1).
+# Parity bars for bf16 (and fp16) inputs drawn from N(0, 1).
 O_MAX_ABS = 1e-2
 O_MEAN_ABS = 1e-3
 LSE_MAX_ABS = 1e-3
 GRAD_REL_FRO = 2e-2
 
 
-def bits_to_torch(bits: np.ndarray, device) -> torch.Tensor:
-    return synth.to_torch_bf16(bits, device)
-
-
-def bits_to_f64(bits: np.ndarray) -> np.ndarray:
-    return synth.bf16_bits_to_f32(bits).astype(np.float64)
-
-
 @functools.lru_cache(maxsize=8)
-def _stream(seed: int, n: int) -> np.ndarray:
-    return synth.normal_bf16(seed, n)
+def _stream(seed: int, n: int, dtype: str) -> np.ndarray:
+    return synth.normal_bits(seed, n, dtype)
 
 
-def make_case(B, H, N, d, seed=synth.BASE_SEED, device="cuda", with_do=True):
-    """Same bytes as synth.attention_inputs (cached: many cases share stream lengths)."""
+def make_case(B, H, N, d, seed=synth.BASE_SEED, device="cuda", with_do=True, dtype="bf16"):
+    """Same bytes as synth.attention_inputs (cached: many cases share stream lengths): the
+    16-bit tensors for the GPU and their exact fp64 values for the oracle."""
     n, shape = B * H * N * d, (B, H, N, d)
     names = ("q", "k", "v", "do") if with_do else ("q", "k", "v")
     offs = (synth.SEED_Q, synth.SEED_K, synth.SEED_V, synth.SEED_DO)
-    bits = {k: _stream(seed + o, n).reshape(shape) for k, o in zip(names, offs)}
-    gpu = {k: bits_to_torch(v, device) for k, v in bits.items()}
-    f64 = {k: bits_to_f64(v) for k, v in bits.items()}
+    bits = {k: _stream(seed + o, n, dtype).reshape(shape) for k, o in zip(names, offs)}
+    gpu = {k: synth.to_torch(v, dtype, device) for k, v in bits.items()}
+    f64 = {k: synth.bits_to_f32(v, dtype).astype(np.float64) for k, v in bits.items()}
     return gpu, f64
 
 

@@ -80,6 +80,20 @@ def test_workspace_size_and_checks(lib):
     assert lib.fa_bwd_main(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 48, 0.1, 0, None, FAKE, need, None) == 2
 
 
+def test_typed_entry_points_check_dtype(lib):
+    # the element type must be FA_DTYPE_BF16 (0) or FA_DTYPE_F16 (1); checked before anything else
+    need = lib.fa_bwd_workspace_bytes(1, 1, 128, 64)
+    for bad in (-1, 2, 7):
+        assert lib.fa_fwd_typed(bad, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0, None, None) == 1
+        assert lib.fa_bwd_typed(bad, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0,
+                                None, FAKE, need, None) == 1
+        assert lib.fa_bwd_dq_finish_typed(bad, FAKE, 1, 1, 128, 64, FAKE, need, None) == 1
+    # valid types still get the ordinary argument checks
+    for dt in (0, 1):
+        assert lib.fa_fwd_typed(dt, None, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0, None, None) == 1
+        assert lib.fa_fwd_typed(dt, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 96, 0.125, 0, None, None) == 2
+
+
 @pytest.mark.parametrize("scale", [0.0, -0.125])
 def test_backward_needs_positive_scale(lib, scale):
     # The backward folds log2(scale) into the recomputed probabilities: scale <= 0 is refused

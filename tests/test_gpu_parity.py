@@ -82,6 +82,43 @@ def test_fwd_bwd_small(fa, oracle_mod, B, Hh, N, d, causal, mask):
     H.assert_grads_close([H.to_f64(x) for x in (dq, dk, dv)], g_ref, f"bwd {B,Hh,N,d,causal,mask}")
 
 
+FP16 = [
+    # B, H, N, d, causal, mask: fp16 inputs and outputs through the *_typed entry points
+    (1, 2, 384, 64, False, None),
+    (2, 1, 640, 64, True, None),
+    (1, 2, 512, 128, True, None),
+    (1, 1, 333, 128, False, "bernoulli"),
+]
+
+
+@pytest.mark.parametrize("B,Hh,N,d,causal,mask", FP16)
+def test_fwd_bwd_fp16(fa, oracle_mod, B, Hh, N, d, causal, mask):
+    gpu, ref = H.make_case(B, Hh, N, d, seed=synth.BASE_SEED + 3 * N + d, dtype="f16")
+    assert gpu["q"].dtype == torch.float16
+    scale = 1.0 / np.sqrt(d)
+    m = mask_for(mask, N)
+    mt = None if m is None else torch.from_numpy(m).cuda()
+    o, lse = run_fwd(fa, gpu, causal, mt, scale)
+    assert o.dtype == torch.float16
+    o_ref, lse_ref = oracle_mod.attention_fwd(ref["q"], ref["k"], ref["v"], scale, causal=causal, mask=m)
+    H.assert_fwd_close(H.to_f64(o), H.to_f64(lse), o_ref, lse_ref, f"fp16 fwd {B,Hh,N,d,causal,mask}")
+    dq, dk, dv = run_bwd(fa, gpu, o, lse, causal, mt, scale)
+    assert dq.dtype == dk.dtype == dv.dtype == torch.float16
+    g_ref = oracle_mod.attention_bwd(ref["q"], ref["k"], ref["v"], ref["do"], scale, causal=causal, mask=m)[:3]
+    H.assert_grads_close([H.to_f64(x) for x in (dq, dk, dv)], g_ref, f"fp16 bwd {B,Hh,N,d,causal,mask}")
+
+
+def test_fp16_and_bf16_agree(fa):
+    # The same draws rounded to each type give nearly the same attention: the element type
+    # only changes input rounding and the 16-bit P (fp16 carries three more mantissa bits).
+    g16, _ = H.make_case(1, 2, 512, 128, seed=synth.BASE_SEED + 5, dtype="f16")
+    gbf, _ = H.make_case(1, 2, 512, 128, seed=synth.BASE_SEED + 5, dtype="bf16")
+    o16, l16 = run_fwd(fa, g16, False, None, 0.0884)
+    obf, lbf = run_fwd(fa, gbf, False, None, 0.0884)
+    assert (o16.float() - obf.float()).abs().max().item() < 3e-2
+    assert (l16 - lbf).abs().max().item() < 3e-2
+
+
 def sampled_heads(B, Hh, n, seed):
     rng = np.random.default_rng(seed)
     flat = rng.choice(B * Hh, size=min(n, B * Hh), replace=False)
