@@ -7,7 +7,8 @@ N=4096 point (16k tokens, hidden 2048 -> B=4, H=16, d=128), non-causal, bf16 N(0
 inputs from the seeded generator. Prints ONE JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--seqlen N] [--headdim d]
-                    [--causal] [--block-sparse] [--dtype bf16|f16] [--impl reference] [--sweep]
+                    [--causal] [--block-sparse [--block-density P]] [--dtype bf16|f16]
+                    [--impl reference] [--sweep] [--density-sweep]
 
 Metric: fwd+bwd TFLOPS with FLOPs counted as 4*B*H*N^2*d for the forward (halved for causal,
 scaled by block density for block-sparse) and 2.5x that for the backward.
@@ -38,10 +39,10 @@ UNIT = "TFLOPS"
 
 
 # ----------------------------------------------------------------------------- host logic
-def workload(seqlen: int, headdim: int, causal: bool, block_sparse: bool):
+def workload(seqlen: int, headdim: int, causal: bool, block_sparse: bool, p_on: float = 0.25):
     if block_sparse:
-        return dict(B=4, H=16, N=4096, d=64, causal=False, block_sparse=True,
-                    name="block-sparse B=4 H=16 N=4096 d=64, 128x128 blocks Bernoulli(0.25), diagonal on")
+        return dict(B=4, H=16, N=4096, d=64, causal=False, block_sparse=True, p_on=p_on,
+                    name=f"block-sparse B=4 H=16 N=4096 d=64, 128x128 blocks Bernoulli({p_on:g}), diagonal on")
     B, H = TOKENS // seqlen, HIDDEN // headdim
     return dict(B=B, H=H, N=seqlen, d=headdim, causal=causal, block_sparse=False,
                 name=f"seq-len sweep (16k tokens, hidden 2048): N={seqlen} d={headdim} B={B} H={H} "
@@ -157,7 +158,7 @@ def oracle_sample(wl, nheads: int, seed: int, dtype: str = "bf16"):
     import oracle
     import synth
     B, H, N, d = wl["B"], wl["H"], wl["N"], wl["d"]
-    mask = synth.block_mask_for(N) if wl["block_sparse"] else None
+    mask = synth.block_mask_for(N, p=wl.get("p_on", 0.25)) if wl["block_sparse"] else None
     n = nheads * N * d
     q, k, v, do = (synth.bits_to_f32(synth.normal_bits(seed + i, n, dtype), dtype).astype(np.float64)
                    .reshape(1, nheads, N, d) for i in range(4))
@@ -172,7 +173,8 @@ def oracle_sample(wl, nheads: int, seed: int, dtype: str = "bf16"):
 
 
 def heads_for_seconds(wl, target_s: float, rate_gflops: float = 20.0) -> int:
-    per_head = 3.5 * fwd_flops(1, 1, wl["N"], wl["d"], wl["causal"], 0.27 if wl["block_sparse"] else 1.0)
+    per_head = 3.5 * fwd_flops(1, 1, wl["N"], wl["d"], wl["causal"],
+                               wl.get("p_on", 0.25) + 0.03 if wl["block_sparse"] else 1.0)
     return max(1, min(wl["B"] * wl["H"], int(target_s * rate_gflops * 1e9 / per_head)))
 
 
@@ -225,7 +227,7 @@ def run_gpu(args, wl, rank, world, local_rank, dist_on):
     offs = (synth.SEED_Q, synth.SEED_K, synth.SEED_V, synth.SEED_DO)
     q, k, v, do = (synth.to_torch(_stream(seed + o, B * H * N * d, args.dtype).reshape(B, H, N, d), args.dtype, dev)
                    for o in offs)
-    mask_np = synth.block_mask_for(N) if wl["block_sparse"] else None
+    mask_np = synth.block_mask_for(N, p=wl.get("p_on", 0.25)) if wl["block_sparse"] else None
     mask = None if mask_np is None else torch.from_numpy(mask_np).to(dev)
     density = float(mask_np.mean()) if mask_np is not None else 1.0
     scale = 1.0 / math.sqrt(d)
@@ -317,6 +319,7 @@ def run_gpu(args, wl, rank, world, local_rank, dist_on):
     main_flops = 2.5 * f_fwd
     achieved = main_flops / (main_ms * 1e-3) / 1e12
     traffic = recorded_traffic(f"bwd_main N={N} d={d} causal={int(causal)} bs={int(wl['block_sparse'])}"
+                               + (f" p={wl['p_on']:g}" if wl["block_sparse"] and wl["p_on"] != 0.25 else "")
                                + ("" if args.dtype == "bf16" else f" {args.dtype}"))
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"], "traffic": traffic, "kernel": "fa_bwd_kernel",
@@ -375,6 +378,10 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="one JSON line per sweep point (N x d x causal)")
+    ap.add_argument("--block-density", type=float, default=0.25,
+                    help="with --block-sparse: probability that an off-diagonal 128x128 block is on")
+    ap.add_argument("--density-sweep", action="store_true",
+                    help="block-sparse config at densities 0.05..1: runtime should follow the blocks that are on")
     ap.add_argument("--dtype", choices=["bf16", "f16"], default="bf16",
                     help="element type of q, k, v, o, dO and the gradients (fp32 accumulation either way)")
     args = ap.parse_args(argv)
@@ -386,7 +393,7 @@ def main(argv=None):
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     dist_on = world > 1
     if args.impl == "reference":
-        wl = workload(args.seqlen, args.headdim, args.causal, args.block_sparse)
+        wl = workload(args.seqlen, args.headdim, args.causal, args.block_sparse, args.block_density)
         return run_reference(args, wl, rank, world)
     if dist_on:
         import datetime
@@ -396,10 +403,15 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.density_sweep:
+            args.no_cpu_baseline, args.no_e2e = True, True
+            for p_on in (0.05, 0.1, 0.25, 0.5, 1.0):
+                run_gpu(args, workload(args.seqlen, args.headdim, False, True, p_on), rank, world, local_rank, dist_on)
+            return 0
         points = ([(n, dd, c) for dd in (64, 128) for c in (False, True) for n in (512, 1024, 2048, 4096, 8192, 16384)]
                   if args.sweep else [(args.seqlen, args.headdim, args.causal)])
         for (n, dd, c) in points:
-            wl = workload(n, dd, c, args.block_sparse)
+            wl = workload(n, dd, c, args.block_sparse, args.block_density)
             if args.sweep:
                 args.no_cpu_baseline, args.no_e2e = True, True
             run_gpu(args, wl, rank, world, local_rank, dist_on)

@@ -10,7 +10,8 @@ the library is missing, every call raises -- there is no fallback implementation
 
 q, k, v, o, do: bf16 (or fp16) CUDA tensors [B, H, N, d] of one type, contiguous, d in {64, 128},
 any N >= 1.
-lse: fp32 [B, H, N]. block_mask: uint8 CUDA tensor [ceil(N/128), ceil(N/128)] or None.
+lse: fp32 [B, H, N]. block_mask: uint8 CUDA tensor [nb, nb] shared by every head, or one mask per
+head [B, H, nb, nb] (nb = ceil(N/128)), or None.
 """
 from __future__ import annotations
 
@@ -64,12 +65,18 @@ def library() -> ctypes.CDLL:
         lib.fa_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, vp, vp, sz, vp]
         lib.fa_bwd_dq_finish.restype = i32
         lib.fa_bwd_dq_finish.argtypes = [vp, i32, i32, i32, i32, vp, sz, vp]
-        for name, base in (("fa_fwd_typed", lib.fa_fwd), ("fa_bwd_typed", lib.fa_bwd),
-                           ("fa_bwd_preprocess_typed", lib.fa_bwd_preprocess),
-                           ("fa_bwd_main_typed", lib.fa_bwd_main), ("fa_bwd_dq_finish_typed", lib.fa_bwd_dq_finish)):
-            f = getattr(lib, name)
-            f.restype = i32
-            f.argtypes = [i32] + list(base.argtypes)
+        i64 = ctypes.c_longlong
+        lib.fa_fwd_ex.restype = i32
+        lib.fa_fwd_ex.argtypes = [i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, vp, i64, vp]
+        lib.fa_bwd_ex.restype = i32
+        lib.fa_bwd_ex.argtypes = [i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, vp, i64,
+                                  vp, sz, vp]
+        lib.fa_bwd_preprocess_ex.restype = i32
+        lib.fa_bwd_preprocess_ex.argtypes = [i32] + list(lib.fa_bwd_preprocess.argtypes)
+        lib.fa_bwd_main_ex.restype = i32
+        lib.fa_bwd_main_ex.argtypes = [i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, vp, i64, vp, sz, vp]
+        lib.fa_bwd_dq_finish_ex.restype = i32
+        lib.fa_bwd_dq_finish_ex.argtypes = [i32] + list(lib.fa_bwd_dq_finish.argtypes)
         lib.fa_last_device_status.restype = i32
         lib.fa_last_device_status.argtypes = [vp]
         lib.fa_selftest_wait_timeout.restype = i32
@@ -108,14 +115,22 @@ def _check_qkv(*ts):
     return q.shape
 
 
-def _check_mask(block_mask, N, dev):
+def _check_mask(block_mask, B, H, N, dev):
+    """Returns (mask, per-head stride in elements): 0 for one shared [nb, nb] mask."""
     if block_mask is None:
-        return None
+        return None, 0
     nb = (N + 127) // 128
-    if (not block_mask.is_cuda or block_mask.dtype != torch.uint8 or not block_mask.is_contiguous()
-            or tuple(block_mask.shape) != (nb, nb) or block_mask.device != dev):
-        raise ValueError(f"block_mask must be a contiguous uint8 CUDA tensor of shape ({nb}, {nb})")
-    return block_mask
+    shape = tuple(block_mask.shape)
+    if shape == (nb, nb):
+        stride = 0
+    elif shape in ((B, H, nb, nb), (B * H, nb, nb)):
+        stride = nb * nb
+    else:
+        raise ValueError(f"block_mask must have shape ({nb}, {nb}) or ({B}, {H}, {nb}, {nb})")
+    if not block_mask.is_cuda or block_mask.dtype != torch.uint8 or not block_mask.is_contiguous() \
+            or block_mask.device != dev:
+        raise ValueError("block_mask must be a contiguous uint8 CUDA tensor on the tensors' device")
+    return block_mask, stride
 
 
 def _scale(scale, d):
@@ -125,11 +140,11 @@ def _scale(scale, d):
 def forward(q, k, v, causal: bool = False, block_mask=None, scale=None, out=None, lse=None):
     """O = softmax(scale * Q K^T [masked]) V and the per-row log-sum-exp (natural log)."""
     B, H, N, d = _check_qkv(q, k, v)
-    mask = _check_mask(block_mask, N, q.device)
+    mask, mstride = _check_mask(block_mask, B, H, N, q.device)
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
-    _check(library().fa_fwd_typed(_DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, N, d,
-                                  _scale(scale, d), int(bool(causal)), _ptr(mask), _stream(q.device)), "fa_fwd")
+    _check(library().fa_fwd_ex(_DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, N, d,
+                               _scale(scale, d), int(bool(causal)), _ptr(mask), mstride, _stream(q.device)), "fa_fwd")
     return o, l
 
 
@@ -148,35 +163,35 @@ def backward(q, k, v, o, do, lse, causal: bool = False, block_mask=None, scale=N
              dq=None, dk=None, dv=None):
     """dQ, dK, dV of sum(O * dO) by recomputation from the saved LSE."""
     B, H, N, d = _check_qkv(q, k, v, o, do)
-    mask = _check_mask(block_mask, N, q.device)
+    mask, mstride = _check_mask(block_mask, B, H, N, q.device)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     ws, nbytes = _workspace(B, H, N, d, q.device, workspace)
-    _check(library().fa_bwd_typed(_DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
-                                  _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, _scale(scale, d), int(bool(causal)),
-                                  _ptr(mask), _ptr(ws), nbytes, _stream(q.device)), "fa_bwd")
+    _check(library().fa_bwd_ex(_DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                               _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, _scale(scale, d), int(bool(causal)),
+                               _ptr(mask), mstride, _ptr(ws), nbytes, _stream(q.device)), "fa_bwd")
     return dq, dk, dv
 
 
 def bwd_preprocess(o, do, lse, scale=None, workspace=None):
     B, H, N, d = _check_qkv(o, do)
     ws, nbytes = _workspace(B, H, N, d, o.device, workspace)
-    _check(library().fa_bwd_preprocess_typed(_DTYPES[o.dtype], _ptr(o), _ptr(do), _ptr(lse), B, H, N, d,
-                                             _scale(scale, d), _ptr(ws), nbytes, _stream(o.device)),
+    _check(library().fa_bwd_preprocess_ex(_DTYPES[o.dtype], _ptr(o), _ptr(do), _ptr(lse), B, H, N, d,
+                                          _scale(scale, d), _ptr(ws), nbytes, _stream(o.device)),
            "fa_bwd_preprocess")
     return ws
 
 
 def bwd_main(q, k, v, do, workspace, causal=False, block_mask=None, scale=None, dk=None, dv=None):
     B, H, N, d = _check_qkv(q, k, v, do)
-    mask = _check_mask(block_mask, N, q.device)
+    mask, mstride = _check_mask(block_mask, B, H, N, q.device)
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     nbytes = workspace.numel() * workspace.element_size()
-    _check(library().fa_bwd_main_typed(_DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dk), _ptr(dv),
-                                       B, H, N, d, _scale(scale, d), int(bool(causal)), _ptr(mask), _ptr(workspace),
-                                       nbytes, _stream(q.device)), "fa_bwd_main")
+    _check(library().fa_bwd_main_ex(_DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dk), _ptr(dv),
+                                    B, H, N, d, _scale(scale, d), int(bool(causal)), _ptr(mask), mstride,
+                                    _ptr(workspace), nbytes, _stream(q.device)), "fa_bwd_main")
     return dk, dv
 
 
@@ -186,8 +201,8 @@ def bwd_dq_finish(workspace, shape, device, dq=None, dtype=torch.bfloat16):
     if dq.dtype not in _DTYPES:
         raise ValueError("dq must be bf16 or fp16")
     nbytes = workspace.numel() * workspace.element_size()
-    _check(library().fa_bwd_dq_finish_typed(_DTYPES[dq.dtype], _ptr(dq), B, H, N, d, _ptr(workspace), nbytes,
-                                            _stream(device)), "fa_bwd_dq_finish")
+    _check(library().fa_bwd_dq_finish_ex(_DTYPES[dq.dtype], _ptr(dq), B, H, N, d, _ptr(workspace), nbytes,
+                                         _stream(device)), "fa_bwd_dq_finish")
     return dq
 
 

@@ -54,6 +54,14 @@ bool encode_dq_acc(CUtensorMap* map, float* base, long long rows, int D) {
 
 bool valid_dtype(int dt) { return dt == FA_DTYPE_BF16 || dt == FA_DTYPE_F16; }
 
+// A per-(b, h) block-mask stride is 0 (one mask shared by every head) or at least one whole
+// ceil(N/128)^2 mask; it is ignored without a mask.
+bool mask_stride_ok(const uint8_t* mask, long long stride, int N) {
+  if (mask == nullptr) return true;
+  const long long nb = (N + 127) / 128;
+  return stride == 0 || stride >= nb * nb;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 fa_status check_common(int B, int H, int N, int d, float scale) {
@@ -105,9 +113,11 @@ const char* fa_status_string(fa_status s) {
   return "unknown fa_status";
 }
 
-fa_status fa_fwd_typed(int dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                       int N, int d, float scale, int causal, const uint8_t* block_mask, void* stream) {
+fa_status fa_fwd_ex(int dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                    int N, int d, float scale, int causal, const uint8_t* block_mask, long long block_mask_head_stride,
+                    void* stream) {
   if (!valid_dtype(dtype)) return FA_ERR_INVALID;
+  if (!mask_stride_ok(block_mask, block_mask_head_stride, N)) return FA_ERR_INVALID;
   const int f16 = dtype == FA_DTYPE_F16;
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID;
@@ -122,6 +132,7 @@ fa_status fa_fwd_typed(int dtype, const void* q, const void* k, const void* v, v
   fa::FwdParams p;
   p.lse = lse;
   p.block_mask = block_mask;
+  p.mask_stride = block_mask_head_stride;
   p.N = N;
   p.nb = (N + 127) / 128;  // the last tile may be partial: TMA zero-fills rows >= N
   p.causal = causal ? 1 : 0;
@@ -133,7 +144,7 @@ fa_status fa_fwd_typed(int dtype, const void* q, const void* k, const void* v, v
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                  float scale, int causal, const uint8_t* block_mask, void* stream) {
-  return fa_fwd_typed(FA_DTYPE_BF16, q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, stream);
+  return fa_fwd_ex(FA_DTYPE_BF16, q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, 0, stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
@@ -141,7 +152,7 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   return layout(nullptr, B, H, N, d).bytes;
 }
 
-fa_status fa_bwd_preprocess_typed(int dtype, const void* o, const void* dO, const float* lse, int B, int H, int N,
+fa_status fa_bwd_preprocess_ex(int dtype, const void* o, const void* dO, const float* lse, int B, int H, int N,
                                   int d, float scale, void* workspace, size_t workspace_bytes, void* stream) {
   if (!valid_dtype(dtype)) return FA_ERR_INVALID;
   if (!o || !dO || !lse) return FA_ERR_INVALID;
@@ -170,13 +181,14 @@ fa_status fa_bwd_preprocess_typed(int dtype, const void* o, const void* dO, cons
 
 fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int B, int H, int N, int d,
                             float scale, void* workspace, size_t workspace_bytes, void* stream) {
-  return fa_bwd_preprocess_typed(FA_DTYPE_BF16, o, dO, lse, B, H, N, d, scale, workspace, workspace_bytes, stream);
+  return fa_bwd_preprocess_ex(FA_DTYPE_BF16, o, dO, lse, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
 
-fa_status fa_bwd_main_typed(int dtype, const void* q, const void* k, const void* v, const void* dO, void* dk,
-                            void* dv, int B, int H, int N, int d, float scale, int causal,
-                            const uint8_t* block_mask, void* workspace, size_t workspace_bytes, void* stream) {
+fa_status fa_bwd_main_ex(int dtype, const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                         int B, int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
+                         long long block_mask_head_stride, void* workspace, size_t workspace_bytes, void* stream) {
   if (!valid_dtype(dtype)) return FA_ERR_INVALID;
+  if (!mask_stride_ok(block_mask, block_mask_head_stride, N)) return FA_ERR_INVALID;
   const int f16 = dtype == FA_DTYPE_F16;
   if (!q || !k || !v || !dO || !dk || !dv) return FA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) || !aligned16(dv))
@@ -201,6 +213,7 @@ fa_status fa_bwd_main_typed(int dtype, const void* q, const void* k, const void*
   p.lse2 = w.lse2;
   p.dq_acc = w.dq_acc;
   p.block_mask = block_mask;
+  p.mask_stride = block_mask_head_stride;
   p.N = N;
   p.Np = (N + 127) / 128 * 128;
   p.nb = (N + 127) / 128;
@@ -216,11 +229,11 @@ fa_status fa_bwd_main_typed(int dtype, const void* q, const void* k, const void*
 fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B,
                       int H, int N, int d, float scale, int causal, const uint8_t* block_mask, void* workspace,
                       size_t workspace_bytes, void* stream) {
-  return fa_bwd_main_typed(FA_DTYPE_BF16, q, k, v, dO, dk, dv, B, H, N, d, scale, causal, block_mask, workspace,
-                           workspace_bytes, stream);
+  return fa_bwd_main_ex(FA_DTYPE_BF16, q, k, v, dO, dk, dv, B, H, N, d, scale, causal, block_mask, 0, workspace,
+                        workspace_bytes, stream);
 }
 
-fa_status fa_bwd_dq_finish_typed(int dtype, void* dq, int B, int H, int N, int d, void* workspace,
+fa_status fa_bwd_dq_finish_ex(int dtype, void* dq, int B, int H, int N, int d, void* workspace,
                                  size_t workspace_bytes, void* stream) {
   if (!valid_dtype(dtype)) return FA_ERR_INVALID;
   if (!dq || !aligned16(dq)) return FA_ERR_INVALID;
@@ -243,29 +256,29 @@ fa_status fa_bwd_dq_finish_typed(int dtype, void* dq, int B, int H, int N, int d
 
 fa_status fa_bwd_dq_finish(void* dq, int B, int H, int N, int d, void* workspace, size_t workspace_bytes,
                            void* stream) {
-  return fa_bwd_dq_finish_typed(FA_DTYPE_BF16, dq, B, H, N, d, workspace, workspace_bytes, stream);
+  return fa_bwd_dq_finish_ex(FA_DTYPE_BF16, dq, B, H, N, d, workspace, workspace_bytes, stream);
 }
 
-fa_status fa_bwd_typed(int dtype, const void* q, const void* k, const void* v, const void* o, const void* dO,
-                       const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
-                       int causal, const uint8_t* block_mask, void* workspace, size_t workspace_bytes,
-                       void* stream) {
+fa_status fa_bwd_ex(int dtype, const void* q, const void* k, const void* v, const void* o, const void* dO,
+                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
+                    int causal, const uint8_t* block_mask, long long block_mask_head_stride, void* workspace,
+                    size_t workspace_bytes, void* stream) {
   if (!valid_dtype(dtype)) return FA_ERR_INVALID;
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID;
-  fa_status st =
-      fa_bwd_preprocess_typed(dtype, o, dO, lse, B, H, N, d, scale, workspace, workspace_bytes, stream);
+  if (!mask_stride_ok(block_mask, block_mask_head_stride, N)) return FA_ERR_INVALID;
+  fa_status st = fa_bwd_preprocess_ex(dtype, o, dO, lse, B, H, N, d, scale, workspace, workspace_bytes, stream);
   if (st != FA_OK) return st;
-  st = fa_bwd_main_typed(dtype, q, k, v, dO, dk, dv, B, H, N, d, scale, causal, block_mask, workspace,
-                         workspace_bytes, stream);
+  st = fa_bwd_main_ex(dtype, q, k, v, dO, dk, dv, B, H, N, d, scale, causal, block_mask, block_mask_head_stride,
+                      workspace, workspace_bytes, stream);
   if (st != FA_OK) return st;
-  return fa_bwd_dq_finish_typed(dtype, dq, B, H, N, d, workspace, workspace_bytes, stream);
+  return fa_bwd_dq_finish_ex(dtype, dq, B, H, N, d, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                  void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
                  const uint8_t* block_mask, void* workspace, size_t workspace_bytes, void* stream) {
-  return fa_bwd_typed(FA_DTYPE_BF16, q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, block_mask,
-                      workspace, workspace_bytes, stream);
+  return fa_bwd_ex(FA_DTYPE_BF16, q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, block_mask, 0,
+                   workspace, workspace_bytes, stream);
 }
 
 fa_status fa_last_device_status(void* stream) {

@@ -94,9 +94,10 @@ struct BwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-__device__ __forceinline__ bool bwd_tile_active(const BwdParams& p, int i, int j) {
+// bmask: this (b, h)'s block mask (or null).
+__device__ __forceinline__ bool bwd_tile_active(const BwdParams& p, const uint8_t* bmask, int i, int j) {
   if (p.causal && i < j) return false;
-  if (p.block_mask != nullptr && p.block_mask[i * p.nb + j] == 0) return false;
+  if (bmask != nullptr && bmask[i * p.nb + j] == 0) return false;
   return true;
 }
 
@@ -159,6 +160,7 @@ __global__ void __launch_bounds__(512, 1)
   AbortState* ab = reinterpret_cast<AbortState*>(smem + C::OFF_MISC + 4);
 
   const int bh = blockIdx.y;
+  const uint8_t* bmask = p.block_mask == nullptr ? nullptr : p.block_mask + (size_t)bh * p.mask_stride;
   const int j = blockIdx.x;  // key tile (causal: j = 0 has the most work and starts first)
   const int i_begin = p.causal ? j : 0;
   const uint64_t lim = p.timeout_ns;
@@ -216,7 +218,7 @@ __global__ void __launch_bounds__(512, 1)
       for (int s = 0; s < NS_DO; ++s) issued_do[s] = -1;
       bool ok = true;
       for (int i = i_begin; i < p.nb; ++i) {
-        if (!bwd_tile_active(p, i, j)) continue;
+        if (!bwd_tile_active(p, bmask, i, j)) continue;
         // Q_i first: its stage frees at dK_{i-NS}, before dO_i's stage frees at dV_{i-NS_DO}.
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
@@ -288,7 +290,7 @@ __global__ void __launch_bounds__(512, 1)
       };
 
       int i = i_begin;
-      while (i < p.nb && !bwd_tile_active(p, i, j)) ++i;
+      while (i < p.nb && !bwd_tile_active(p, bmask, i, j)) ++i;
       int it = 0;
       if (ok && i < p.nb) {
         ok = mbar_wait_spin(&bar_qf[0], 0, ab, lim, WAIT_BWD_MMA + 2);
@@ -307,7 +309,7 @@ __global__ void __launch_bounds__(512, 1)
       while (ok && i < p.nb) {
         const int s = it % NS;
         int inext = i + 1;
-        while (inext < p.nb && !bwd_tile_active(p, inext, j)) ++inext;
+        while (inext < p.nb && !bwd_tile_active(p, bmask, inext, j)) ++inext;
         const bool has_next = inext < p.nb;
         const int sn = (it + 1) % NS;
         const int sd = it % NS_DO, sdn = (it + 1) % NS_DO;
@@ -390,7 +392,7 @@ __global__ void __launch_bounds__(512, 1)
     bool ok = true;
     int it = 0;
     for (int i = i_begin; i < p.nb; ++i) {
-      if (!bwd_tile_active(p, i, j)) continue;
+      if (!bwd_tile_active(p, bmask, i, j)) continue;
       const int s = it % NS;
       const float* nlse2 = reinterpret_cast<const float*>(smem + C::OFF_LSE + s * 512) + 64 * h;
       const float* ndel = reinterpret_cast<const float*>(smem + C::OFF_DEL + s * 512) + 64 * h;
@@ -541,7 +543,7 @@ __global__ void __launch_bounds__(512, 1)
     int it = 0;
     uint32_t nred = 0;  // bulk reductions issued so far (staging slot = nred % DQ_SLOTS)
     for (int i = i_begin; i < p.nb; ++i) {
-      if (!bwd_tile_active(p, i, j)) continue;
+      if (!bwd_tile_active(p, bmask, i, j)) continue;
       ok = warp_wait(bar_dq, it & 1, ab, lim, WAIT_BWD_DQ + 1);
       // Read the whole row and release the TMEM columns before anything else (at d = 128 the
       // next dP^T is written there). When aborting (!ok) the values are not used; the columns

@@ -69,10 +69,11 @@ struct FwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-__device__ __forceinline__ bool fwd_tile_active(const FwdParams& p, int qb, int j) {
+// bmask: this (b, h)'s block mask (or null).
+__device__ __forceinline__ bool fwd_tile_active(const FwdParams& p, const uint8_t* bmask, int qb, int j) {
   if (qb >= p.nb) return false;
   if (p.causal && j > qb) return false;
-  if (p.block_mask != nullptr && p.block_mask[qb * p.nb + j] == 0) return false;
+  if (bmask != nullptr && bmask[qb * p.nb + j] == 0) return false;
   return true;
 }
 
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(384, 1)
   AbortState* ab = reinterpret_cast<AbortState*>(smem + C::OFF_MISC + 4);
 
   const int bh = blockIdx.y;
+  const uint8_t* bmask = p.block_mask == nullptr ? nullptr : p.block_mask + (size_t)bh * p.mask_stride;
   const int pair = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;  // heavy first
   const int qb0 = 2 * pair;  // 128-row tile index of tile 0
   const int j_end = p.causal ? min(p.nb, qb0 + 2) : p.nb;
@@ -211,7 +213,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int s = 0; s < NS; ++s) issued_k[s] = issued_v[s] = -1;
       bool ok = true;
       for (int j = 0; j < j_end && ok; ++j) {
-        if (!fwd_tile_active(p, qb0, j) && !fwd_tile_active(p, qb0 + 1, j)) continue;
+        if (!fwd_tile_active(p, bmask, qb0, j) && !fwd_tile_active(p, bmask, qb0 + 1, j)) continue;
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
         ok = mbar_wait(&bar_ke[s], ph ^ 1, ab, lim, WAIT_FWD_LOAD + 1);
@@ -265,7 +267,7 @@ __global__ void __launch_bounds__(384, 1)
       int it = 0;
 
       for (int j = 0; j < j_end && ok; ++j) {
-        const bool act0 = fwd_tile_active(p, qb0, j), act1 = fwd_tile_active(p, qb0 + 1, j);
+        const bool act0 = fwd_tile_active(p, bmask, qb0, j), act1 = fwd_tile_active(p, bmask, qb0 + 1, j);
         if (!act0 && !act1) continue;
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
@@ -364,7 +366,7 @@ __global__ void __launch_bounds__(384, 1)
 
     if (tvalid) {
       for (int j = 0; j < j_end; ++j) {
-        if (!fwd_tile_active(p, qb, j)) continue;
+        if (!fwd_tile_active(p, bmask, qb, j)) continue;
         ok = warp_wait(&bar_s[t], s_phase, ab, lim, WAIT_FWD_SOFTMAX + 1);
         if (!ok) break;
         s_phase ^= 1u;

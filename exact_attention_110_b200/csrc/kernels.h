@@ -25,8 +25,9 @@ enum WaitSite : int {
 
 struct FwdParams {
   float* lse;                  // [BH][N]
-  const uint8_t* block_mask;   // [nb][nb] or null
-  int N;                       // keys = queries per head (multiple of 128)
+  const uint8_t* block_mask;   // [nb][nb] (or one per (b, h), mask_stride apart) or null
+  long long mask_stride;       // elements between consecutive (b, h) masks; 0 = one shared mask
+  int N;                       // keys = queries per head
   int nb;                      // N / 128
   int causal;
   float scale_log2;            // scale * log2(e)
@@ -52,6 +53,7 @@ struct BwdParams {
   const float* lse2;     // [BH][Np]  -LSE * log2(e) + log2(scale)
   float* dq_acc;         // [BH][Np][D]
   const uint8_t* block_mask;
+  long long mask_stride; // elements between consecutive (b, h) masks; 0 = one shared mask
   int N, Np, nb;
   int causal;
   float inv_scale;       // 1 / scale (dV epilogue: P carries the scale)

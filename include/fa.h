@@ -54,7 +54,7 @@ typedef enum {
   FA_ERR_WORKSPACE = 5    /* workspace pointer null or smaller than fa_bwd_workspace_bytes */
 } fa_status;
 
-/* Element type of q, k, v, o, dO, dq, dk, dv for the *_typed entry points. */
+/* Element type of q, k, v, o, dO, dq, dk, dv for the *_ex entry points. */
 typedef enum {
   FA_DTYPE_BF16 = 0, /* bfloat16: the type of every untyped entry point */
   FA_DTYPE_F16 = 1   /* IEEE half; the kernels still compute S, P, O and gradients in fp32 */
@@ -131,30 +131,38 @@ fa_status fa_bwd_dq_finish(void* dq, int B, int H, int N, int d, void* workspace
  * re-initialises everything it reads from the array.
  */
 /*
- * The same calls for either 16-bit element type (dtype: an fa_dtype value, anything else
- * returns FA_ERR_INVALID). Arguments, layouts, workspace and errors as above; the tensor
- * operands of one call all have the element type `dtype` (lse and the workspace stay fp32).
+ * Extended forms of the calls above: the 16-bit element type and per-(b, h) block masks.
+ *   dtype: an fa_dtype value (anything else returns FA_ERR_INVALID); the tensor operands of
+ *          one call all have that element type (lse and the workspace stay fp32).
+ *   block_mask_head_stride: 0 = one ceil(N/128)^2 mask shared by every (b, h), as in the
+ *          calls above; otherwise the mask of head (b, h) starts at
+ *          block_mask + (b*H + h) * block_mask_head_stride (at least ceil(N/128)^2, else
+ *          FA_ERR_INVALID), so B*H masks can give every head its own sparsity pattern
+ *          ([P1] §Block-Sparse FlashAttention: the work scales with the blocks that are on).
+ *          The forward and fa_bwd_main of one problem must see the same masks.
+ * Arguments, layouts, workspace and errors are otherwise those of the plain calls.
  * The pages discuss fp16's narrow range for exp ([P2] §时间复杂度): here exponentials,
  * the softmax statistics and every accumulator are fp32 in both types, and P (bounded by
  * 2^8 by the reference-max rule) is the only 16-bit intermediate besides the inputs.
- * fa_bwd_noalloc is bf16 only.
+ * fa_bwd_noalloc is bf16 with a shared mask only.
  */
-fa_status fa_fwd_typed(int dtype, const void* q, const void* k, const void* v, void* o, float* lse,
-                       int B, int H, int N, int d, float scale, int causal,
-                       const uint8_t* block_mask, void* stream);
-fa_status fa_bwd_typed(int dtype, const void* q, const void* k, const void* v, const void* o,
-                       const void* dO, const float* lse, void* dq, void* dk, void* dv, int B, int H,
-                       int N, int d, float scale, int causal, const uint8_t* block_mask,
-                       void* workspace, size_t workspace_bytes, void* stream);
-fa_status fa_bwd_preprocess_typed(int dtype, const void* o, const void* dO, const float* lse, int B,
-                                  int H, int N, int d, float scale, void* workspace,
-                                  size_t workspace_bytes, void* stream);
-fa_status fa_bwd_main_typed(int dtype, const void* q, const void* k, const void* v, const void* dO,
-                            void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
-                            const uint8_t* block_mask, void* workspace, size_t workspace_bytes,
-                            void* stream);
-fa_status fa_bwd_dq_finish_typed(int dtype, void* dq, int B, int H, int N, int d, void* workspace,
-                                 size_t workspace_bytes, void* stream);
+fa_status fa_fwd_ex(int dtype, const void* q, const void* k, const void* v, void* o, float* lse,
+                    int B, int H, int N, int d, float scale, int causal,
+                    const uint8_t* block_mask, long long block_mask_head_stride, void* stream);
+fa_status fa_bwd_ex(int dtype, const void* q, const void* k, const void* v, const void* o,
+                    const void* dO, const float* lse, void* dq, void* dk, void* dv, int B, int H,
+                    int N, int d, float scale, int causal, const uint8_t* block_mask,
+                    long long block_mask_head_stride, void* workspace, size_t workspace_bytes,
+                    void* stream);
+fa_status fa_bwd_preprocess_ex(int dtype, const void* o, const void* dO, const float* lse, int B,
+                               int H, int N, int d, float scale, void* workspace,
+                               size_t workspace_bytes, void* stream);
+fa_status fa_bwd_main_ex(int dtype, const void* q, const void* k, const void* v, const void* dO,
+                         void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                         const uint8_t* block_mask, long long block_mask_head_stride,
+                         void* workspace, size_t workspace_bytes, void* stream);
+fa_status fa_bwd_dq_finish_ex(int dtype, void* dq, int B, int H, int N, int d, void* workspace,
+                              size_t workspace_bytes, void* stream);
 
 #define FA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,

@@ -80,18 +80,23 @@ def test_workspace_size_and_checks(lib):
     assert lib.fa_bwd_main(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 48, 0.1, 0, None, FAKE, need, None) == 2
 
 
-def test_typed_entry_points_check_dtype(lib):
+def test_ex_entry_points_check_dtype_and_mask_stride(lib):
     # the element type must be FA_DTYPE_BF16 (0) or FA_DTYPE_F16 (1); checked before anything else
     need = lib.fa_bwd_workspace_bytes(1, 1, 128, 64)
     for bad in (-1, 2, 7):
-        assert lib.fa_fwd_typed(bad, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0, None, None) == 1
-        assert lib.fa_bwd_typed(bad, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0,
-                                None, FAKE, need, None) == 1
-        assert lib.fa_bwd_dq_finish_typed(bad, FAKE, 1, 1, 128, 64, FAKE, need, None) == 1
+        assert lib.fa_fwd_ex(bad, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0, None, 0, None) == 1
+        assert lib.fa_bwd_ex(bad, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0,
+                             None, 0, FAKE, need, None) == 1
+        assert lib.fa_bwd_dq_finish_ex(bad, FAKE, 1, 1, 128, 64, FAKE, need, None) == 1
     # valid types still get the ordinary argument checks
     for dt in (0, 1):
-        assert lib.fa_fwd_typed(dt, None, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0, None, None) == 1
-        assert lib.fa_fwd_typed(dt, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 96, 0.125, 0, None, None) == 2
+        assert lib.fa_fwd_ex(dt, None, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.125, 0, None, 0, None) == 1
+        assert lib.fa_fwd_ex(dt, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 96, 0.125, 0, None, 0, None) == 2
+    # a per-head mask stride shorter than one ceil(N/128)^2 mask (here 3 x 3) is rejected
+    for stride in (1, 8, -9):
+        assert lib.fa_fwd_ex(0, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 300, 64, 0.125, 0, FAKE, stride, None) == 1
+        assert lib.fa_bwd_main_ex(0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 300, 64, 0.125, 0, FAKE, stride,
+                                  FAKE, lib.fa_bwd_workspace_bytes(1, 2, 300, 64), None) == 1
 
 
 @pytest.mark.parametrize("scale", [0.0, -0.125])

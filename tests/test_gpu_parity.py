@@ -83,7 +83,7 @@ def test_fwd_bwd_small(fa, oracle_mod, B, Hh, N, d, causal, mask):
 
 
 FP16 = [
-    # B, H, N, d, causal, mask: fp16 inputs and outputs through the *_typed entry points
+    # B, H, N, d, causal, mask: fp16 inputs and outputs through the *_ex entry points
     (1, 2, 384, 64, False, None),
     (2, 1, 640, 64, True, None),
     (1, 2, 512, 128, True, None),
@@ -106,6 +106,29 @@ def test_fwd_bwd_fp16(fa, oracle_mod, B, Hh, N, d, causal, mask):
     assert dq.dtype == dk.dtype == dv.dtype == torch.float16
     g_ref = oracle_mod.attention_bwd(ref["q"], ref["k"], ref["v"], ref["do"], scale, causal=causal, mask=m)[:3]
     H.assert_grads_close([H.to_f64(x) for x in (dq, dk, dv)], g_ref, f"fp16 bwd {B,Hh,N,d,causal,mask}")
+
+
+@pytest.mark.parametrize("B,Hh,N,d,causal", [(2, 2, 640, 64, False), (1, 3, 513, 128, True)])
+def test_per_head_block_masks(fa, oracle_mod, B, Hh, N, d, causal):
+    # Every (b, h) has its own Bernoulli mask, of a different density; each head must match the
+    # oracle run with that head's mask.
+    gpu, ref = H.make_case(B, Hh, N, d, seed=synth.BASE_SEED + 17 + N)
+    nb = (N + 127) // 128
+    masks = np.stack([synth.bernoulli_block_mask(synth.BASE_SEED + 100 + x, nb, p=0.15 + 0.2 * x)
+                      for x in range(B * Hh)]).reshape(B, Hh, nb, nb)
+    scale = 1.0 / np.sqrt(d)
+    mt = torch.from_numpy(masks).cuda()
+    o, lse = run_fwd(fa, gpu, causal, mt, scale)
+    dq, dk, dv = run_bwd(fa, gpu, o, lse, causal, mt, scale)
+    outs = [H.to_f64(x) for x in (o, lse, dq, dk, dv)]
+    for b in range(B):
+        for h in range(Hh):
+            sl = (slice(b, b + 1), slice(h, h + 1))
+            args = [ref[k][sl] for k in ("q", "k", "v")]
+            o_ref, l_ref = oracle_mod.attention_fwd(*args, scale, causal=causal, mask=masks[b, h])
+            H.assert_fwd_close(outs[0][sl], outs[1][sl], o_ref, l_ref, f"head {b},{h}")
+            g_ref = oracle_mod.attention_bwd(*args, ref["do"][sl], scale, causal=causal, mask=masks[b, h])[:3]
+            H.assert_grads_close([x[sl] for x in outs[2:]], g_ref, f"head {b},{h}")
 
 
 def test_fp16_and_bf16_agree(fa):
