@@ -49,6 +49,7 @@ def _load():
                                         ctypes.POINTER(ctypes.c_int), i32, dp, dp]
         lib.oracle_bwd.argtypes = [dp, dp, dp, dp, i64, i32, i32, f64, i32, u8p, i32, dp, dp, dp, dp]
         lib.oracle_online_fwd.argtypes = [dp, dp, dp, i64, i32, i32, f64, i32, u8p, i32, i32, i32, dp, dp]
+        lib.oracle_fwd_qk.argtypes = [dp, dp, dp, i64, i32, i32, i32, f64, i32, dp, dp]
         _lib = lib
     return _lib
 
@@ -91,6 +92,20 @@ def attention_fwd(q, k, v, scale: float, causal: bool = False, mask=None, mask_b
     m, mp = _mask_arg(mask, N, mask_bs)
     _load().oracle_fwd(_ptr(q), _ptr(k), _ptr(v), B * H, N, d, float(scale), int(causal), mp,
                        mask_bs, _ptr(o), _ptr(lse))
+    return o, lse
+
+
+def attention_fwd_qk(q, k, v, scale: float, causal: bool = False):
+    """General shapes: q [B, H, Nq, d] against k, v [B, H, Nk, d] (bottom-right causal
+    alignment: key j visible to query i iff j <= i + Nk - Nq). Returns (O, LSE)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, d = _shape(q)
+    Nk = k.shape[2]
+    if k.shape != (B, H, Nk, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, H, Nk, d] with q's B, H and d")
+    o = np.empty_like(q)
+    lse = np.empty((B, H, Nq), dtype=np.float64)
+    _load().oracle_fwd_qk(_ptr(q), _ptr(k), _ptr(v), B * H, Nq, Nk, d, float(scale), int(causal), _ptr(o), _ptr(lse))
     return o, lse
 
 

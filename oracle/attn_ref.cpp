@@ -20,6 +20,10 @@
 //   (causal: [P1] benchmark setting "with or without causal mask"; block mask: [P1] §Block-Sparse).
 // A row with no allowed key has O_i = 0 and LSE_i = -inf (a reading; the pages are silent).
 //
+// General shapes (oracle_fwd_qk): N_q query rows against N_k keys per head. The pages only
+// treat N_q = N_k; the reading taken is the bottom-right alignment, where the last query row
+// sees every key: causal allows j <= i + (N_k - N_q), which is j <= i when N_q = N_k.
+//
 // Backward with upstream gradient dO. The pages only say that the backward recomputes S and
 // P from the saved statistics and goes through the softmax Jacobian ([P3] §4.1, §4.2); the
 // formulas below are the textbook chain rule through steps above:
@@ -51,8 +55,9 @@ struct Mask {
   const uint8_t* blocks;  // nullable, [nb][nb] row-major
   int nb;                 // blocks per side
   int bs;                 // block size in rows/keys
+  int off = 0;            // causal alignment: key j visible to query i iff j <= i + off
   bool allowed(int i, int j) const {
-    if (causal && j > i) return false;
+    if (causal && j > i + off) return false;
     if (blocks && blocks[(int64_t)(i / bs) * nb + (j / bs)] == 0) return false;
     return true;
   }
@@ -132,6 +137,36 @@ void oracle_fwd(const double* q, const double* k, const double* v, int64_t BH, i
         double* oi = oh + (int64_t)i * d;
         for (int t = 0; t < d; ++t) oi[t] = 0.0;
         for (int j = 0; j < N; ++j) {
+          if (p_row[j] == 0.0) continue;
+          const double* vj = vh + (int64_t)j * d;
+          for (int t = 0; t < d; ++t) oi[t] += p_row[j] * vj[t];
+        }
+      }
+    }
+  }
+}
+
+// Forward for general shapes: q, o: [BH][Nq][d]; k, v: [BH][Nk][d]; lse: [BH][Nq]. No block
+// mask; causal uses the bottom-right alignment described at the top of this file.
+void oracle_fwd_qk(const double* q, const double* k, const double* v, int64_t BH, int Nq, int Nk, int d,
+                   double scale, int causal, double* o, double* lse) {
+  Mask mk = make_mask(Nk, causal, nullptr, 128);
+  mk.off = Nk - Nq;
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    const double* qh = q + bh * Nq * d;
+    const double* kh = k + bh * Nk * d;
+    const double* vh = v + bh * Nk * d;
+    double* oh = o + bh * Nq * d;
+    double* lh = lse + bh * Nq;
+#pragma omp parallel
+    {
+      std::vector<double> s_row(Nk), p_row(Nk);
+#pragma omp for schedule(dynamic, 4)
+      for (int i = 0; i < Nq; ++i) {
+        lh[i] = softmax_row(qh + (int64_t)i * d, kh, Nk, d, scale, mk, i, s_row.data(), p_row.data());
+        double* oi = oh + (int64_t)i * d;
+        for (int t = 0; t < d; ++t) oi[t] = 0.0;
+        for (int j = 0; j < Nk; ++j) {
           if (p_row[j] == 0.0) continue;
           const double* vj = vh + (int64_t)j * d;
           for (int t = 0; t < d; ++t) oi[t] += p_row[j] * vj[t];

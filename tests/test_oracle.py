@@ -284,3 +284,67 @@ def test_bf16_inputs_are_exact_in_fp64():
     f = synth.bf16_bits_to_f32(bits).astype(np.float64)
     assert np.array_equal(synth.f32_to_bf16_bits(f.astype(np.float32)), bits)
     assert abs(f.mean()) < 0.15 and abs(f.std() - 1.0) < 0.1
+
+
+# ---------------------------------------------------------------------------------------
+# General shapes (N_q queries against N_k keys) and the split-KV combine
+# ---------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_general_shapes_reduce_to_square(oracle_mod, causal):
+    # N_q = N_k: the offset is zero and the result is the square oracle's
+    q, k, v = rnd((1, 2, 45, 8), 60), rnd((1, 2, 45, 8), 61), rnd((1, 2, 45, 8), 62)
+    o1, l1 = oracle_mod.attention_fwd_qk(q, k, v, 0.4, causal=causal)
+    o2, l2 = oracle_mod.attention_fwd(q, k, v, 0.4, causal=causal)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+
+
+def test_bottom_right_causal_is_the_suffix_of_the_square_problem(oracle_mod):
+    # The last N_q rows of a square causal problem see exactly the keys the bottom-right
+    # alignment gives N_q queries against the same N_k keys.
+    N, nq = 53, 7
+    q, k, v = rnd((2, 1, N, 8), 63), rnd((2, 1, N, 8), 64), rnd((2, 1, N, 8), 65)
+    o_sq, l_sq = oracle_mod.attention_fwd(q, k, v, 0.3, causal=True)
+    o, l = oracle_mod.attention_fwd_qk(q[:, :, N - nq:], k, v, 0.3, causal=True)
+    np.testing.assert_allclose(o, o_sq[:, :, N - nq:], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(l, l_sq[:, :, N - nq:], rtol=1e-13, atol=1e-14)
+
+
+def test_general_shapes_match_scipy(oracle_mod):
+    # N_q != N_k against a library softmax over the explicitly built allowed matrix
+    nq, nk, d = 9, 40, 6
+    q, k, v = rnd((1, 2, nq, d), 66), rnd((1, 2, nk, d), 67), rnd((1, 2, nk, d), 68)
+    for causal in (False, True):
+        o, l = oracle_mod.attention_fwd_qk(q, k, v, 0.5, causal=causal)
+        i = np.arange(nq)[:, None]
+        j = np.arange(nk)[None, :]
+        allowed = (j <= i + (nk - nq)) if causal else np.ones((nq, nk), dtype=bool)
+        for h in range(2):
+            s = np.where(allowed, 0.5 * q[0, h] @ k[0, h].T, -np.inf)
+            np.testing.assert_allclose(o[0, h], scipy.special.softmax(s, axis=1) @ v[0, h], rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(l[0, h], scipy.special.logsumexp(s, axis=1), rtol=1e-13, atol=1e-13)
+
+
+def test_more_queries_than_keys_causal_rows_see_nothing(oracle_mod):
+    # bottom-right alignment with N_q > N_k: the first N_q - N_k rows have no visible key
+    q, k, v = rnd((1, 1, 10, 4), 69), rnd((1, 1, 6, 4), 70), rnd((1, 1, 6, 4), 71)
+    o, l = oracle_mod.attention_fwd_qk(q, k, v, 0.5, causal=True)
+    assert np.all(o[0, 0, :4] == 0) and np.all(np.isneginf(l[0, 0, :4]))
+    assert np.all(np.isfinite(l[0, 0, 4:]))
+
+
+def test_split_keys_and_merge_by_lse_equals_full(oracle_mod):
+    # The split-KV forward computes (O_s, LSE_s) on key chunks and combines them with
+    # LSE = log sum_s exp(LSE_s), O = sum_s exp(LSE_s - LSE) O_s: the online normaliser's
+    # combine step, here checked against the unsplit result in fp64.
+    nq, nk, d = 5, 300, 8
+    q, k, v = rnd((1, 2, nq, d), 72), rnd((1, 2, nk, d), 73), rnd((1, 2, nk, d), 74)
+    o_full, l_full = oracle_mod.attention_fwd_qk(q, k, v, 0.35)
+    cuts = [0, 64, 65, 190, 300]  # uneven chunks, one of a single key
+    parts = [oracle_mod.attention_fwd_qk(q, k[:, :, a:b], v[:, :, a:b], 0.35) for a, b in zip(cuts, cuts[1:])]
+    ls = np.stack([p[1] for p in parts])
+    lse = scipy.special.logsumexp(ls, axis=0)
+    o = sum(np.exp(p[1] - lse)[..., None] * p[0] for p in parts)
+    np.testing.assert_allclose(o, o_full, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, l_full, rtol=1e-13, atol=1e-13)
