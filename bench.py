@@ -8,7 +8,7 @@ inputs from the seeded generator. Prints ONE JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--seqlen N] [--headdim d]
                     [--causal] [--block-sparse [--block-density P]] [--dtype bf16|f16]
-                    [--impl reference] [--sweep] [--density-sweep]
+                    [--impl reference] [--sweep] [--density-sweep] [--decode NQ]
 
 Metric: fwd+bwd TFLOPS with FLOPs counted as 4*B*H*N^2*d for the forward (halved for causal,
 scaled by block density for block-sparse) and 2.5x that for the backward.
@@ -203,6 +203,60 @@ def run_reference(args, wl, rank, world):
     return 0
 
 
+# ----------------------------------------------------------------------------- decode arm
+def run_decode(args, rank, world, local_rank, dist_on):
+    """Decode-shaped forward: args.decode queries per head against --seqlen keys, B=8, H=16
+    (hidden 2048 at d=128), split over the key range and merged. HBM-bound: the metric is the
+    K/V bytes read per second against the measured HBM copy bandwidth."""
+    import torch
+    import exact_attention_110_b200 as fa
+    import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    B, H, nq, nk, d = 8, HIDDEN // args.headdim, args.decode, args.seqlen, args.headdim
+    seed = synth.BASE_SEED + 97 * rank
+    q = synth.to_torch(_stream(seed + synth.SEED_Q, B * H * nq * d, args.dtype).reshape(B, H, nq, d), args.dtype, dev)
+    k, v = (synth.to_torch(_stream(seed + o, B * H * nk * d, args.dtype).reshape(B, H, nk, d), args.dtype, dev)
+            for o in (synth.SEED_K, synth.SEED_V))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, nq), device=dev, dtype=torch.float32)
+    need = int(fa.library().fa_fwd_decode_workspace_bytes(B, H, nq, nk, d, 0))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        fa.forward_decode(q, k, v, causal=args.causal, out=o, lse=lse, workspace=ws)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist_on:
+        torch.distributed.barrier()
+    with ClockSampler(physical_gpu(local_rank)) as clk:
+        time.sleep(0.3)
+        start.record()
+        for _ in range(args.steps):
+            fa.forward_decode(q, k, v, causal=args.causal, out=o, lse=lse, workspace=ws)
+        end.record()
+        torch.cuda.synchronize()
+    if fa.last_device_status(dev) != 0:
+        raise RuntimeError("device wait timed out")
+    ms = reduce_max(start.elapsed_time(end), dist_on, dev) / args.steps
+    kv_bytes = 2 * B * H * nk * d * 2
+    peaks = load_peaks()
+    gbs = world * kv_bytes / (ms * 1e-3) / 1e9
+    line = {"metric": "decode forward K/V read bandwidth", "value": gbs, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+            "config": {"workload": f"decode B={B} H={H} Nq={nq} Nk={nk} d={d} "
+                                   f"{'causal' if args.causal else 'non-causal'}, split keys (library's choice)",
+                       "workspace_bytes": need},
+            "tflops": world * fwd_flops(B, H, 1, d) * nq * nk / (ms * 1e-3) / 1e12,
+            "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / world / peaks["hbm_gbs"], "traffic": None, "kernel": "fa_fwd_kernel"},
+            "gpu_launches": args.steps * (2 if need > 0 else 1), "clocks": clk.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- GPU arm
 @functools.lru_cache(maxsize=4)
 def _stream(seed: int, n: int, dtype: str = "bf16"):
@@ -382,6 +436,8 @@ def main(argv=None):
                     help="with --block-sparse: probability that an off-diagonal 128x128 block is on")
     ap.add_argument("--density-sweep", action="store_true",
                     help="block-sparse config at densities 0.05..1: runtime should follow the blocks that are on")
+    ap.add_argument("--decode", type=int, default=0, metavar="NQ",
+                    help="decode-shaped forward: NQ queries per head against --seqlen keys (B=8)")
     ap.add_argument("--dtype", choices=["bf16", "f16"], default="bf16",
                     help="element type of q, k, v, o, dO and the gradients (fp32 accumulation either way)")
     args = ap.parse_args(argv)
@@ -403,6 +459,8 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.decode > 0:
+            return run_decode(args, rank, world, local_rank, dist_on)
         if args.density_sweep:
             args.no_cpu_baseline, args.no_e2e = True, True
             for p_on in (0.05, 0.1, 0.25, 0.5, 1.0):

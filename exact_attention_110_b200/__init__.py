@@ -7,6 +7,7 @@ the library is missing, every call raises -- there is no fallback implementation
 
     o, lse = forward(q, k, v, causal=False, block_mask=None, scale=None)
     dq, dk, dv = backward(q, k, v, o, do, lse, causal=False, block_mask=None, scale=None)
+    o, lse = forward_decode(q, k, v, causal=False, scale=None, num_splits=0)   # Nq != Nk
 
 q, k, v, o, do: bf16 (or fp16) CUDA tensors [B, H, N, d] of one type, contiguous, d in {64, 128},
 any N >= 1.
@@ -22,7 +23,7 @@ from pathlib import Path
 import torch
 
 __all__ = [
-    "FAError", "forward", "backward", "bwd_workspace_bytes", "bwd_preprocess", "bwd_main",
+    "FAError", "forward", "forward_decode", "backward", "bwd_workspace_bytes", "bwd_preprocess", "bwd_main",
     "bwd_dq_finish", "last_device_status", "selftest_wait_timeout", "library", "LIB_PATH",
 ]
 
@@ -77,6 +78,10 @@ def library() -> ctypes.CDLL:
         lib.fa_bwd_main_ex.argtypes = [i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, vp, i64, vp, sz, vp]
         lib.fa_bwd_dq_finish_ex.restype = i32
         lib.fa_bwd_dq_finish_ex.argtypes = [i32] + list(lib.fa_bwd_dq_finish.argtypes)
+        lib.fa_fwd_decode_workspace_bytes.restype = sz
+        lib.fa_fwd_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
+        lib.fa_fwd_decode.restype = i32
+        lib.fa_fwd_decode.argtypes = [i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32, i32, vp, sz, vp]
         lib.fa_last_device_status.restype = i32
         lib.fa_last_device_status.argtypes = [vp]
         lib.fa_selftest_wait_timeout.restype = i32
@@ -145,6 +150,35 @@ def forward(q, k, v, causal: bool = False, block_mask=None, scale=None, out=None
     l = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
     _check(library().fa_fwd_ex(_DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, N, d,
                                _scale(scale, d), int(bool(causal)), _ptr(mask), mstride, _stream(q.device)), "fa_fwd")
+    return o, l
+
+
+def forward_decode(q, k, v, causal: bool = False, scale=None, num_splits: int = 0, out=None, lse=None,
+                   workspace=None):
+    """Nq queries against Nk keys per head (q [B, H, Nq, d]; k, v [B, H, Nk, d]), the key range
+    split over num_splits thread blocks (0: chosen by the library) and merged by LSE. causal
+    uses the bottom-right alignment (key j visible to query i iff j <= i + Nk - Nq)."""
+    if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape:
+        raise ValueError("q: [B, H, Nq, d]; k, v: [B, H, Nk, d]")
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if k.shape[:2] != (B, H) or k.shape[3] != d:
+        raise ValueError("k and v must share q's B, H and d")
+    for t in (q, k, v):
+        if not t.is_cuda or t.dtype != q.dtype or not t.is_contiguous() or t.device != q.device:
+            raise ValueError("q, k, v must be contiguous CUDA tensors of one type and device")
+    if q.dtype not in _DTYPES:
+        raise ValueError("q, k, v must be bf16 or fp16")
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, Nq), device=q.device, dtype=torch.float32) if lse is None else lse
+    lib = library()
+    need = int(lib.fa_fwd_decode_workspace_bytes(B, H, Nq, Nk, d, int(num_splits)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.fa_fwd_decode(_DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, H, Nq, Nk, d,
+                             _scale(scale, d), int(bool(causal)), int(num_splits), _ptr(workspace), nbytes,
+                             _stream(q.device)), "fa_fwd_decode")
     return o, l
 
 

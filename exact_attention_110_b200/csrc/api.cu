@@ -135,6 +135,14 @@ fa_status fa_fwd_ex(int dtype, const void* q, const void* k, const void* v, void
   p.mask_stride = block_mask_head_stride;
   p.N = N;
   p.nb = (N + 127) / 128;  // the last tile may be partial: TMA zero-fills rows >= N
+  p.Nk = N;
+  p.nbk = p.nb;
+  p.causal_off = 0;
+  p.nsplit = 1;
+  p.kv_per_split = p.nbk;
+  p.Np = p.nb * 128;
+  p.o_part = nullptr;
+  p.lse_part = nullptr;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
@@ -145,6 +153,112 @@ fa_status fa_fwd_ex(int dtype, const void* q, const void* k, const void* v, void
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                  float scale, int causal, const uint8_t* block_mask, void* stream) {
   return fa_fwd_ex(FA_DTYPE_BF16, q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, 0, stream);
+}
+
+// ------------------------------------------------------------------------- decode-shaped forward
+namespace {
+
+// Key-range splits for the decode forward: enough thread blocks for about three quarters of
+// a wave (measured: with 128 query-tile pairs one piece streams K/V faster than three, the
+// partial writes and the merge cost more than the idle SMs), but at least two key tiles per
+// split; an explicit request is only capped by the number of key tiles.
+int decode_splits(long long BH, int Nq, int Nk, int requested) {
+  const int nbk = (Nk + 127) / 128;
+  if (requested > 0) return requested < nbk ? requested : nbk;
+  const long long pairs = BH * (((Nq + 127) / 128 + 1) / 2);
+  const long long target = 3ll * fa::device_sm_count() / 4;
+  long long s = (target + pairs - 1) / pairs;
+  const long long cap = nbk / 2 > 1 ? nbk / 2 : 1;
+  if (s > cap) s = cap;
+  return s < 1 ? 1 : (int)s;
+}
+
+struct DecodeWorkspace {
+  float* o_part;
+  float* lse_part;
+  size_t bytes;
+};
+
+DecodeWorkspace decode_layout(void* base, long long BH, int Nq, int d, int nsplit) {
+  const size_t Np = ((size_t)Nq + 127) / 128 * 128;
+  const size_t s_o = align256((size_t)BH * nsplit * Np * d * sizeof(float));
+  const size_t s_l = align256((size_t)BH * nsplit * Np * sizeof(float));
+  DecodeWorkspace w;
+  char* c = static_cast<char*>(base);
+  w.o_part = reinterpret_cast<float*>(c);
+  w.lse_part = reinterpret_cast<float*>(c + s_o);
+  w.bytes = nsplit > 1 ? s_o + s_l : 0;
+  return w;
+}
+
+fa_status check_decode(int B, int H, int Nq, int Nk, int d, float scale, int nsplit) {
+  if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || nsplit < 0 || !isfinite(scale)) return FA_ERR_INVALID;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH > 65535) return FA_ERR_UNSUPPORTED;
+  if ((long long)Nq * d > (1ll << 31) / 2 || (long long)Nk * d > (1ll << 31) / 2) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+}  // namespace
+
+size_t fa_fwd_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d, int nsplit) {
+  if (check_decode(B, H, Nq, Nk, d, 1.0f, nsplit) != FA_OK) return 0;
+  const long long BH = (long long)B * H;
+  return decode_layout(nullptr, BH, Nq, d, decode_splits(BH, Nq, Nk, nsplit)).bytes;
+}
+
+fa_status fa_fwd_decode(int dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                        int Nq, int Nk, int d, float scale, int causal, int nsplit, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (!valid_dtype(dtype)) return FA_ERR_INVALID;
+  const int f16 = dtype == FA_DTYPE_F16;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID;
+  fa_status st = check_decode(B, H, Nq, Nk, d, scale, nsplit);
+  if (st != FA_OK) return st;
+  const long long BH = (long long)B * H;
+  const int ns = decode_splits(BH, Nq, Nk, nsplit);
+  DecodeWorkspace w = decode_layout(workspace, BH, Nq, d, ns);
+  if (ns > 1 && (!workspace || !aligned16(workspace) || workspace_bytes < w.bytes)) return FA_ERR_WORKSPACE;
+  if (!get_encoder()) return FA_ERR_CUDA;
+  alignas(64) CUtensorMap tq, tk, tv, to;
+  if (!encode_bhnd(&tq, q, BH, Nq, d, f16) || !encode_bhnd(&tk, k, BH, Nk, d, f16) ||
+      !encode_bhnd(&tv, v, BH, Nk, d, f16) || !encode_bhnd(&to, o, BH, Nq, d, f16))
+    return FA_ERR_CUDA;
+  fa::FwdParams p;
+  p.lse = lse;
+  p.block_mask = nullptr;
+  p.mask_stride = 0;
+  p.N = Nq;
+  p.nb = (Nq + 127) / 128;
+  p.Nk = Nk;
+  p.nbk = (Nk + 127) / 128;
+  p.causal_off = Nk - Nq;  // bottom-right alignment: the last query sees every key
+  p.nsplit = ns;
+  p.kv_per_split = (p.nbk + ns - 1) / ns;
+  p.Np = p.nb * 128;
+  p.o_part = ns > 1 ? w.o_part : nullptr;
+  p.lse_part = ns > 1 ? w.lse_part : nullptr;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = kWaitLimitNs;
+  p.f16 = f16;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = fa::launch_fwd(d, tq, tk, tv, to, p, (int)BH, s);
+  if (e != cudaSuccess || ns == 1) return from_cuda(e);
+  fa::FwdMergeParams m;
+  m.o_part = w.o_part;
+  m.lse_part = w.lse_part;
+  m.o = static_cast<uint16_t*>(o);
+  m.lse = lse;
+  m.rows = BH * Nq;
+  m.N = Nq;
+  m.Np = p.Np;
+  m.nsplit = ns;
+  m.D = d;
+  m.f16 = f16;
+  return from_cuda(fa::launch_fwd_merge(m, s));
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {

@@ -81,19 +81,9 @@ __global__ void __launch_bounds__(256) fa_dq_finish_kernel(const DqFinishParams 
   }
 }
 
-static int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
 
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream) {
-  const int grid = sm_count() * 8;  // 8 resident 256-thread blocks per SM
+  const int grid = device_sm_count() * 8;  // 8 resident 256-thread blocks per SM
   if (p.D == 64)
     p.f16 ? fa_bwd_pre_kernel<64, true><<<grid, 256, 0, stream>>>(p) : fa_bwd_pre_kernel<64, false><<<grid, 256, 0, stream>>>(p);
   else
@@ -103,7 +93,7 @@ cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_dq_finish(const DqFinishParams& p, cudaStream_t stream) {
-  const int grid = sm_count() * 8;
+  const int grid = device_sm_count() * 8;
   if (p.D == 64)
     p.f16 ? fa_dq_finish_kernel<64, true><<<grid, 256, 0, stream>>>(p)
           : fa_dq_finish_kernel<64, false><<<grid, 256, 0, stream>>>(p);

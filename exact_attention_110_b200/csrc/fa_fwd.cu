@@ -69,11 +69,12 @@ struct FwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// bmask: this (b, h)'s block mask (or null).
+// bmask: this (b, h)'s block mask (or null). Causal: tile j is active when the last row of
+// tile qb sees its first key (128j <= 128qb + 127 + causal_off; j <= qb for the square problem).
 __device__ __forceinline__ bool fwd_tile_active(const FwdParams& p, const uint8_t* bmask, int qb, int j) {
   if (qb >= p.nb) return false;
-  if (p.causal && j > qb) return false;
-  if (bmask != nullptr && bmask[qb * p.nb + j] == 0) return false;
+  if (p.causal && 128 * j > 128 * qb + 127 + p.causal_off) return false;
+  if (bmask != nullptr && bmask[qb * p.nbk + j] == 0) return false;
   return true;
 }
 
@@ -155,9 +156,18 @@ __global__ void __launch_bounds__(384, 1)
 
   const int bh = blockIdx.y;
   const uint8_t* bmask = p.block_mask == nullptr ? nullptr : p.block_mask + (size_t)bh * p.mask_stride;
-  const int pair = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;  // heavy first
+  // blockIdx.x = pair index * nsplit + split; causal grids start with the heaviest pairs
+  const int pi = (int)blockIdx.x / p.nsplit, split = (int)blockIdx.x - pi * p.nsplit;
+  const int npairs = (int)gridDim.x / p.nsplit;
+  const int pair = p.causal ? npairs - 1 - pi : pi;
   const int qb0 = 2 * pair;  // 128-row tile index of tile 0
-  const int j_end = p.causal ? min(p.nb, qb0 + 2) : p.nb;
+  // this CTA's key tiles: its split's range, cut at the last key the pair's last row sees
+  const int j_begin = split * p.kv_per_split;
+  int j_end = min(p.nbk, j_begin + p.kv_per_split);
+  if (p.causal) {
+    const int last_key = 128 * qb0 + 255 + p.causal_off;
+    j_end = min(j_end, last_key < 0 ? 0 : last_key / 128 + 1);
+  }
   const uint64_t lim = p.timeout_ns;
 
   if (warp == 0 && lane == 0) {
@@ -212,7 +222,7 @@ __global__ void __launch_bounds__(384, 1)
       int issued_k[NS], issued_v[NS];
       for (int s = 0; s < NS; ++s) issued_k[s] = issued_v[s] = -1;
       bool ok = true;
-      for (int j = 0; j < j_end && ok; ++j) {
+      for (int j = j_begin; j < j_end && ok; ++j) {
         if (!fwd_tile_active(p, bmask, qb0, j) && !fwd_tile_active(p, bmask, qb0 + 1, j)) continue;
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
@@ -266,7 +276,7 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t prev_ph = 0;
       int it = 0;
 
-      for (int j = 0; j < j_end && ok; ++j) {
+      for (int j = j_begin; j < j_end && ok; ++j) {
         const bool act0 = fwd_tile_active(p, bmask, qb0, j), act1 = fwd_tile_active(p, bmask, qb0 + 1, j);
         if (!act0 && !act1) continue;
         const int s = it % NS;
@@ -365,7 +375,7 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
 
     if (tvalid) {
-      for (int j = 0; j < j_end; ++j) {
+      for (int j = j_begin; j < j_end; ++j) {
         if (!fwd_tile_active(p, bmask, qb, j)) continue;
         ok = warp_wait(&bar_s[t], s_phase, ab, lim, WAIT_FWD_SOFTMAX + 1);
         if (!ok) break;
@@ -374,11 +384,13 @@ __global__ void __launch_bounds__(384, 1)
 
         uint32_t su[128];  // this row's 128 scores (fp32 bits)
         tmem_ld128(tS_row, su);
-        // Elementwise mask: on the causal diagonal key 128j+c is visible to row 128qb+r iff
-        // c <= r; in a partial last key tile keys 128j+c >= N do not exist (TMA filled zeros).
-        const bool masked = (p.causal && j == qb) || (128 * j + 128 > p.N);
+        // Elementwise mask: on the causal diagonal band key 128j+c is visible to row 128qb+r iff
+        // 128j+c <= 128qb+r+causal_off (c <= r for the square problem); in a partial last key
+        // tile keys 128j+c >= Nk do not exist (TMA filled zeros).
+        const bool diag = p.causal && (128 * j + 127 > 128 * qb + p.causal_off);
+        const bool masked = diag || (128 * j + 128 > p.Nk);
         if (masked) {
-          const int lim = min((p.causal && j == qb) ? r + 1 : 128, p.N - 128 * j);
+          const int lim = min(diag ? 128 * (qb - j) + r + p.causal_off + 1 : 128, p.Nk - 128 * j);
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c >= lim) su[c] = 0xff800000u;  // -inf
@@ -453,12 +465,34 @@ __global__ void __launch_bounds__(384, 1)
         }
         fence_proxy_async_smem();
         const int row = qb * 128 + r;
-        if (row < p.N)  // rows of a partial last tile beyond N are not stored (the O store clips them)
-          p.lse[(size_t)bh * p.N + row] = (l > 0.f) ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        const float lse_row = (l > 0.f) ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (p.nsplit > 1) {
+          // Split of the key range: this split's O / l (fp32, re-read from TMEM) and LSE for the
+          // merge kernel, every row of the tile (the buffers are padded to Np).
+          const size_t prow = ((size_t)bh * p.nsplit + split) * p.Np + row;
+          float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D);
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t u[32];
+            if (o_started) {
+              tmem_ld32(tO_row + c * 32, u);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) u[i] = 0u;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[c * 8 + q] = make_float4(__uint_as_float(u[4 * q]) * inv_l, __uint_as_float(u[4 * q + 1]) * inv_l,
+                                           __uint_as_float(u[4 * q + 2]) * inv_l, __uint_as_float(u[4 * q + 3]) * inv_l);
+          }
+          p.lse_part[prow] = lse_row;
+        } else if (row < p.N) {  // rows of a partial last tile beyond N are not stored (the O store clips them)
+          p.lse[(size_t)bh * p.N + row] = lse_row;
+        }
       }
       // Every thread of the warpgroup reaches this barrier (tvalid is uniform per warpgroup).
       named_bar_sync(1 + t, 128);
-      if (wq == 0 && lane == 0 && *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
+      if (p.nsplit == 1 && wq == 0 && lane == 0 && *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
         for (int pn = 0; pn < C::PANELS; ++pn) tma_store_3d(&tmO, stage + pn * C::PANEL_BYTES, pn * 64, qb * 128, bh);
         bulk_commit_group();
         bulk_wait_group_read0();
@@ -482,7 +516,7 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   cudaError_t e =
       cudaFuncSetAttribute(fa_fwd_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.nb + 1) / 2, BH);
+  dim3 grid((p.nb + 1) / 2 * p.nsplit, BH);
   fa_fwd_kernel<D, F16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }

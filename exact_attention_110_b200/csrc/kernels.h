@@ -27,8 +27,16 @@ struct FwdParams {
   float* lse;                  // [BH][N]
   const uint8_t* block_mask;   // [nb][nb] (or one per (b, h), mask_stride apart) or null
   long long mask_stride;       // elements between consecutive (b, h) masks; 0 = one shared mask
-  int N;                       // keys = queries per head
-  int nb;                      // N / 128
+  int N;                       // query rows per head
+  int nb;                      // ceil(N / 128) query tiles
+  int Nk;                      // keys per head (N for the square problem)
+  int nbk;                     // ceil(Nk / 128) key tiles
+  int causal_off;              // causal: key j is visible to query i iff j <= i + causal_off
+  int nsplit;                  // key-range splits per pair of query tiles (1: no split)
+  int kv_per_split;            // key tiles per split
+  int Np;                      // N rounded up to 128 (rows of the split partials)
+  float* o_part;               // nsplit > 1: fp32 [BH][nsplit][Np][D], each split's O / l
+  float* lse_part;             // nsplit > 1: fp32 [BH][nsplit][Np], each split's LSE
   int causal;
   float scale_log2;            // scale * log2(e)
   unsigned long long timeout_ns;
@@ -62,6 +70,16 @@ struct BwdParams {
   int f16;               // element type: fp16 if non-zero, bf16 otherwise
 };
 
+struct FwdMergeParams {
+  const float* o_part;   // [BH][nsplit][Np][D]
+  const float* lse_part; // [BH][nsplit][Np]
+  uint16_t* o;           // bf16 / fp16 [BH][N][D]
+  float* lse;            // [BH][N]
+  long long rows;        // BH * N
+  int N, Np, nsplit, D;
+  int f16;
+};
+
 struct DqFinishParams {
   const float* dq_acc;   // [BH][Np][D]
   uint16_t* dq;          // bf16 [BH][N][D]
@@ -71,9 +89,24 @@ struct DqFinishParams {
   int f16;               // element type: fp16 if non-zero, bf16 otherwise
 };
 
+// Streaming multiprocessors of the current device (cached per device ordinal).
+inline int device_sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] <= 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
 // Launchers (return the launch error, if any).
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream);
+cudaError_t launch_fwd_merge(const FwdMergeParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,

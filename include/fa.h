@@ -164,6 +164,32 @@ fa_status fa_bwd_main_ex(int dtype, const void* q, const void* k, const void* v,
 fa_status fa_bwd_dq_finish_ex(int dtype, void* dq, int B, int H, int N, int d, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/*
+ * Decode-shaped forward: Nq query rows against Nk keys per head (typically few queries and a
+ * long key/value history), for inference; there is no matching backward. The key range is
+ * cut into `nsplit` pieces processed by separate thread blocks, each producing its own
+ * normalised output and log-sum-exp, which a second kernel merges with the online
+ * normaliser's combine rule ([P2] §时间复杂度; [P3] §3.2): LSE = log sum_s exp(LSE_s),
+ * O = sum_s exp(LSE_s - LSE) O_s. (The pages mention inference use only in passing; the
+ * split is ours.)
+ *   in : q [B][H][Nq][d], k, v [B][H][Nk][d] (dtype as for fa_fwd_ex)
+ *   out: o [B][H][Nq][d], lse [B][H][Nq] (natural log, scale included)
+ *   causal: bottom-right alignment, the last query sees every key: key j is visible to
+ *           query i iff j <= i + Nk - Nq (j <= i when Nq = Nk). Rows that see no key get
+ *           O = 0 and LSE = -inf. No block mask.
+ *   nsplit: key-range pieces; 0 = chosen from the problem size and SM count (about three
+ *           quarters of a wave of thread blocks, at least two 128-key tiles per piece);
+ *           capped at ceil(Nk / 128). With one piece the output is written directly.
+ *   workspace: fa_fwd_decode_workspace_bytes(B, H, Nq, Nk, d, nsplit) bytes (0 when the
+ *           problem runs as one piece; pass the same nsplit to both calls), caller-owned,
+ *           contents ignored on entry.
+ * Errors as for fa_fwd; a too-small workspace returns FA_ERR_WORKSPACE.
+ */
+size_t fa_fwd_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d, int nsplit);
+fa_status fa_fwd_decode(int dtype, const void* q, const void* k, const void* v, void* o,
+                        float* lse, int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                        int nsplit, void* workspace, size_t workspace_bytes, void* stream);
+
 #define FA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
                          const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,

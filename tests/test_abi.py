@@ -123,3 +123,23 @@ def test_selftest_rejects_out_of_range_limit(lib):
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, ctypes.c_void_p]
     assert lib.fa_selftest_wait_timeout(0, None) == 1
     assert lib.fa_selftest_wait_timeout(2000000, None) == 1
+
+
+def test_decode_argument_checks_and_workspace(lib):
+    lib.fa_fwd_decode_workspace_bytes.restype = ctypes.c_size_t
+    ws = lib.fa_fwd_decode_workspace_bytes
+    # one piece: written directly, no workspace; k pieces: fp32 O / l and LSE per piece,
+    # rows padded to whole 128-row tiles, each 256-byte aligned
+    assert ws(1, 1, 5, 100, 64, 1) == 0
+    B, H, nq, nk, d, ns = 2, 3, 5, 1000, 64, 4
+    o_bytes = (B * H * ns * 128 * d * 4 + 255) // 256 * 256
+    l_bytes = (B * H * ns * 128 * 4 + 255) // 256 * 256
+    assert ws(B, H, nq, nk, d, ns) == o_bytes + l_bytes
+    assert ws(1, 1, 5, 300, 64, 99) == ws(1, 1, 5, 300, 64, 3)  # capped at ceil(Nk / 128) pieces
+    assert ws(1, 1, 0, 100, 64, 1) == 0 and ws(1, 1, 5, 100, 80, 1) == 0 and ws(1, 1, 5, 100, 64, -1) == 0
+    call = lambda **kw: lib.fa_fwd_decode(kw.get("dt", 0), FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, kw.get("nq", 4),
+                                          kw.get("nk", 256), kw.get("d", 64), 0.125, 0, kw.get("ns", 2), FAKE,
+                                          kw.get("wsb", 1 << 30), None)
+    assert call(nq=0) == 1 and call(nk=0) == 1 and call(ns=-1) == 1 and call(dt=5) == 1
+    assert call(d=96) == 2
+    assert call(wsb=10) == 5  # two pieces need a workspace

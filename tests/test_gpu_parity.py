@@ -131,6 +131,41 @@ def test_per_head_block_masks(fa, oracle_mod, B, Hh, N, d, causal):
             H.assert_grads_close([x[sl] for x in outs[2:]], g_ref, f"head {b},{h}")
 
 
+DECODE = [
+    # B, H, Nq, Nk, d, causal, num_splits (0: the library's choice), dtype
+    (2, 4, 1, 4096, 128, False, 0, "bf16"),      # one query per head, long key history
+    (1, 2, 16, 1000, 64, True, 0, "bf16"),       # bottom-right causal, ragged key tail
+    (1, 2, 130, 777, 128, True, 3, "bf16"),      # two query tiles, uneven pieces
+    (1, 1, 300, 200, 64, True, 2, "bf16"),       # more queries than keys: 100 rows see nothing
+    (2, 1, 64, 2048, 128, False, 1, "bf16"),     # one piece: written directly, no merge
+    (1, 3, 8, 3000, 64, False, 5, "f16"),
+]
+
+
+@pytest.mark.parametrize("B,Hh,Nq,Nk,d,causal,splits,dtype", DECODE)
+def test_decode_forward(fa, oracle_mod, B, Hh, Nq, Nk, d, causal, splits, dtype):
+    seed = synth.BASE_SEED + 31 * Nq + Nk
+    gq, rq = H.make_case(B, Hh, Nq, d, seed=seed, with_do=False, dtype=dtype)
+    gk, rk = H.make_case(B, Hh, Nk, d, seed=seed + 1000, with_do=False, dtype=dtype)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = fa.forward_decode(gq["q"], gk["k"], gk["v"], causal=causal, scale=scale, num_splits=splits)
+    torch.cuda.synchronize()
+    assert fa.last_device_status() == 0
+    o_ref, l_ref = oracle_mod.attention_fwd_qk(rq["q"], rk["k"], rk["v"], scale, causal=causal)
+    H.assert_fwd_close(H.to_f64(o), H.to_f64(lse), o_ref, l_ref, f"decode {B,Hh,Nq,Nk,d,causal,splits}")
+
+
+def test_decode_path_agrees_with_square_forward(fa):
+    # Nq = Nk through the split-and-merge path gives the square forward's result up to rounding
+    gpu, _ = H.make_case(1, 2, 640, 128, seed=synth.BASE_SEED + 77, with_do=False)
+    for causal in (False, True):
+        o1, l1 = run_fwd(fa, gpu, causal, None, 0.0884)
+        o2, l2 = fa.forward_decode(gpu["q"], gpu["k"], gpu["v"], causal=causal, scale=0.0884, num_splits=3)
+        torch.cuda.synchronize()
+        assert (o1.float() - o2.float()).abs().max().item() < 8e-3
+        assert (l1 - l2).abs().max().item() < 1e-4
+
+
 def test_fp16_and_bf16_agree(fa):
     # The same draws rounded to each type give nearly the same attention: the element type
     # only changes input rounding and the 16-bit P (fp16 carries three more mantissa bits).
