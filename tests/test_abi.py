@@ -54,6 +54,7 @@ def test_fwd_argument_checks(lib):
     assert fwd(lib, d=96) == 2                   # unsupported head dim
     assert fwd(lib, d=256) == 2
     assert fwd(lib, N=0) == 1                    # empty sequence -> INVALID
+    assert fwd(lib, B=65536) == 2 and fwd(lib, B=256, H=256) == 2  # B*H above the grid's y limit
 
 
 def test_workspace_size_and_checks(lib):

@@ -282,3 +282,67 @@ def test_bounded_wait_timeout_is_reported_and_context_survives(fa):
     gpu, _ = H.make_case(1, 1, 256, 64, seed=13)
     o, lse = run_fwd(fa, gpu, False, None, 0.125)
     assert torch.isfinite(o.float()).all()
+
+
+@pytest.mark.parametrize("scale", [0.5, 3.0])
+@pytest.mark.parametrize("causal", [False, True])
+def test_large_scale_exercises_the_rescale_path(fa, oracle_mod, scale, causal):
+    # With scale well above 1/sqrt(d) the row maxima jump by far more than the reference-max
+    # threshold from tile to tile, so O is rescaled in TMEM over and over; P is nearly one-hot.
+    # The absolute bars assume scale = 1/sqrt(d), where O averages many rows of V and stays
+    # small. Here |O| approaches single rows of V (up to ~4.5), where half a bf16 ulp alone is
+    # up to 2^-7 and P's own 2^-9 rounding adds as much again: the bar is relative to |O|
+    # (1% of max(1, |O|)), the mean is 2e-3, and the LSE (up to ~100) is held to 1e-3 of
+    # max(1, |LSE|).
+    N, d = 1000, 128
+    gpu, ref = H.make_case(1, 2, N, d, seed=synth.BASE_SEED + 41)
+    o, lse = run_fwd(fa, gpu, causal, None, scale)
+    o_ref, l_ref = oracle_mod.attention_fwd(ref["q"], ref["k"], ref["v"], scale, causal=causal)
+    err = np.abs(H.to_f64(o) - o_ref)
+    assert (err / np.maximum(1.0, np.abs(o_ref))).max() <= 1e-2, f"scale {scale}: O rel err {err.max():.3e}"
+    assert err.mean() <= 2e-3, f"scale {scale}: O mean err {err.mean():.3e}"
+    lerr = np.abs(H.to_f64(lse) - l_ref) / np.maximum(1.0, np.abs(l_ref))
+    assert lerr.max() <= 1e-3, f"scale {scale}: LSE rel err {lerr.max():.3e}"
+    dq, dk, dv = run_bwd(fa, gpu, o, lse, causal, None, scale)
+    g_ref = oracle_mod.attention_bwd(ref["q"], ref["k"], ref["v"], ref["do"], scale, causal=causal)[:3]
+    H.assert_grads_close([H.to_f64(x) for x in (dq, dk, dv)], g_ref, f"scale {scale}")
+
+
+def test_bench_workload_backward_full_size(fa, oracle_mod):
+    # The bench's default workload (B=4, H=16, N=4096, d=128) in one launch: one sampled head
+    # against the oracle in full, and on every head two identities that hold at any size:
+    # sum_j dK_j = 0 (rows of dS sum to zero) and sum_j dV_j = sum_i dO_i (rows of P sum to one).
+    B, Hh, N, d = 4, 16, 4096, 128
+    check_heads(fa, oracle_mod, B, Hh, N, d, False, None, nheads=1, seed=synth.BASE_SEED + 3)
+    gpu, _ = H.make_case(B, Hh, N, d, seed=synth.BASE_SEED + 3)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = run_fwd(fa, gpu, False, None, scale)
+    dq, dk, dv = run_bwd(fa, gpu, o, lse, False, None, scale)
+    dk_sum = dk.float().sum(dim=2)
+    dv_sum = dv.float().sum(dim=2)
+    do_sum = gpu["do"].float().sum(dim=2)
+    # bf16 rounding of each dK row (~2^-9 relative) bounds the column sums against the rows' size
+    assert (dk_sum.norm(dim=-1) / dk.float().norm(dim=(2, 3))).max().item() < 2e-2
+    assert ((dv_sum - do_sum).norm(dim=-1) / do_sum.norm(dim=-1)).max().item() < 2e-2
+
+
+def test_largest_head_count(fa, oracle_mod):
+    # B*H = 65535 (the grid's y limit) with one 128-row tile per head, forward and backward.
+    # Heads are independent: the bulk is seeded device-side random data, and five heads across
+    # the range carry synth's draws, which the oracle gets bit for bit.
+    B, N, d, scale = 65535, 128, 64, 0.125
+    g = torch.Generator(device="cuda").manual_seed(synth.BASE_SEED)
+    gpu = {k: torch.randn(B, 1, N, d, device="cuda", dtype=torch.bfloat16, generator=g) for k in ("q", "k", "v", "do")}
+    sample = (0, 1, 32767, 65533, 65534)
+    small, ref = H.make_case(len(sample), 1, N, d, seed=synth.BASE_SEED + 9)
+    for x, b in enumerate(sample):
+        for k in gpu:
+            gpu[k][b] = small[k][x]
+    o, lse = run_fwd(fa, gpu, False, None, scale)
+    dq, dk, dv = run_bwd(fa, gpu, o, lse, False, None, scale)
+    for x, b in enumerate(sample):
+        args = [ref[k][x:x + 1] for k in ("q", "k", "v")]
+        o_ref, l_ref = oracle_mod.attention_fwd(*args, scale)
+        H.assert_fwd_close(H.to_f64(o[b:b + 1]), H.to_f64(lse[b:b + 1]), o_ref, l_ref, f"head {b}")
+        g_ref = oracle_mod.attention_bwd(*args, ref["do"][x:x + 1], scale)[:3]
+        H.assert_grads_close([H.to_f64(t[b:b + 1]) for t in (dq, dk, dv)], g_ref, f"head {b}")
