@@ -84,6 +84,8 @@ def library() -> ctypes.CDLL:
         lib.fa_fwd_decode.argtypes = [i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32, i32, vp, sz, vp]
         lib.fa_last_device_status.restype = i32
         lib.fa_last_device_status.argtypes = [vp]
+        lib.fa_selftest_ex2.restype = i32
+        lib.fa_selftest_ex2.argtypes = [vp, vp, vp, i32, vp]
         lib.fa_selftest_wait_timeout.restype = i32
         lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
         _lib = lib
@@ -244,6 +246,17 @@ def selftest_wait_timeout(limit_us: int = 20000, device=None) -> None:
     """Enqueues the failure-detection self-test (a bounded wait that is meant to give up)."""
     dev = torch.device("cuda") if device is None else device
     _check(library().fa_selftest_wait_timeout(int(limit_us), _stream(dev)), "fa_selftest_wait_timeout")
+
+
+def selftest_ex2(x):
+    """The library's FMA-pipe exp2 and the special-function unit's ex2.approx on fp32 CUDA
+    tensor x: returns (poly, sfu)."""
+    if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
+    poly, sfu = torch.empty_like(x), torch.empty_like(x)
+    _check(library().fa_selftest_ex2(_ptr(x), _ptr(poly), _ptr(sfu), x.numel(), _stream(x.device)),
+           "fa_selftest_ex2")
+    return poly, sfu
 
 
 def last_device_status(device=None) -> int:

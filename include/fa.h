@@ -212,6 +212,15 @@ fa_status fa_last_device_status(void* stream);
  */
 fa_status fa_selftest_wait_timeout(unsigned int limit_us, void* stream);
 
+/*
+ * Accuracy self-test of the library's own FMA-pipe exp2 (no counterpart on the pages): a
+ * compile-time option of the softmax kernels, off in the shipped build, kept testable. For n
+ * device fp32 inputs x, writes the packed polynomial's 2^x to y_poly and the special-function
+ * unit's ex2.approx to y_sfu (device buffers of n floats). Meant for inputs in [-125, 127]
+ * (softmax exponents are <= 8). Returns FA_ERR_INVALID for n < 0 or null buffers.
+ */
+fa_status fa_selftest_ex2(const float* x, float* y_poly, float* y_sfu, int n, void* stream);
+
 /* Static, human-readable name of a status code. Never NULL. */
 const char* fa_status_string(fa_status status);
 

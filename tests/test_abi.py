@@ -119,6 +119,12 @@ def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):
         fa.library()
 
 
+def test_ex2_selftest_checks_arguments(lib):
+    assert lib.fa_selftest_ex2(None, None, None, -1, None) == 1
+    assert lib.fa_selftest_ex2(None, None, None, 4, None) == 1
+    assert lib.fa_selftest_ex2(None, None, None, 0, None) == 0
+
+
 def test_selftest_rejects_out_of_range_limit(lib):
     lib.fa_selftest_wait_timeout.restype = ctypes.c_int
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, ctypes.c_void_p]

@@ -346,3 +346,18 @@ def test_largest_head_count(fa, oracle_mod):
         H.assert_fwd_close(H.to_f64(o[b:b + 1]), H.to_f64(lse[b:b + 1]), o_ref, l_ref, f"head {b}")
         g_ref = oracle_mod.attention_bwd(*args, ref["do"][x:x + 1], scale)[:3]
         H.assert_grads_close([H.to_f64(t[b:b + 1]) for t in (dq, dk, dv)], g_ref, f"head {b}")
+
+
+def test_fma_pipe_exp2_accuracy(fa):
+    # The own cubic exp2 (a compile-time option of the softmax kernels) against exact 2^x and
+    # against the special-function unit, over the range softmax exponents take.
+    g = torch.Generator().manual_seed(5)
+    x = torch.cat([torch.linspace(-120.0, 8.0, 200001, dtype=torch.float64),
+                   torch.rand(100000, generator=g, dtype=torch.float64) * 16 - 12]).float()
+    poly, sfu = fa.selftest_ex2(x.cuda())
+    torch.cuda.synchronize()
+    exact = torch.exp2(x.double())
+    rel_poly = ((poly.double().cpu() - exact).abs() / exact).max().item()
+    rel_sfu = ((sfu.double().cpu() - exact).abs() / exact).max().item()
+    assert rel_poly < 1e-4, rel_poly   # fitted bound: 7.5e-5 in fp32 Horner form
+    assert rel_sfu < 1e-5, rel_sfu
