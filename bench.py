@@ -8,7 +8,7 @@ inputs from the seeded generator. Prints ONE JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--seqlen N] [--headdim d]
                     [--causal] [--block-sparse [--block-density P]] [--dtype bf16|f16]
-                    [--impl reference] [--sweep] [--density-sweep] [--decode NQ]
+                    [--impl reference] [--sweep] [--density-sweep] [--decode NQ] [--forward-only]
 
 Metric: fwd+bwd TFLOPS with FLOPs counted as 4*B*H*N^2*d for the forward (halved for causal,
 scaled by block density for block-sparse) and 2.5x that for the backward.
@@ -257,6 +257,54 @@ def run_decode(args, rank, world, local_rank, dist_on):
     return 0
 
 
+def run_forward_only(args, wl, rank, world, local_rank, dist_on):
+    """Forward pass alone on the sweep's workload (the one line for head dimension 256, which
+    has a forward but no backward). Metric: forward TFLOPS (4·N²·d per head, halved when
+    causal) against the measured dense bf16 peak."""
+    import torch
+    import exact_attention_110_b200 as fa
+    import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    B, H, N, d, causal = wl["B"], wl["H"], wl["N"], wl["d"], wl["causal"]
+    seed = synth.BASE_SEED + 97 * rank
+    q, k, v = (synth.to_torch(_stream(seed + o, B * H * N * d, args.dtype).reshape(B, H, N, d), args.dtype, dev)
+               for o in (synth.SEED_Q, synth.SEED_K, synth.SEED_V))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    scale = 1.0 / math.sqrt(d)
+    for _ in range(args.warmup):
+        fa.forward(q, k, v, causal=causal, scale=scale, out=o, lse=lse)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist_on:
+        torch.distributed.barrier()
+    with ClockSampler(physical_gpu(local_rank)) as clk:
+        time.sleep(0.3)
+        start.record()
+        for _ in range(args.steps):
+            fa.forward(q, k, v, causal=causal, scale=scale, out=o, lse=lse)
+        end.record()
+        torch.cuda.synchronize()
+    if fa.last_device_status(dev) != 0:
+        raise RuntimeError("device wait timed out")
+    ms = reduce_max(start.elapsed_time(end), dist_on, dev) / args.steps
+    tflops = fwd_flops(B, H, N, d, causal) / (ms * 1e-3) / 1e12
+    peaks = load_peaks()
+    line = {"metric": "attention forward TFLOPS", "value": world * tflops, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+            "config": {"workload": wl["name"] + ", forward only", "B": B, "H": H, "N": N, "d": d,
+                       "causal": causal},
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tflops / peaks["bf16_tflops"], "traffic": None, "kernel": "fa_fwd_kernel"},
+            "gpu_launches": args.steps, "clocks": clk.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- GPU arm
 @functools.lru_cache(maxsize=4)
 def _stream(seed: int, n: int, dtype: str = "bf16"):
@@ -438,6 +486,8 @@ def main(argv=None):
                     help="block-sparse config at densities 0.05..1: runtime should follow the blocks that are on")
     ap.add_argument("--decode", type=int, default=0, metavar="NQ",
                     help="decode-shaped forward: NQ queries per head against --seqlen keys (B=8)")
+    ap.add_argument("--forward-only", action="store_true",
+                    help="time the forward alone (the only pass built at head dimension 256)")
     ap.add_argument("--dtype", choices=["bf16", "f16"], default="bf16",
                     help="element type of q, k, v, o, dO and the gradients (fp32 accumulation either way)")
     args = ap.parse_args(argv)
@@ -461,6 +511,9 @@ def main(argv=None):
     try:
         if args.decode > 0:
             return run_decode(args, rank, world, local_rank, dist_on)
+        if args.forward_only:
+            return run_forward_only(args, workload(args.seqlen, args.headdim, args.causal, False),
+                                    rank, world, local_rank, dist_on)
         if args.density_sweep:
             args.no_cpu_baseline, args.no_e2e = True, True
             for p_on in (0.05, 0.1, 0.25, 0.5, 1.0):

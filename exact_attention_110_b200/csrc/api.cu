@@ -64,9 +64,11 @@ bool mask_stride_ok(const uint8_t* mask, long long stride, int N) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-fa_status check_common(int B, int H, int N, int d, float scale) {
+// Head dimensions: 64 and 128 everywhere; 256 in the forward only (its backward's dK and dV
+// accumulators alone would fill the 512 TMEM columns).
+fa_status check_common(int B, int H, int N, int d, float scale, bool allow_d256 = false) {
   if (B <= 0 || H <= 0 || N <= 0 || !isfinite(scale)) return FA_ERR_INVALID;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && !(allow_d256 && d == 256)) return FA_ERR_UNSUPPORTED;
   const long long BH = (long long)B * H;
   if (BH > 65535) return FA_ERR_UNSUPPORTED;               // grid.y limit
   if ((long long)N * d > (1ll << 31) / 2) return FA_ERR_UNSUPPORTED;  // per-head elements
@@ -121,7 +123,7 @@ fa_status fa_fwd_ex(int dtype, const void* q, const void* k, const void* v, void
   const int f16 = dtype == FA_DTYPE_F16;
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID;
-  fa_status st = check_common(B, H, N, d, scale);
+  fa_status st = check_common(B, H, N, d, scale, true);
   if (st != FA_OK) return st;
   if (!get_encoder()) return FA_ERR_CUDA;
   const long long BH = (long long)B * H;
@@ -162,10 +164,11 @@ namespace {
 // a wave (measured: with 128 query-tile pairs one piece streams K/V faster than three, the
 // partial writes and the merge cost more than the idle SMs), but at least two key tiles per
 // split; an explicit request is only capped by the number of key tiles.
-int decode_splits(long long BH, int Nq, int Nk, int requested) {
+int decode_splits(long long BH, int Nq, int Nk, int d, int requested) {
   const int nbk = (Nk + 127) / 128;
   if (requested > 0) return requested < nbk ? requested : nbk;
-  const long long pairs = BH * (((Nq + 127) / 128 + 1) / 2);
+  const int tiles_per_cta = d == 256 ? 1 : 2;  // the forward kernel's query tiles per CTA
+  const long long pairs = BH * (((Nq + 127) / 128 + tiles_per_cta - 1) / tiles_per_cta);
   const long long target = 3ll * fa::device_sm_count() / 4;
   long long s = (target + pairs - 1) / pairs;
   const long long cap = nbk / 2 > 1 ? nbk / 2 : 1;
@@ -193,7 +196,7 @@ DecodeWorkspace decode_layout(void* base, long long BH, int Nq, int d, int nspli
 
 fa_status check_decode(int B, int H, int Nq, int Nk, int d, float scale, int nsplit) {
   if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || nsplit < 0 || !isfinite(scale)) return FA_ERR_INVALID;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   const long long BH = (long long)B * H;
   if (BH > 65535) return FA_ERR_UNSUPPORTED;
   if ((long long)Nq * d > (1ll << 31) / 2 || (long long)Nk * d > (1ll << 31) / 2) return FA_ERR_UNSUPPORTED;
@@ -205,7 +208,7 @@ fa_status check_decode(int B, int H, int Nq, int Nk, int d, float scale, int nsp
 size_t fa_fwd_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d, int nsplit) {
   if (check_decode(B, H, Nq, Nk, d, 1.0f, nsplit) != FA_OK) return 0;
   const long long BH = (long long)B * H;
-  return decode_layout(nullptr, BH, Nq, d, decode_splits(BH, Nq, Nk, nsplit)).bytes;
+  return decode_layout(nullptr, BH, Nq, d, decode_splits(BH, Nq, Nk, d, nsplit)).bytes;
 }
 
 fa_status fa_fwd_decode(int dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -218,7 +221,7 @@ fa_status fa_fwd_decode(int dtype, const void* q, const void* k, const void* v, 
   fa_status st = check_decode(B, H, Nq, Nk, d, scale, nsplit);
   if (st != FA_OK) return st;
   const long long BH = (long long)B * H;
-  const int ns = decode_splits(BH, Nq, Nk, nsplit);
+  const int ns = decode_splits(BH, Nq, Nk, d, nsplit);
   DecodeWorkspace w = decode_layout(workspace, BH, Nq, d, ns);
   if (ns > 1 && (!workspace || !aligned16(workspace) || workspace_bytes < w.bytes)) return FA_ERR_WORKSPACE;
   if (!get_encoder()) return FA_ERR_CUDA;

@@ -51,12 +51,15 @@ struct FwdCfg {
   // the control warpgroup (TMA, MMA, 2 idle warps) keeps 88, the softmax warpgroups get 208.
   static constexpr int REGS_CTRL = 88, REGS_SOFTMAX = 208;
   static_assert(128 * REGS_CTRL + 256 * REGS_SOFTMAX <= 384 * 168, "setmaxnreg split exceeds the launch");
-  static constexpr int NS = (D == 128) ? 2 : 4;        // K ring and V ring depth
+  static constexpr int NS = (D == 128) ? 2 : (D == 64 ? 4 : 1);  // K ring and V ring depth
+  // 128-row query tiles per CTA: two that ping-pong, or one at d = 256, where two tiles'
+  // S and O would need 768 TMEM columns (one tile: S [0,128), O [256,512)).
+  static constexpr int TILES = (D == 256) ? 1 : 2;
   static constexpr int PANEL_BYTES = 128 * 128;        // 128 rows x 64 bf16 (one swizzle panel)
   static constexpr int PANELS = D / 64;
   static constexpr int TILE_BYTES = PANELS * PANEL_BYTES;  // 128 x D bf16
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
+  static constexpr int OFF_K = OFF_Q + TILES * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + NS * TILE_BYTES;
   static constexpr int NBAR = 2 + 4 * NS + 2 + 4 + 2 + 1;
@@ -160,12 +163,12 @@ __global__ void __launch_bounds__(384, 1)
   const int pi = (int)blockIdx.x / p.nsplit, split = (int)blockIdx.x - pi * p.nsplit;
   const int npairs = (int)gridDim.x / p.nsplit;
   const int pair = p.causal ? npairs - 1 - pi : pi;
-  const int qb0 = 2 * pair;  // 128-row tile index of tile 0
+  const int qb0 = C::TILES * pair;  // 128-row tile index of tile 0
   // this CTA's key tiles: its split's range, cut at the last key the pair's last row sees
   const int j_begin = split * p.kv_per_split;
   int j_end = min(p.nbk, j_begin + p.kv_per_split);
   if (p.causal) {
-    const int last_key = 128 * qb0 + 255 + p.causal_off;
+    const int last_key = 128 * qb0 + 128 * C::TILES - 1 + p.causal_off;
     j_end = min(j_end, last_key < 0 ? 0 : last_key / 128 + 1);
   }
   const uint64_t lim = p.timeout_ns;
@@ -211,7 +214,7 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmO);
       for (int t = 0; t < 2; ++t) {
-        if (qb0 + t < p.nb) {
+        if (qb0 + t < p.nb && (C::TILES == 2 || t == 0)) {
           mbar_arrive_expect_tx(&bar_q[t], C::TILE_BYTES);
           for (int pn = 0; pn < C::PANELS; ++pn)
             tma_load_3d(smem + C::OFF_Q + t * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &bar_q[t], pn * 64,
@@ -223,7 +226,8 @@ __global__ void __launch_bounds__(384, 1)
       for (int s = 0; s < NS; ++s) issued_k[s] = issued_v[s] = -1;
       bool ok = true;
       for (int j = j_begin; j < j_end && ok; ++j) {
-        if (!fwd_tile_active(p, bmask, qb0, j) && !fwd_tile_active(p, bmask, qb0 + 1, j)) continue;
+        if (!fwd_tile_active(p, bmask, qb0, j) && (C::TILES == 1 || !fwd_tile_active(p, bmask, qb0 + 1, j)))
+          continue;
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
         ok = mbar_wait(&bar_ke[s], ph ^ 1, ab, lim, WAIT_FWD_LOAD + 1);
@@ -250,7 +254,7 @@ __global__ void __launch_bounds__(384, 1)
           if (issued_v[s] >= 0) mbar_wait(&bar_vf[s], issued_v[s], &none, lim, WAIT_FWD_LOAD + 3);
         }
         for (int t = 0; t < 2; ++t)
-          if (qb0 + t < p.nb) mbar_wait(&bar_q[t], 0, &none, lim, WAIT_FWD_LOAD + 4);
+          if (qb0 + t < p.nb && (C::TILES == 2 || t == 0)) mbar_wait(&bar_q[t], 0, &none, lim, WAIT_FWD_LOAD + 4);
       }
     }
   } else if (warp == 1) {
@@ -268,7 +272,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t dv_base = sdesc_sw128(sV, C::PANEL_BYTES, 1024);
       bool ok = true;
       for (int t = 0; t < 2 && ok; ++t)
-        if (qb0 + t < p.nb) ok = mbar_wait_spin(&bar_q[t], 0, ab, lim, WAIT_FWD_MMA + 1);
+        if (qb0 + t < p.nb && (C::TILES == 2 || t == 0)) ok = mbar_wait_spin(&bar_q[t], 0, ab, lim, WAIT_FWD_MMA + 1);
       uint32_t p_phase[2] = {0u, 0u};
       bool o_started[2] = {false, false};
       bool prev_act[2] = {false, false};
@@ -277,7 +281,8 @@ __global__ void __launch_bounds__(384, 1)
       int it = 0;
 
       for (int j = j_begin; j < j_end && ok; ++j) {
-        const bool act0 = fwd_tile_active(p, bmask, qb0, j), act1 = fwd_tile_active(p, bmask, qb0 + 1, j);
+        const bool act0 = fwd_tile_active(p, bmask, qb0, j);
+        const bool act1 = C::TILES == 2 && fwd_tile_active(p, bmask, qb0 + 1, j);
         if (!act0 && !act1) continue;
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
@@ -362,7 +367,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t wq = warp & 3;      // TMEM lane quarter this warp may touch
     const int r = wq * 32 + lane;      // row inside the tile
     const int qb = qb0 + t;
-    const bool tvalid = qb < p.nb;
+    const bool tvalid = qb < p.nb && (C::TILES == 2 || t == 0);
     const uint32_t lane_off = (wq * 32u) << 16;
     const uint32_t tS_row = tmem + lane_off + t * 128u;
     const uint32_t tO_row = tmem + lane_off + 256u + t * D;
@@ -516,7 +521,7 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   cudaError_t e =
       cudaFuncSetAttribute(fa_fwd_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.nb + 1) / 2 * p.nsplit, BH);
+  dim3 grid((p.nb + C::TILES - 1) / C::TILES * p.nsplit, BH);
   fa_fwd_kernel<D, F16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
@@ -525,9 +530,11 @@ cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, cons
                        const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream) {
   if (p.f16) {
     if (D == 64) return launch_fwd_t<64, true>(tq, tk, tv, to, p, BH, stream);
+    if (D == 256) return launch_fwd_t<256, true>(tq, tk, tv, to, p, BH, stream);
     return launch_fwd_t<128, true>(tq, tk, tv, to, p, BH, stream);
   }
   if (D == 64) return launch_fwd_t<64, false>(tq, tk, tv, to, p, BH, stream);
+  if (D == 256) return launch_fwd_t<256, false>(tq, tk, tv, to, p, BH, stream);
   return launch_fwd_t<128, false>(tq, tk, tv, to, p, BH, stream);
 }
 

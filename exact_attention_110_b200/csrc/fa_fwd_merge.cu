@@ -55,6 +55,11 @@ cudaError_t launch_fwd_merge(const FwdMergeParams& p, cudaStream_t stream) {
       fa_fwd_merge_kernel<64, true><<<grid, 256, 0, stream>>>(p);
     else
       fa_fwd_merge_kernel<64, false><<<grid, 256, 0, stream>>>(p);
+  } else if (p.D == 256) {
+    if (p.f16)
+      fa_fwd_merge_kernel<256, true><<<grid, 256, 0, stream>>>(p);
+    else
+      fa_fwd_merge_kernel<256, false><<<grid, 256, 0, stream>>>(p);
   } else {
     if (p.f16)
       fa_fwd_merge_kernel<128, true><<<grid, 256, 0, stream>>>(p);

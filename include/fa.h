@@ -27,7 +27,9 @@
  *  - All pointers are device memory owned by the caller. The library allocates no device
  *    memory apart from one static device status word and the fixed scratch array that
  *    fa_bwd_noalloc uses.
- *  - Every pointer must be 16-byte aligned. d must be 64 or 128. N is any positive length;
+ *  - Every pointer must be 16-byte aligned. d must be 64 or 128, or 256 in the forward calls
+ *    (fa_fwd, fa_fwd_ex, fa_fwd_decode: one 128-row query tile per thread block there; the
+ *    backward's dK and dV accumulators would not fit tensor memory). N is any positive length;
  *    a partial last 128-row tile is handled inside the kernels (rows and keys beyond N take no
  *    part and are never written).
  *  - stream is a cudaStream_t (NULL = legacy default stream). All calls are asynchronous
@@ -48,7 +50,8 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID = 1,     /* null/misaligned pointer, non-positive size, non-finite scale */
-  FA_ERR_UNSUPPORTED = 2, /* valid but not implemented: d not in {64,128}; backward scale <= 0 */
+  FA_ERR_UNSUPPORTED = 2, /* valid but not implemented: d not in {64,128} (256: forward only);
+                             backward scale <= 0 */
   FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call or a kernel launch failed */
   FA_ERR_TIMEOUT = 4,     /* a device-side bounded wait gave up (see fa_last_device_status) */
   FA_ERR_WORKSPACE = 5    /* workspace pointer null or smaller than fa_bwd_workspace_bytes */

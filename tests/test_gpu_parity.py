@@ -131,6 +131,22 @@ def test_per_head_block_masks(fa, oracle_mod, B, Hh, N, d, causal):
             H.assert_grads_close([x[sl] for x in outs[2:]], g_ref, f"head {b},{h}")
 
 
+@pytest.mark.parametrize("B,Hh,N,causal,mask", [(1, 2, 384, False, None), (2, 1, 333, True, None),
+                                                (1, 1, 640, False, "bernoulli")])
+def test_forward_head_dim_256(fa, oracle_mod, B, Hh, N, causal, mask):
+    # d = 256: one 128-row query tile per thread block (forward only)
+    d = 256
+    gpu, ref = H.make_case(B, Hh, N, d, seed=synth.BASE_SEED + N + 256, with_do=False)
+    scale = 1.0 / np.sqrt(d)
+    m = mask_for(mask, N)
+    mt = None if m is None else torch.from_numpy(m).cuda()
+    o, lse = run_fwd(fa, gpu, causal, mt, scale)
+    o_ref, l_ref = oracle_mod.attention_fwd(ref["q"], ref["k"], ref["v"], scale, causal=causal, mask=m)
+    H.assert_fwd_close(H.to_f64(o), H.to_f64(lse), o_ref, l_ref, f"d=256 {B,Hh,N,causal,mask}")
+    with pytest.raises(fa.FAError):  # no backward at d = 256
+        fa.backward(gpu["q"], gpu["k"], gpu["v"], o, gpu["q"], lse, causal=causal, block_mask=mt, scale=scale)
+
+
 DECODE = [
     # B, H, Nq, Nk, d, causal, num_splits (0: the library's choice), dtype
     (2, 4, 1, 4096, 128, False, 0, "bf16"),      # one query per head, long key history
@@ -139,6 +155,7 @@ DECODE = [
     (1, 1, 300, 200, 64, True, 2, "bf16"),       # more queries than keys: 100 rows see nothing
     (2, 1, 64, 2048, 128, False, 1, "bf16"),     # one piece: written directly, no merge
     (1, 3, 8, 3000, 64, False, 5, "f16"),
+    (1, 2, 40, 900, 256, True, 0, "bf16"),      # head dim 256
 ]
 
 
