@@ -167,7 +167,7 @@ namespace {
 int decode_splits(long long BH, int Nq, int Nk, int d, int requested) {
   const int nbk = (Nk + 127) / 128;
   if (requested > 0) return requested < nbk ? requested : nbk;
-  const int tiles_per_cta = d == 256 ? 1 : 2;  // the forward kernel's query tiles per CTA
+  const int tiles_per_cta = fa::fwd_tiles_per_cta(d);  // the forward kernel's query tiles per CTA
   const long long pairs = BH * (((Nq + 127) / 128 + tiles_per_cta - 1) / tiles_per_cta);
   const long long target = 3ll * fa::device_sm_count() / 4;
   long long s = (target + pairs - 1) / pairs;

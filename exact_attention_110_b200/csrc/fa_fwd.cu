@@ -41,6 +41,15 @@
 #ifndef FA_FWD_EXP_EMU_MASK
 #define FA_FWD_EXP_EMU_MASK 0x0u
 #endif
+// Head dimensions (bit d/64: 0x2 d=64, 0x4 d=128, 0x10 d=256) whose forward runs one query
+// tile per CTA with double-buffered S and the softmax split by columns; the others run two
+// ping-ponged tiles. d = 256 has to.
+#ifndef FA_FWD_ONE_TILE_DIMS
+#define FA_FWD_ONE_TILE_DIMS 0x10u
+#endif
+#ifndef FA_FWD_ONE_TILE_STAGES_D128
+#define FA_FWD_ONE_TILE_STAGES_D128 2
+#endif
 
 namespace fa {
 
@@ -51,10 +60,16 @@ struct FwdCfg {
   // the control warpgroup (TMA, MMA, 2 idle warps) keeps 88, the softmax warpgroups get 208.
   static constexpr int REGS_CTRL = 88, REGS_SOFTMAX = 208;
   static_assert(128 * REGS_CTRL + 256 * REGS_SOFTMAX <= 384 * 168, "setmaxnreg split exceeds the launch");
-  static constexpr int NS = (D == 128) ? 2 : (D == 64 ? 4 : 1);  // K ring and V ring depth
-  // 128-row query tiles per CTA: two that ping-pong, or one at d = 256, where two tiles'
-  // S and O would need 768 TMEM columns (one tile: S [0,128), O [256,512)).
-  static constexpr int TILES = (D == 256) ? 1 : 2;
+  // 128-row query tiles per CTA. Two that ping-pong (S_t in columns [128t, 128t+128), O_t
+  // after them), or one (required at d = 256, where two tiles' S and O would need 768 TMEM
+  // columns): then S is double-buffered -- S(a) of the a-th active KV tile in columns
+  // [0,128) or [128,256) by the parity of a, O in [256, 256+D) -- so the tensor core computes
+  // S(a+1) while the softmax works on S(a), and both softmax warpgroups share the tile, each
+  // taking 64 of the 128 key columns.
+  static constexpr int TILES = ((FA_FWD_ONE_TILE_DIMS >> (D / 64)) & 1u) ? 1 : 2;
+  static_assert(D != 256 || TILES == 1, "d = 256 needs the one-tile layout");
+  static constexpr int NS = TILES == 2 ? ((D == 128) ? 2 : 4)  // K ring and V ring depth
+                                       : (D == 256 ? 1 : (D == 128 ? FA_FWD_ONE_TILE_STAGES_D128 : 4));
   static constexpr int PANEL_BYTES = 128 * 128;        // 128 rows x 64 bf16 (one swizzle panel)
   static constexpr int PANELS = D / 64;
   static constexpr int TILE_BYTES = PANELS * PANEL_BYTES;  // 128 x D bf16
@@ -62,8 +77,11 @@ struct FwdCfg {
   static constexpr int OFF_K = OFF_Q + TILES * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + NS * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + NS * TILE_BYTES;
-  static constexpr int NBAR = 2 + 4 * NS + 2 + 4 + 2 + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int NBAR = 2 + 4 * NS + 2 + 4 + 2 + 1 + (TILES == 1 ? 1 : 0);
+  // one tile: the two warpgroups' row maxima [2 parities][2 halves][128] (row sums at the end)
+  static constexpr int OFF_XCH = OFF_BAR + NBAR * 8;
+  static constexpr int XCH_BYTES = TILES == 1 ? 2 * 2 * 128 * 4 : 0;
+  static constexpr int OFF_MISC = OFF_XCH + XCH_BYTES;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int TMEM_COLS = 512;
   // Which of the 16 score pairs of each 32-score chunk take 2^x on the FMA pipe (ex2_poly)
@@ -129,6 +147,42 @@ __device__ __forceinline__ float softmax_exp_store(const uint32_t (&su)[128], ui
   return a + b;
 }
 
+// The one-tile form of softmax_exp_store: one warpgroup's 64 scores of a row (keys 64h..64h+63)
+// -> P in 32 packed columns at tP; the caller signals the half. Returns this half's row sum.
+template <bool F16, bool EMU, uint32_t EMU_MASK>
+__device__ __forceinline__ float softmax_exp_store64(const uint32_t (&su)[64], uint64_t sl2_2, uint64_t mneg_2,
+                                                     uint32_t tP, const Ex2PolyConsts& K) {
+  uint64_t ls2[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) ls2[k] = 0ull;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint64_t s2 = f2_pack(__uint_as_float(su[32 * c + 2 * i]), __uint_as_float(su[32 * c + 2 * i + 1]));
+      const uint64_t x2 = ffma2(s2, sl2_2, mneg_2);
+      uint64_t p2;
+      if (EMU && ((EMU_MASK >> i) & 1u)) {
+        p2 = ex2_poly2(x2, K);
+      } else {
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        p2 = f2_pack(ex2(x0), ex2(x1));
+      }
+      ls2[i & 3] = fadd2(ls2[i & 3], p2);
+      float p0, p1;
+      f2_unpack(p2, p0, p1);
+      pk[i] = pack16<F16>(p0, p1);
+    }
+    tmem_st16(tP + c * 16, pk);
+  }
+  const uint64_t t2 = fadd2(fadd2(ls2[0], ls2[1]), fadd2(ls2[2], ls2[3]));
+  float a, b;
+  f2_unpack(t2, a, b);
+  return a + b;
+}
+
 template <int D, bool F16>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -154,6 +208,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* bar_p = bar_s + 2;       // [2][2] P_t keys 0-63 / 64-127 written (O_t rescaled before)
   uint64_t* bar_o = bar_p + 4;       // [2]  all MMAs of tile t complete
   uint64_t* bar_done = bar_o + 2;    // [1]  every MMA of the CTA complete
+  uint64_t* bar_pv = bar_done + 1;   // [1]  (one tile only) O += P V of one more KV tile complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   AbortState* ab = reinterpret_cast<AbortState*>(smem + C::OFF_MISC + 4);
 
@@ -189,6 +244,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bar_o[t], 1);
     }
     mbar_init(bar_done, 1);
+    if (C::TILES == 1) mbar_init(bar_pv, 1);
     ab->flag = 0;
     fence_mbar_init();
   }
@@ -225,9 +281,41 @@ __global__ void __launch_bounds__(384, 1)
       int issued_k[NS], issued_v[NS];
       for (int s = 0; s < NS; ++s) issued_k[s] = issued_v[s] = -1;
       bool ok = true;
-      for (int j = j_begin; j < j_end && ok; ++j) {
-        if (!fwd_tile_active(p, bmask, qb0, j) && (C::TILES == 1 || !fwd_tile_active(p, bmask, qb0 + 1, j)))
-          continue;
+      if constexpr (C::TILES == 1) {
+        // S(a+1) is issued before O += P(a) V(a), so K runs ahead of V: K0 V0 K1 K2 V1 K3 V2 ...
+        // K(a) waits for S(a-NS) to release its stage, V(a-1) for O += P(a-1-NS) V(a-1-NS).
+        int a = 0, j_prev = -1;
+        auto load_v = [&](int jv, int m) -> bool {
+          const int vs = m % NS;
+          const uint32_t vph = (uint32_t)(m / NS) & 1u;
+          if (!mbar_wait(&bar_ve[vs], vph ^ 1u, ab, lim, WAIT_FWD_LOAD + 2)) return false;
+          mbar_arrive_expect_tx(&bar_vf[vs], C::TILE_BYTES);
+          for (int pn = 0; pn < C::PANELS; ++pn)
+            tma_load_3d(smem + C::OFF_V + vs * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmV, &bar_vf[vs], pn * 64,
+                        jv * 128, bh);
+          issued_v[vs] = (int)vph;
+          return true;
+        };
+        for (int j = j_begin; j < j_end && ok; ++j) {
+          if (!fwd_tile_active(p, bmask, qb0, j)) continue;
+          const int ks = a % NS;
+          const uint32_t kph = (uint32_t)(a / NS) & 1u;
+          ok = mbar_wait(&bar_ke[ks], kph ^ 1u, ab, lim, WAIT_FWD_LOAD + 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bar_kf[ks], C::TILE_BYTES);
+          for (int pn = 0; pn < C::PANELS; ++pn)
+            tma_load_3d(smem + C::OFF_K + ks * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmK, &bar_kf[ks], pn * 64,
+                        j * 128, bh);
+          issued_k[ks] = (int)kph;
+          if (a == 0) ok = load_v(j, 0);
+          else if (a >= 2) ok = load_v(j_prev, a - 1);
+          j_prev = j;
+          ++a;
+        }
+        if (ok && a >= 2) ok = load_v(j_prev, a - 1);
+      }
+      for (int j = j_begin; C::TILES == 2 && j < j_end && ok; ++j) {
+        if (!fwd_tile_active(p, bmask, qb0, j) && !fwd_tile_active(p, bmask, qb0 + 1, j)) continue;
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
         ok = mbar_wait(&bar_ke[s], ph ^ 1, ab, lim, WAIT_FWD_LOAD + 1);
@@ -273,6 +361,48 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = true;
       for (int t = 0; t < 2 && ok; ++t)
         if (qb0 + t < p.nb && (C::TILES == 2 || t == 0)) ok = mbar_wait_spin(&bar_q[t], 0, ab, lim, WAIT_FWD_MMA + 1);
+      if constexpr (C::TILES == 1) {
+        // Order S(0), S(1), PV(0), S(2), PV(1), ...: S(a) lands in buffer a & 1 right behind
+        // PV(a-2), the last reader of that buffer's P (the tensor pipe runs in order).
+        auto issue_pv = [&](int k) -> bool {  // O += P(k) V(k)
+          const uint32_t b = (uint32_t)(k & 1), use = (uint32_t)(k >> 1) & 1u;
+          const int vs = k % NS;
+          if (!mbar_wait_spin(&bar_vf[vs], (uint32_t)(k / NS) & 1u, ab, lim, WAIT_FWD_MMA + 3)) return false;
+          const uint64_t dv = dv_base + (uint64_t)(vs * TILE16);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {  // keys 0-63 come from softmax warpgroup 0, 64-127 from 1
+            if (!mbar_wait_spin(&bar_p[2 * b + hf], use, ab, lim, WAIT_FWD_MMA + 4)) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
+              umma_ts(tmem + 256u, tmem + b * 128u + kk * 8, dv + (uint64_t)(kk * (2048 >> 4)), IDESC_O,
+                      (k > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&bar_ve[vs]);
+          umma_commit(bar_pv);
+          return true;
+        };
+        int a = 0;
+        for (int j = j_begin; j < j_end && ok; ++j) {
+          if (!fwd_tile_active(p, bmask, qb0, j)) continue;
+          if (a >= 2) ok = issue_pv(a - 2);
+          const int ks = a % NS;
+          if (ok) ok = mbar_wait_spin(&bar_kf[ks], (uint32_t)(a / NS) & 1u, ab, lim, WAIT_FWD_MMA + 2);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t b = (uint32_t)(a & 1);
+          const uint64_t dk = dk_base + (uint64_t)(ks * TILE16);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {  // S(a) = Q K_j^T
+            const uint32_t off16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
+            umma_ss(tmem + b * 128u, dq_base + off16, dk + off16, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bar_s[b]);
+          umma_commit(&bar_ke[ks]);
+          ++a;
+        }
+        for (int k = a >= 2 ? a - 2 : 0; k < a && ok; ++k) ok = issue_pv(k);
+      }
       uint32_t p_phase[2] = {0u, 0u};
       bool o_started[2] = {false, false};
       bool prev_act[2] = {false, false};
@@ -280,9 +410,9 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t prev_ph = 0;
       int it = 0;
 
-      for (int j = j_begin; j < j_end && ok; ++j) {
+      for (int j = j_begin; C::TILES == 2 && j < j_end && ok; ++j) {
         const bool act0 = fwd_tile_active(p, bmask, qb0, j);
-        const bool act1 = C::TILES == 2 && fwd_tile_active(p, bmask, qb0 + 1, j);
+        const bool act1 = fwd_tile_active(p, bmask, qb0 + 1, j);
         if (!act0 && !act1) continue;
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
@@ -363,93 +493,120 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ softmax warpgroups
     reg_alloc<C::REGS_SOFTMAX>();
-    const int t = (warp - 4) >> 2;    // warps 4-7: tile 0, warps 8-11: tile 1
-    const uint32_t wq = warp & 3;      // TMEM lane quarter this warp may touch
-    const int r = wq * 32 + lane;      // row inside the tile
-    const int qb = qb0 + t;
-    const bool tvalid = qb < p.nb && (C::TILES == 2 || t == 0);
-    const uint32_t lane_off = (wq * 32u) << 16;
-    const uint32_t tS_row = tmem + lane_off + t * 128u;
-    const uint32_t tO_row = tmem + lane_off + 256u + t * D;
-    const float sl2 = p.scale_log2;
-    const Ex2PolyConsts ek = ex2_poly_consts();
-    float m_ref = -INFINITY;  // reference max, log2 domain, scale folded in
-    float l = 0.f;            // running sum of exp2(x - m_ref)
-    uint32_t s_phase = 0;
-    bool o_started = false;
-    bool ok = true;
+    if constexpr (C::TILES == 1) {
+      // One tile: warpgroup h takes key columns [64h, 64h+64) of every row; row r is thread r
+      // of each. The halves exchange their row maxima once per KV tile, so both keep the same
+      // reference max; P of keys [64h, 64h+64) is the half that O += P V waits on as half h.
+      const int h = (warp - 4) >> 2;
+      const uint32_t wq = warp & 3;      // TMEM lane quarter this warp may touch
+      const int r = wq * 32 + lane;      // row inside the tile
+      const int qb = qb0;
+      const bool tvalid = qb < p.nb;     // uniform over the CTA
+      const uint32_t lane_off = (wq * 32u) << 16;
+      const uint32_t tS_row = tmem + lane_off;  // S buffer b at column 128 b
+      const uint32_t tO_row = tmem + lane_off + 256u;
+      float* xch = reinterpret_cast<float*>(smem + C::OFF_XCH);  // [parity][half][row]
+      const float sl2 = p.scale_log2;
+      const Ex2PolyConsts ek = ex2_poly_consts();
+      float m_ref = -INFINITY;  // reference max, log2 domain, scale folded in
+      float l = 0.f;            // this half's running sum of exp2(x - m_ref)
+      bool o_started = false;
+      bool ok = true;
+      int a = 0;                // active KV tiles so far
 
-    if (tvalid) {
-      for (int j = j_begin; j < j_end; ++j) {
+      for (int j = j_begin; tvalid && j < j_end; ++j) {
         if (!fwd_tile_active(p, bmask, qb, j)) continue;
-        ok = warp_wait(&bar_s[t], s_phase, ab, lim, WAIT_FWD_SOFTMAX + 1);
-        if (!ok) break;
-        s_phase ^= 1u;
-        tc_fence_after();
-
-        uint32_t su[128];  // this row's 128 scores (fp32 bits)
-        tmem_ld128(tS_row, su);
-        // Elementwise mask: on the causal diagonal band key 128j+c is visible to row 128qb+r iff
-        // 128j+c <= 128qb+r+causal_off (c <= r for the square problem); in a partial last key
-        // tile keys 128j+c >= Nk do not exist (TMA filled zeros).
+        const uint32_t b = (uint32_t)(a & 1);
+        const uint32_t tS = tS_row + b * 128u;
         const bool diag = p.causal && (128 * j + 127 > 128 * qb + p.causal_off);
         const bool masked = diag || (128 * j + 128 > p.Nk);
-        if (masked) {
-          const int lim = min(diag ? 128 * (qb - j) + r + p.causal_off + 1 : 128, p.Nk - 128 * j);
+        uint32_t su[64];  // this row's scores of this half (fp32 bits)
+        float mh = -INFINITY;
+        if (ok) ok = warp_wait(&bar_s[b], (uint32_t)(a >> 1) & 1u, ab, lim, WAIT_FWD_SOFTMAX + 1);
+        if (ok) {
+          tc_fence_after();
+          tmem_ld64(tS + 64u * h, su);
+          if (masked) {  // same rule as two tiles, for key columns 64h..64h+63
+            const int lim_c = min(diag ? 128 * (qb - j) + r + p.causal_off + 1 : 128, p.Nk - 128 * j) - 64 * h;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c >= lim) su[c] = 0xff800000u;  // -inf
+            for (int c = 0; c < 64; ++c)
+              if (c >= lim_c) su[c] = 0xff800000u;  // -inf
+          }
+          float mc[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float m = fmax3(__uint_as_float(su[k]), __uint_as_float(su[k + 4]), __uint_as_float(su[k + 8]));
+#pragma unroll
+            for (int c = 12; c < 60; c += 8) m = fmax3(m, __uint_as_float(su[c + k]), __uint_as_float(su[c + 4 + k]));
+            mc[k] = fmaxf(m, __uint_as_float(su[60 + k]));
+          }
+          mh = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+          xch[(b * 2 + h) * 128 + r] = mh;
         }
-        // Row max: 8 independent chains of three-input max, then a short tree.
-        float mc[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          float m = fmax3(__uint_as_float(su[k]), __uint_as_float(su[k + 8]), __uint_as_float(su[k + 16]));
-#pragma unroll
-          for (int c = 24; c < 120; c += 16) m = fmax3(m, __uint_as_float(su[c + k]), __uint_as_float(su[c + 8 + k]));
-          mc[k] = fmaxf(m, __uint_as_float(su[120 + k]));
+        // Both halves' S columns are read before either half writes P over them (P of keys
+        // 64-127 lands on S columns 32-63); a failed wait anywhere ends the loop for all.
+        tc_fence_before();
+        if (!named_bar_and(1, 256, ok)) {
+          ok = false;
+          break;
         }
-        const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
+        tc_fence_after();
+        const float mx = fmaxf(mh, xch[(b * 2 + (h ^ 1)) * 128 + r]);
         const float cand = mx * sl2;
         float alpha = 1.f;
         if (cand > m_ref + 8.f) {  // also taken on the first visible tile (m_ref = -inf)
           alpha = ex2(m_ref - cand);
           m_ref = cand;
         }
-        if (o_started && __any_sync(0xffffffffu, alpha != 1.f)) {
-          // O_t already holds every earlier PV (S_t's commit retired them): rescale in place.
+        if (h == 0 && o_started && __any_sync(0xffffffffu, alpha != 1.f)) {
+          // S(a) was issued before O += P(a-1) V(a-1): wait for that PV, then rescale O in
+          // place, all columns, before this half's P lets O += P(a) V(a) start.
+          ok = warp_wait(bar_pv, (uint32_t)(a - 1) & 1u, ab, lim, WAIT_FWD_SOFTMAX + 2);
+          if (ok) {
+            tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t u[32];
-            tmem_ld32(tO_row + c * 32, u);
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t u[32];
+              tmem_ld32(tO_row + c * 32, u);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-            tmem_st32(tO_row + c * 32, u);
+              for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+              tmem_st32(tO_row + c * 32, u);
+            }
           }
         }
         l *= alpha;
-        const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        const uint64_t sl2_2 = f2_pack(sl2, sl2), mneg_2 = f2_pack(mneg, mneg);
-        if (masked)
-          l += softmax_exp_store<F16, false, 0u>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[2 * t]);
-        else
-          l += softmax_exp_store<F16, true, C::EXP_EMU_MASK>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[2 * t]);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar_p[2 * t + 1]);
+        if (ok) {
+          const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
+          const uint64_t sl2_2 = f2_pack(sl2, sl2), mneg_2 = f2_pack(mneg, mneg);
+          const uint32_t tP = tS + 32u * h;  // keys 64h..64h+63 -> 32 packed columns
+          if (masked)
+            l += softmax_exp_store64<F16, false, 0u>(su, sl2_2, mneg_2, tP, ek);
+          else
+            l += softmax_exp_store64<F16, true, C::EXP_EMU_MASK>(su, sl2_2, mneg_2, tP, ek);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar_p[2 * b + h]);
+        }
         o_started = true;
+        ++a;
       }
 
       // ---------------------------------------------------------------- epilogue
-      if (ok) ok = warp_wait(&bar_o[t], 0, ab, lim, WAIT_FWD_EPILOGUE + 1);
-      uint8_t* stage = smem + C::OFF_Q + t * C::TILE_BYTES;  // Q_t is no longer read
-      if (ok) {
+      // Row sum of both halves, through the parity slot the last KV tile did not use (its
+      // last readers passed the last exchange barrier before anyone got here).
+      float* lx = xch + (a & 1) * 2 * 128;
+      if (tvalid) lx[h * 128 + r] = l;
+      ok = named_bar_and(1, 256, ok);
+      const float l_tot = tvalid ? lx[r] + lx[128 + r] : 0.f;
+      if (ok && tvalid) ok = warp_wait(&bar_o[0], 0, ab, lim, WAIT_FWD_EPILOGUE + 1);
+      uint8_t* stage = smem + C::OFF_Q;  // Q is no longer read
+      if (ok && tvalid) {
         tc_fence_after();
-        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const float inv_l = (l_tot > 0.f) ? 1.f / l_tot : 0.f;
         const uint32_t sstage = smem_u32(stage);
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = h * (D / 64); c < (h + 1) * (D / 64); ++c) {  // this half's D/2 output columns
           uint32_t u[32];
           if (o_started) {
             tmem_ld32(tO_row + c * 32, u);
@@ -461,23 +618,21 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             w[i] = pack16<F16>(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
-          const int col0 = c * 32;                   // first column of this chunk
+          const int col0 = c * 32;
           const uint32_t panel = sstage + (col0 >> 6) * C::PANEL_BYTES;
-          const uint32_t chunk0 = (col0 & 63) >> 3;  // 16-byte chunk inside the 128-byte row
+          const uint32_t chunk0 = (col0 & 63) >> 3;
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             st_shared_v4(panel + sw128_offset(r, chunk0 + q), w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         }
         fence_proxy_async_smem();
         const int row = qb * 128 + r;
-        const float lse_row = (l > 0.f) ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        const float lse_row = (l_tot > 0.f) ? (m_ref + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
         if (p.nsplit > 1) {
-          // Split of the key range: this split's O / l (fp32, re-read from TMEM) and LSE for the
-          // merge kernel, every row of the tile (the buffers are padded to Np).
           const size_t prow = ((size_t)bh * p.nsplit + split) * p.Np + row;
           float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D);
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = h * (D / 64); c < (h + 1) * (D / 64); ++c) {
             uint32_t u[32];
             if (o_started) {
               tmem_ld32(tO_row + c * 32, u);
@@ -490,17 +645,158 @@ __global__ void __launch_bounds__(384, 1)
               dst[c * 8 + q] = make_float4(__uint_as_float(u[4 * q]) * inv_l, __uint_as_float(u[4 * q + 1]) * inv_l,
                                            __uint_as_float(u[4 * q + 2]) * inv_l, __uint_as_float(u[4 * q + 3]) * inv_l);
           }
-          p.lse_part[prow] = lse_row;
-        } else if (row < p.N) {  // rows of a partial last tile beyond N are not stored (the O store clips them)
+          if (h == 0) p.lse_part[prow] = lse_row;
+        } else if (h == 0 && row < p.N) {
           p.lse[(size_t)bh * p.N + row] = lse_row;
         }
       }
-      // Every thread of the warpgroup reaches this barrier (tvalid is uniform per warpgroup).
-      named_bar_sync(1 + t, 128);
-      if (p.nsplit == 1 && wq == 0 && lane == 0 && *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
+      named_bar_sync(1, 256);  // both halves of the output tile are staged
+      if (tvalid && p.nsplit == 1 && h == 0 && wq == 0 && lane == 0 &&
+          *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
         for (int pn = 0; pn < C::PANELS; ++pn) tma_store_3d(&tmO, stage + pn * C::PANEL_BYTES, pn * 64, qb * 128, bh);
         bulk_commit_group();
         bulk_wait_group_read0();
+      }
+    } else {
+      const int t = (warp - 4) >> 2;    // warps 4-7: tile 0, warps 8-11: tile 1
+      const uint32_t wq = warp & 3;      // TMEM lane quarter this warp may touch
+      const int r = wq * 32 + lane;      // row inside the tile
+      const int qb = qb0 + t;
+      const bool tvalid = qb < p.nb;
+      const uint32_t lane_off = (wq * 32u) << 16;
+      const uint32_t tS_row = tmem + lane_off + t * 128u;
+      const uint32_t tO_row = tmem + lane_off + 256u + t * D;
+      const float sl2 = p.scale_log2;
+      const Ex2PolyConsts ek = ex2_poly_consts();
+      float m_ref = -INFINITY;  // reference max, log2 domain, scale folded in
+      float l = 0.f;            // running sum of exp2(x - m_ref)
+      uint32_t s_phase = 0;
+      bool o_started = false;
+      bool ok = true;
+
+      if (tvalid) {
+        for (int j = j_begin; j < j_end; ++j) {
+          if (!fwd_tile_active(p, bmask, qb, j)) continue;
+          ok = warp_wait(&bar_s[t], s_phase, ab, lim, WAIT_FWD_SOFTMAX + 1);
+          if (!ok) break;
+          s_phase ^= 1u;
+          tc_fence_after();
+
+          uint32_t su[128];  // this row's 128 scores (fp32 bits)
+          tmem_ld128(tS_row, su);
+          // Elementwise mask: on the causal diagonal band key 128j+c is visible to row 128qb+r iff
+          // 128j+c <= 128qb+r+causal_off (c <= r for the square problem); in a partial last key
+          // tile keys 128j+c >= Nk do not exist (TMA filled zeros).
+          const bool diag = p.causal && (128 * j + 127 > 128 * qb + p.causal_off);
+          const bool masked = diag || (128 * j + 128 > p.Nk);
+          if (masked) {
+            const int lim = min(diag ? 128 * (qb - j) + r + p.causal_off + 1 : 128, p.Nk - 128 * j);
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (c >= lim) su[c] = 0xff800000u;  // -inf
+          }
+          // Row max: 8 independent chains of three-input max, then a short tree.
+          float mc[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            float m = fmax3(__uint_as_float(su[k]), __uint_as_float(su[k + 8]), __uint_as_float(su[k + 16]));
+#pragma unroll
+            for (int c = 24; c < 120; c += 16) m = fmax3(m, __uint_as_float(su[c + k]), __uint_as_float(su[c + 8 + k]));
+            mc[k] = fmaxf(m, __uint_as_float(su[120 + k]));
+          }
+          const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
+          const float cand = mx * sl2;
+          float alpha = 1.f;
+          if (cand > m_ref + 8.f) {  // also taken on the first visible tile (m_ref = -inf)
+            alpha = ex2(m_ref - cand);
+            m_ref = cand;
+          }
+          if (o_started && __any_sync(0xffffffffu, alpha != 1.f)) {
+            // O_t already holds every earlier PV (S_t's commit retired them): rescale in place.
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t u[32];
+              tmem_ld32(tO_row + c * 32, u);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+              tmem_st32(tO_row + c * 32, u);
+            }
+          }
+          l *= alpha;
+          const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
+          const uint64_t sl2_2 = f2_pack(sl2, sl2), mneg_2 = f2_pack(mneg, mneg);
+          if (masked)
+            l += softmax_exp_store<F16, false, 0u>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[2 * t]);
+          else
+            l += softmax_exp_store<F16, true, C::EXP_EMU_MASK>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[2 * t]);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar_p[2 * t + 1]);
+          o_started = true;
+        }
+
+        // ---------------------------------------------------------------- epilogue
+        if (ok) ok = warp_wait(&bar_o[t], 0, ab, lim, WAIT_FWD_EPILOGUE + 1);
+        uint8_t* stage = smem + C::OFF_Q + t * C::TILE_BYTES;  // Q_t is no longer read
+        if (ok) {
+          tc_fence_after();
+          const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+          const uint32_t sstage = smem_u32(stage);
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t u[32];
+            if (o_started) {
+              tmem_ld32(tO_row + c * 32, u);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) u[i] = 0u;
+            }
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              w[i] = pack16<F16>(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
+            const int col0 = c * 32;                   // first column of this chunk
+            const uint32_t panel = sstage + (col0 >> 6) * C::PANEL_BYTES;
+            const uint32_t chunk0 = (col0 & 63) >> 3;  // 16-byte chunk inside the 128-byte row
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              st_shared_v4(panel + sw128_offset(r, chunk0 + q), w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          }
+          fence_proxy_async_smem();
+          const int row = qb * 128 + r;
+          const float lse_row = (l > 0.f) ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+          if (p.nsplit > 1) {
+            // Split of the key range: this split's O / l (fp32, re-read from TMEM) and LSE for the
+            // merge kernel, every row of the tile (the buffers are padded to Np).
+            const size_t prow = ((size_t)bh * p.nsplit + split) * p.Np + row;
+            float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D);
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t u[32];
+              if (o_started) {
+                tmem_ld32(tO_row + c * 32, u);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) u[i] = 0u;
+              }
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                dst[c * 8 + q] = make_float4(__uint_as_float(u[4 * q]) * inv_l, __uint_as_float(u[4 * q + 1]) * inv_l,
+                                             __uint_as_float(u[4 * q + 2]) * inv_l, __uint_as_float(u[4 * q + 3]) * inv_l);
+            }
+            p.lse_part[prow] = lse_row;
+          } else if (row < p.N) {  // rows of a partial last tile beyond N are not stored (the O store clips them)
+            p.lse[(size_t)bh * p.N + row] = lse_row;
+          }
+        }
+        // Every thread of the warpgroup reaches this barrier (tvalid is uniform per warpgroup).
+        named_bar_sync(1 + t, 128);
+        if (p.nsplit == 1 && wq == 0 && lane == 0 && *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
+          for (int pn = 0; pn < C::PANELS; ++pn) tma_store_3d(&tmO, stage + pn * C::PANEL_BYTES, pn * 64, qb * 128, bh);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
       }
     }
   }
@@ -512,6 +808,10 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+}
+
+int fwd_tiles_per_cta(int D) {
+  return D == 64 ? FwdCfg<64>::TILES : (D == 256 ? FwdCfg<256>::TILES : FwdCfg<128>::TILES);
 }
 
 template <int D, bool F16>
