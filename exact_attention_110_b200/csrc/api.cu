@@ -167,8 +167,9 @@ namespace {
 int decode_splits(long long BH, int Nq, int Nk, int d, int requested) {
   const int nbk = (Nk + 127) / 128;
   if (requested > 0) return requested < nbk ? requested : nbk;
-  const int tiles_per_cta = fa::fwd_tiles_per_cta(d);  // the forward kernel's query tiles per CTA
-  const long long pairs = BH * (((Nq + 127) / 128 + tiles_per_cta - 1) / tiles_per_cta);
+  const int nb = (Nq + 127) / 128;
+  const int tiles_per_cta = fa::fwd_tiles_per_cta(d, nb);  // the forward kernel's query tiles per CTA
+  const long long pairs = BH * ((nb + tiles_per_cta - 1) / tiles_per_cta);
   const long long target = 3ll * fa::device_sm_count() / 4;
   long long s = (target + pairs - 1) / pairs;
   const long long cap = nbk / 2 > 1 ? nbk / 2 : 1;

@@ -41,19 +41,17 @@
 #ifndef FA_FWD_EXP_EMU_MASK
 #define FA_FWD_EXP_EMU_MASK 0x0u
 #endif
-// Head dimensions (bit d/64: 0x2 d=64, 0x4 d=128, 0x10 d=256) whose forward runs one query
-// tile per CTA with double-buffered S and the softmax split by columns; the others run two
-// ping-ponged tiles. d = 256 has to.
-#ifndef FA_FWD_ONE_TILE_DIMS
-#define FA_FWD_ONE_TILE_DIMS 0x10u
-#endif
+// K/V stages of the one-tile layout at d = 128.
 #ifndef FA_FWD_ONE_TILE_STAGES_D128
 #define FA_FWD_ONE_TILE_STAGES_D128 2
 #endif
 
 namespace fa {
 
-template <int D>
+// ONE: one query tile per CTA (see TILES). Chosen at launch: always at d = 256, and for a
+// problem with a single query tile (N_q <= 128, e.g. decoding), where the two-tile form would
+// leave its second tile empty; two ping-ponged tiles otherwise.
+template <int D, bool ONE>
 struct FwdCfg {
   static constexpr int THREADS = 384;  // warp 0 TMA, warp 1 MMA, warps 4-11 softmax
   // setmaxnreg split of the launch allocation (384 x 168, checked by the build script):
@@ -66,7 +64,7 @@ struct FwdCfg {
   // [0,128) or [128,256) by the parity of a, O in [256, 256+D) -- so the tensor core computes
   // S(a+1) while the softmax works on S(a), and both softmax warpgroups share the tile, each
   // taking 64 of the 128 key columns.
-  static constexpr int TILES = ((FA_FWD_ONE_TILE_DIMS >> (D / 64)) & 1u) ? 1 : 2;
+  static constexpr int TILES = ONE ? 1 : 2;
   static_assert(D != 256 || TILES == 1, "d = 256 needs the one-tile layout");
   static constexpr int NS = TILES == 2 ? ((D == 128) ? 2 : 4)  // K ring and V ring depth
                                        : (D == 256 ? 1 : (D == 128 ? FA_FWD_ONE_TILE_STAGES_D128 : 4));
@@ -183,12 +181,12 @@ __device__ __forceinline__ float softmax_exp_store64(const uint32_t (&su)[64], u
   return a + b;
 }
 
-template <int D, bool F16>
+template <int D, bool F16, bool ONE>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdParams p) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, ONE>;
   constexpr int NS = C::NS;
   extern __shared__ __align__(1024) uint8_t smem[];
 
@@ -810,32 +808,38 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-int fwd_tiles_per_cta(int D) {
-  return D == 64 ? FwdCfg<64>::TILES : (D == 256 ? FwdCfg<256>::TILES : FwdCfg<128>::TILES);
-}
+bool fwd_one_tile(int D, int nb) { return D == 256 || nb == 1; }
 
-template <int D, bool F16>
+int fwd_tiles_per_cta(int D, int nb) { return fwd_one_tile(D, nb) ? 1 : 2; }
+
+template <int D, bool F16, bool ONE>
 static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, ONE>;
   cudaError_t e =
-      cudaFuncSetAttribute(fa_fwd_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+      cudaFuncSetAttribute(fa_fwd_kernel<D, F16, ONE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   dim3 grid((p.nb + C::TILES - 1) / C::TILES * p.nsplit, BH);
-  fa_fwd_kernel<D, F16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
+  fa_fwd_kernel<D, F16, ONE><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
+}
+
+template <bool F16>
+static cudaError_t launch_fwd_dtype(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                    const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream) {
+  if (D == 256) return launch_fwd_t<256, F16, true>(tq, tk, tv, to, p, BH, stream);
+  const bool one = fwd_one_tile(D, p.nb);
+  if (D == 64)
+    return one ? launch_fwd_t<64, F16, true>(tq, tk, tv, to, p, BH, stream)
+               : launch_fwd_t<64, F16, false>(tq, tk, tv, to, p, BH, stream);
+  return one ? launch_fwd_t<128, F16, true>(tq, tk, tv, to, p, BH, stream)
+             : launch_fwd_t<128, F16, false>(tq, tk, tv, to, p, BH, stream);
 }
 
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream) {
-  if (p.f16) {
-    if (D == 64) return launch_fwd_t<64, true>(tq, tk, tv, to, p, BH, stream);
-    if (D == 256) return launch_fwd_t<256, true>(tq, tk, tv, to, p, BH, stream);
-    return launch_fwd_t<128, true>(tq, tk, tv, to, p, BH, stream);
-  }
-  if (D == 64) return launch_fwd_t<64, false>(tq, tk, tv, to, p, BH, stream);
-  if (D == 256) return launch_fwd_t<256, false>(tq, tk, tv, to, p, BH, stream);
-  return launch_fwd_t<128, false>(tq, tk, tv, to, p, BH, stream);
+  return p.f16 ? launch_fwd_dtype<true>(D, tq, tk, tv, to, p, BH, stream)
+               : launch_fwd_dtype<false>(D, tq, tk, tv, to, p, BH, stream);
 }
 
 }  // namespace fa

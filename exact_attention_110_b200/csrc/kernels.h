@@ -107,8 +107,10 @@ inline int device_sm_count() {
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream);
 cudaError_t launch_fwd_merge(const FwdMergeParams& p, cudaStream_t stream);
-// 128-row query tiles one forward CTA processes at head dimension D (1 or 2).
-int fwd_tiles_per_cta(int D);
+// Whether the forward runs one 128-row query tile per CTA (head dimension D, nb query tiles),
+// and the tiles per CTA that follow (1 or 2).
+bool fwd_one_tile(int D, int nb);
+int fwd_tiles_per_cta(int D, int nb);
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,

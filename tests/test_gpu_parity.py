@@ -65,6 +65,9 @@ SMALL = [
     (1, 1, 333, 128, True, None),
     (1, 1, 641, 64, True, "bernoulli"),
     (1, 1, 1000, 128, False, None),
+    # a single query tile runs the one-tile kernel (S double-buffered, columns split)
+    (1, 2, 100, 128, True, None),
+    (2, 1, 128, 128, False, "bernoulli"),
 ]
 
 
@@ -88,6 +91,7 @@ FP16 = [
     (2, 1, 640, 64, True, None),
     (1, 2, 512, 128, True, None),
     (1, 1, 333, 128, False, "bernoulli"),
+    (1, 2, 96, 128, True, None),       # one query tile: the one-tile kernel in fp16
 ]
 
 
@@ -156,6 +160,7 @@ DECODE = [
     (2, 1, 64, 2048, 128, False, 1, "bf16"),     # one piece: written directly, no merge
     (1, 3, 8, 3000, 64, False, 5, "f16"),
     (1, 2, 40, 900, 256, True, 0, "bf16"),      # head dim 256
+    (2, 2, 4, 5000, 128, True, 0, "f16"),       # fp16, bottom-right causal, library's split
 ]
 
 
