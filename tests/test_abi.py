@@ -151,3 +151,30 @@ def test_decode_argument_checks_and_workspace(lib):
     assert call(nq=0) == 1 and call(nk=0) == 1 and call(ns=-1) == 1 and call(dt=5) == 1
     assert call(d=96) == 2
     assert call(wsb=10) == 5  # two pieces need a workspace
+
+
+def test_decode_piece_choice(lib):
+    """The library's piece count (num_splits = 0): enough (b, h, CTA) units for about three
+    quarters of a 148-SM wave, at least two 128-key tiles per piece. A CTA holds one query tile
+    when there is only one (N_q <= 128) or d = 256, else two. (Without a GPU the SM count falls
+    back to 148, the B200's.)"""
+    lib.fa_fwd_decode_workspace_bytes.restype = ctypes.c_size_t
+    ws = lib.fa_fwd_decode_workspace_bytes
+
+    def pieces(B, H, nq, nk, d):
+        n0 = ws(B, H, nq, nk, d, 0)
+        if n0 == 0:
+            return 1
+        hits = [k for k in range(2, 257) if ws(B, H, nq, nk, d, k) == n0]
+        assert len(hits) == 1
+        return hits[0]
+
+    target = 3 * 148 // 4  # 111
+    assert pieces(8, 16, 1, 16384, 128) == 1                    # 128 CTAs already
+    assert pieces(4, 16, 1, 16384, 128) == -(-target // 64)     # 64 heads: 2 pieces
+    assert pieces(1, 1, 1, 16384, 128) == 64                    # 111 wanted, capped at 128 key tiles / 2
+    assert pieces(1, 1, 1, 65536, 128) == target                # 512 key tiles: 111 pieces
+    assert pieces(1, 1, 1, 1024, 128) == 4                      # capped: 8 key tiles / 2
+    # N_q = 200 is two query tiles: one CTA per head at d = 128, two at d = 256
+    assert pieces(4, 16, 200, 16384, 128) == 2
+    assert pieces(4, 16, 200, 16384, 256) == 1
