@@ -125,6 +125,7 @@ fa_status fa_fwd_ex(int dtype, const void* q, const void* k, const void* v, void
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID;
   fa_status st = check_common(B, H, N, d, scale, true);
   if (st != FA_OK) return st;
+  if (!(scale > 0.f)) return FA_ERR_UNSUPPORTED;  // see check_decode
   if (!get_encoder()) return FA_ERR_CUDA;
   const long long BH = (long long)B * H;
   alignas(64) CUtensorMap tq, tk, tv, to;
@@ -198,6 +199,11 @@ DecodeWorkspace decode_layout(void* base, long long BH, int Nq, int d, int nspli
 fa_status check_decode(int B, int H, int Nq, int Nk, int d, float scale, int nsplit) {
   if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || nsplit < 0 || !isfinite(scale)) return FA_ERR_INVALID;
   if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  // The forward's softmax takes (max of a row's raw scores) x scale as its reference max, which
+  // is the row max of the scaled scores only for scale >= 0 (a negative scale would let P grow
+  // to 2^(row range) and overflow), and it masks scores as -inf before scaling, which scale = 0
+  // would turn into NaN. So the scale must be positive, as in the backward.
+  if (!(scale > 0.f)) return FA_ERR_UNSUPPORTED;
   const long long BH = (long long)B * H;
   if (BH > 65535) return FA_ERR_UNSUPPORTED;
   if ((long long)Nq * d > (1ll << 31) / 2 || (long long)Nk * d > (1ll << 31) / 2) return FA_ERR_UNSUPPORTED;

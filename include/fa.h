@@ -51,7 +51,7 @@ typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID = 1,     /* null/misaligned pointer, non-positive size, non-finite scale */
   FA_ERR_UNSUPPORTED = 2, /* valid but not implemented: d not in {64,128} (256: forward only);
-                             backward scale <= 0 */
+                             scale <= 0 */
   FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call or a kernel launch failed */
   FA_ERR_TIMEOUT = 4,     /* a device-side bounded wait gave up (see fa_last_device_status) */
   FA_ERR_WORKSPACE = 5    /* workspace pointer null or smaller than fa_bwd_workspace_bytes */
@@ -69,7 +69,10 @@ typedef enum {
  *   in : q, k, v       bf16 [B][H][N][d]
  *   out: o             bf16 [B][H][N][d]
  *        lse           fp32 [B][H][N]
- *   scale: multiplies q.k (typically 1/sqrt(d)); must be finite.
+ *   scale: multiplies q.k (typically 1/sqrt(d)); must be finite and > 0, else
+ *          FA_ERR_UNSUPPORTED: the softmax's reference max is the largest raw score times the
+ *          scale (the largest scaled score only for a positive scale), and masked scores are
+ *          -inf before scaling (scale 0 would make them NaN).
  * One kernel launch.
  */
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,

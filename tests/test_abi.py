@@ -104,12 +104,22 @@ def test_ex_entry_points_check_dtype_and_mask_stride(lib):
 @pytest.mark.parametrize("scale", [0.0, -0.125])
 def test_backward_needs_positive_scale(lib, scale):
     # The backward folds log2(scale) into the recomputed probabilities: scale <= 0 is refused
-    # up front (the forward accepts any finite scale).
+    # up front (the forward too: see test_forward_refuses_non_positive_scale).
     need = lib.fa_bwd_workspace_bytes(1, 1, 128, 64)
     assert lib.fa_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, scale, 0, None,
                       FAKE, need, None) == 2
     assert lib.fa_bwd_preprocess(FAKE, FAKE, FAKE, 1, 1, 128, 64, scale, FAKE, need, None) == 2
     assert lib.fa_bwd_main(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, scale, 0, None, FAKE, need, None) == 2
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.125, -1.0])
+def test_forward_refuses_non_positive_scale(lib, scale):
+    # The forward's reference max is the largest raw score times the scale (a row max of the
+    # scaled scores only for scale > 0), and masked scores are -inf before scaling (NaN at
+    # scale 0). Refused before any pointer is used.
+    assert lib.fa_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, scale, 0, None, None) == 2
+    assert lib.fa_fwd_ex(1, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, scale, 1, None, 0, None) == 2
+    assert lib.fa_fwd_decode(0, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 4, 256, 64, scale, 0, 1, None, 0, None) == 2
 
 
 def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):
