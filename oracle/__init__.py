@@ -50,6 +50,7 @@ def _load():
         lib.oracle_bwd.argtypes = [dp, dp, dp, dp, i64, i32, i32, f64, i32, u8p, i32, dp, dp, dp, dp]
         lib.oracle_online_fwd.argtypes = [dp, dp, dp, i64, i32, i32, f64, i32, u8p, i32, i32, i32, dp, dp]
         lib.oracle_fwd_qk.argtypes = [dp, dp, dp, i64, i32, i32, i32, f64, i32, dp, dp]
+        lib.oracle_bwd_qk.argtypes = [dp, dp, dp, dp, i64, i32, i32, i32, f64, i32, dp, dp, dp, dp]
         _lib = lib
     return _lib
 
@@ -131,6 +132,21 @@ def attention_bwd(q, k, v, do, scale: float, causal: bool = False, mask=None, ma
     m, mp = _mask_arg(mask, N, mask_bs)
     _load().oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), B * H, N, d, float(scale), int(causal), mp,
                        mask_bs, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(D))
+    return dq, dk, dv, D
+
+
+def attention_bwd_qk(q, k, v, do, scale: float, causal: bool = False):
+    """Analytic backward for general shapes (the gradient of attention_fwd_qk): q, do
+    [B, H, Nq, d]; k, v [B, H, Nk, d]; bottom-right causal alignment. Returns (dQ, dK, dV, D)."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, Nq, d = _shape(q)
+    Nk = k.shape[2]
+    if k.shape != (B, H, Nk, d) or v.shape != k.shape or do.shape != q.shape:
+        raise ValueError("k and v must be [B, H, Nk, d] with q's B, H and d; do must have q's shape")
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    D = np.empty((B, H, Nq), dtype=np.float64)
+    _load().oracle_bwd_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(do), B * H, Nq, Nk, d, float(scale), int(causal),
+                          _ptr(dq), _ptr(dk), _ptr(dv), _ptr(D))
     return dq, dk, dv, D
 
 

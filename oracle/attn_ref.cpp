@@ -39,6 +39,7 @@
 // unnormalised, divide once at the end), which is how [P1] §主要操作 cuts non-matmul work.
 // It exists only to check that the running recurrence reproduces three-pass softmax.
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -199,6 +200,74 @@ void oracle_fwd_rows(const double* qh, const double* kh, const double* vh, int N
   }
 }
 
+}  // extern "C"
+
+namespace {
+
+// Backward of one head: Nq query rows (qh, doh, dqh: [Nq][d]) against Nk keys (kh, vh, dkh,
+// dvh: [Nk][d]); mk decides which (i, j) are allowed. dK and dV are summed over query rows,
+// so each thread accumulates its own partial copy (dk_part, dv_part: T x Nk x d) and the
+// copies are added at the end. Dh (nullable): [Nq], D_i from its definition.
+void bwd_head(const double* qh, const double* kh, const double* vh, const double* doh, int Nq, int Nk, int d,
+              double scale, const Mask& mk, int T, std::vector<double>& dk_part, std::vector<double>& dv_part,
+              double* dqh, double* dkh, double* dvh, double* Dh) {
+  std::fill(dk_part.begin(), dk_part.end(), 0.0);
+  std::fill(dv_part.begin(), dv_part.end(), 0.0);
+#pragma omp parallel num_threads(T)
+  {
+    int tid = 0;
+#ifdef _OPENMP
+    tid = omp_get_thread_num();
+#endif
+    double* dk_t = dk_part.data() + (size_t)tid * Nk * d;
+    double* dv_t = dv_part.data() + (size_t)tid * Nk * d;
+    std::vector<double> s_row(Nk), p_row(Nk), dp_row(Nk);
+#pragma omp for schedule(dynamic, 4)
+    for (int i = 0; i < Nq; ++i) {
+      const double* qi = qh + (int64_t)i * d;
+      const double* doi = doh + (int64_t)i * d;
+      softmax_row(qi, kh, Nk, d, scale, mk, i, s_row.data(), p_row.data());
+      double Di = 0.0;
+      for (int j = 0; j < Nk; ++j) {
+        if (p_row[j] == 0.0) { dp_row[j] = 0.0; continue; }
+        dp_row[j] = dot(doi, vh + (int64_t)j * d, d);  // dP_ij = dO_i . v_j
+        Di += p_row[j] * dp_row[j];
+      }
+      if (Dh) Dh[i] = Di;
+      double* dqi = dqh + (int64_t)i * d;
+      for (int t = 0; t < d; ++t) dqi[t] = 0.0;
+      for (int j = 0; j < Nk; ++j) {
+        const double pij = p_row[j];
+        if (pij == 0.0) continue;
+        const double dsij = pij * (dp_row[j] - Di);  // dS_ij = P_ij (dP_ij - D_i)
+        const double* kj = kh + (int64_t)j * d;
+        double* dkj = dk_t + (int64_t)j * d;
+        double* dvj = dv_t + (int64_t)j * d;
+        for (int t = 0; t < d; ++t) {
+          dqi[t] += scale * dsij * kj[t];
+          dkj[t] += scale * dsij * qi[t];
+          dvj[t] += pij * doi[t];
+        }
+      }
+    }
+  }
+  // Sum the per-thread partial dK, dV.
+#pragma omp parallel for schedule(static)
+  for (int64_t e = 0; e < (int64_t)Nk * d; ++e) {
+    double a = 0.0, b = 0.0;
+    for (int t = 0; t < T; ++t) {
+      a += dk_part[(size_t)t * Nk * d + e];
+      b += dv_part[(size_t)t * Nk * d + e];
+    }
+    dkh[e] = a;
+    dvh[e] = b;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
 // Backward for all BH heads. Outputs dq, dk, dv: [BH][N][d]; Dvec: [BH][N] holds
 // D_i = sum_j P_ij dP_ij computed from that definition.
 void oracle_bwd(const double* q, const double* k, const double* v, const double* dout, int64_t BH,
@@ -208,64 +277,23 @@ void oracle_bwd(const double* q, const double* k, const double* v, const double*
   const int T = nthreads_used();
   std::vector<double> dk_part((size_t)T * N * d), dv_part((size_t)T * N * d);
   for (int64_t bh = 0; bh < BH; ++bh) {
-    const double* qh = q + bh * N * d;
-    const double* kh = k + bh * N * d;
-    const double* vh = v + bh * N * d;
-    const double* doh = dout + bh * N * d;
-    double* dqh = dq + bh * N * d;
-    double* dkh = dk + bh * N * d;
-    double* dvh = dv + bh * N * d;
-    std::fill(dk_part.begin(), dk_part.end(), 0.0);
-    std::fill(dv_part.begin(), dv_part.end(), 0.0);
-#pragma omp parallel num_threads(T)
-    {
-      int tid = 0;
-#ifdef _OPENMP
-      tid = omp_get_thread_num();
-#endif
-      double* dk_t = dk_part.data() + (size_t)tid * N * d;
-      double* dv_t = dv_part.data() + (size_t)tid * N * d;
-      std::vector<double> s_row(N), p_row(N), dp_row(N);
-#pragma omp for schedule(dynamic, 4)
-      for (int i = 0; i < N; ++i) {
-        const double* qi = qh + (int64_t)i * d;
-        const double* doi = doh + (int64_t)i * d;
-        softmax_row(qi, kh, N, d, scale, mk, i, s_row.data(), p_row.data());
-        double Di = 0.0;
-        for (int j = 0; j < N; ++j) {
-          if (p_row[j] == 0.0) { dp_row[j] = 0.0; continue; }
-          dp_row[j] = dot(doi, vh + (int64_t)j * d, d);  // dP_ij = dO_i . v_j
-          Di += p_row[j] * dp_row[j];
-        }
-        if (Dvec) Dvec[bh * N + i] = Di;
-        double* dqi = dqh + (int64_t)i * d;
-        for (int t = 0; t < d; ++t) dqi[t] = 0.0;
-        for (int j = 0; j < N; ++j) {
-          const double pij = p_row[j];
-          if (pij == 0.0) continue;
-          const double dsij = pij * (dp_row[j] - Di);  // dS_ij = P_ij (dP_ij - D_i)
-          const double* kj = kh + (int64_t)j * d;
-          double* dkj = dk_t + (int64_t)j * d;
-          double* dvj = dv_t + (int64_t)j * d;
-          for (int t = 0; t < d; ++t) {
-            dqi[t] += scale * dsij * kj[t];
-            dkj[t] += scale * dsij * qi[t];
-            dvj[t] += pij * doi[t];
-          }
-        }
-      }
-    }
-    // Sum the per-thread partial dK, dV.
-#pragma omp parallel for schedule(static)
-    for (int64_t e = 0; e < (int64_t)N * d; ++e) {
-      double a = 0.0, b = 0.0;
-      for (int t = 0; t < T; ++t) {
-        a += dk_part[(size_t)t * N * d + e];
-        b += dv_part[(size_t)t * N * d + e];
-      }
-      dkh[e] = a;
-      dvh[e] = b;
-    }
+    const int64_t off = bh * N * d;
+    bwd_head(q + off, k + off, v + off, dout + off, N, N, d, scale, mk, T, dk_part, dv_part, dq + off, dk + off,
+             dv + off, Dvec ? Dvec + bh * N : nullptr);
+  }
+}
+
+// Backward for general shapes (the gradient of oracle_fwd_qk): q, dout, dq: [BH][Nq][d];
+// k, v, dk, dv: [BH][Nk][d]; Dvec: [BH][Nq]. Causal uses the bottom-right alignment; no mask.
+void oracle_bwd_qk(const double* q, const double* k, const double* v, const double* dout, int64_t BH, int Nq,
+                   int Nk, int d, double scale, int causal, double* dq, double* dk, double* dv, double* Dvec) {
+  Mask mk = make_mask(Nk, causal, nullptr, 128);
+  mk.off = Nk - Nq;
+  const int T = nthreads_used();
+  std::vector<double> dk_part((size_t)T * Nk * d), dv_part((size_t)T * Nk * d);
+  for (int64_t bh = 0; bh < BH; ++bh) {
+    bwd_head(q + bh * Nq * d, k + bh * Nk * d, v + bh * Nk * d, dout + bh * Nq * d, Nq, Nk, d, scale, mk, T,
+             dk_part, dv_part, dq + bh * Nq * d, dk + bh * Nk * d, dv + bh * Nk * d, Dvec ? Dvec + bh * Nq : nullptr);
   }
 }
 

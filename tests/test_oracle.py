@@ -348,3 +348,91 @@ def test_split_keys_and_merge_by_lse_equals_full(oracle_mod):
     o = sum(np.exp(p[1] - lse)[..., None] * p[0] for p in parts)
     np.testing.assert_allclose(o, o_full, rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(lse, l_full, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------------------
+# General-shape backward (the gradient of attention_fwd_qk)
+# ---------------------------------------------------------------------------------------
+
+def allowed_qk(nq, nk, causal):
+    """Bottom-right alignment built directly from its definition: j <= i + (N_k - N_q)."""
+    i = np.arange(nq)[:, None]
+    j = np.arange(nk)[None, :]
+    return (j <= i + (nk - nq)) if causal else np.ones((nq, nk), dtype=bool)
+
+
+@pytest.mark.parametrize("nq,nk,causal", [(9, 40, False), (9, 40, True), (33, 20, False), (20, 20, True)])
+def test_general_backward_matches_torch_autograd(oracle_mod, nq, nk, causal):
+    d = 6
+    q, do = rnd((2, 2, nq, d), 80), rnd((2, 2, nq, d), 81)
+    k, v = rnd((2, 2, nk, d), 82), rnd((2, 2, nk, d), 83)
+    dq, dk, dv, D = oracle_mod.attention_bwd_qk(q, k, v, do, 0.45, causal=causal)
+    tq, tk, tv, to = torch_reference_grads(q, k, v, do, 0.45, allowed_qk(nq, nk, causal))
+    np.testing.assert_allclose(dq, tq, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dk, tk, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dv, tv, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(D, (do * to).sum(-1), rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("nq,nk,causal", [(3, 7, True), (7, 5, True), (4, 9, False)])
+def test_general_backward_matches_finite_differences(oracle_mod, nq, nk, causal):
+    # (7, 5, causal): rows 0 and 1 see no key; their output is the constant 0.
+    d, scale, h = 3, 0.7, 1e-6
+    q, do = rnd((1, 1, nq, d), 84), rnd((1, 1, nq, d), 85)
+    k, v = rnd((1, 1, nk, d), 86), rnd((1, 1, nk, d), 87)
+
+    def loss(q_, k_, v_):
+        o, _ = oracle_mod.attention_fwd_qk(q_, k_, v_, scale, causal=causal)
+        return float((o * do).sum())
+
+    grads = oracle_mod.attention_bwd_qk(q, k, v, do, scale, causal=causal)[:3]
+    for idx, (x, g) in enumerate(zip((q, k, v), grads)):
+        num = np.zeros_like(x)
+        for pos in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[pos] += h
+            xm[pos] -= h
+            args_p, args_m = [q, k, v], [q, k, v]
+            args_p[idx], args_m[idx] = xp, xm
+            num[pos] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        err = np.linalg.norm(num - g) / max(np.linalg.norm(g), 1e-30)
+        assert err < 1e-7, (idx, err)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_general_backward_reduces_to_square(oracle_mod, causal):
+    q, k, v, do = (rnd((1, 2, 45, 8), s) for s in (88, 89, 90, 91))
+    a = oracle_mod.attention_bwd_qk(q, k, v, do, 0.4, causal=causal)
+    b = oracle_mod.attention_bwd(q, k, v, do, 0.4, causal=causal)
+    for x, y in zip(a, b):  # dK, dV: per-thread partial sums, added in a schedule-dependent order
+        np.testing.assert_allclose(x, y, rtol=1e-12, atol=1e-14)
+
+
+def test_general_backward_is_the_suffix_of_the_square_problem(oracle_mod):
+    # A square causal problem whose upstream gradient is zero on all but the last nq rows
+    # has the same dK and dV, and the same dQ on those rows, as nq bottom-right-aligned queries
+    # against all N keys (and dQ = 0 on the other rows).
+    N, nq, d = 50, 11, 5
+    q, k, v = rnd((1, 2, N, d), 92), rnd((1, 2, N, d), 93), rnd((1, 2, N, d), 94)
+    do = rnd((1, 2, N, d), 95)
+    do[:, :, :N - nq] = 0.0
+    dq_sq, dk_sq, dv_sq, _ = oracle_mod.attention_bwd(q, k, v, do, 0.3, causal=True)
+    dq, dk, dv, _ = oracle_mod.attention_bwd_qk(q[:, :, N - nq:], k, v, do[:, :, N - nq:], 0.3, causal=True)
+    np.testing.assert_allclose(dq, dq_sq[:, :, N - nq:], rtol=1e-12, atol=1e-13)
+    np.testing.assert_array_equal(dq_sq[:, :, :N - nq], 0.0)
+    np.testing.assert_allclose(dk, dk_sq, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dv, dv_sq, rtol=1e-12, atol=1e-13)
+
+
+def test_general_backward_rows_that_see_nothing(oracle_mod):
+    # N_q > N_k, causal: the first N_q - N_k rows see no key. Their dQ is exactly zero and
+    # their upstream gradient reaches neither dK nor dV.
+    nq, nk, d = 12, 5, 4
+    q, k, v, do = rnd((1, 1, nq, d), 96), rnd((1, 1, nk, d), 97), rnd((1, 1, nk, d), 98), rnd((1, 1, nq, d), 99)
+    dq, dk, dv, D = oracle_mod.attention_bwd_qk(q, k, v, do, 0.5, causal=True)
+    assert np.all(dq[0, 0, :nq - nk] == 0) and np.all(D[0, 0, :nq - nk] == 0)
+    do2 = do.copy()
+    do2[:, :, :nq - nk] = rnd((1, 1, nq - nk, d), 100) * 7.0
+    _, dk2, dv2, _ = oracle_mod.attention_bwd_qk(q, k, v, do2, 0.5, causal=True)
+    np.testing.assert_allclose(dk, dk2, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(dv, dv2, rtol=1e-13, atol=1e-15)
