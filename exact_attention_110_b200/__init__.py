@@ -8,6 +8,7 @@ the library is missing, every call raises -- there is no fallback implementation
     o, lse = forward(q, k, v, causal=False, block_mask=None, scale=None)
     dq, dk, dv = backward(q, k, v, o, do, lse, causal=False, block_mask=None, scale=None)
     o, lse = forward_decode(q, k, v, causal=False, scale=None, num_splits=0)   # Nq != Nk
+    dq, dk, dv = backward_qk(q, k, v, o, do, lse, causal=False, scale=None)     # its gradients
 
 q, k, v, o, do: bf16 (or fp16) CUDA tensors [B, H, N, d] of one type, contiguous, d in {64, 128},
 any N >= 1.
@@ -23,7 +24,7 @@ from pathlib import Path
 import torch
 
 __all__ = [
-    "FAError", "forward", "forward_decode", "backward", "bwd_workspace_bytes", "bwd_preprocess", "bwd_main",
+    "FAError", "forward", "forward_decode", "backward", "backward_qk", "bwd_workspace_bytes", "bwd_preprocess", "bwd_main",
     "bwd_dq_finish", "last_device_status", "selftest_wait_timeout", "library", "LIB_PATH",
 ]
 
@@ -82,6 +83,9 @@ def library() -> ctypes.CDLL:
         lib.fa_fwd_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
         lib.fa_fwd_decode.restype = i32
         lib.fa_fwd_decode.argtypes = [i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32, i32, vp, sz, vp]
+        lib.fa_bwd_qk.restype = i32
+        lib.fa_bwd_qk.argtypes = [i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32, vp, sz,
+                                  vp]
         lib.fa_last_device_status.restype = i32
         lib.fa_last_device_status.argtypes = [vp]
         lib.fa_selftest_ex2.restype = i32
@@ -207,6 +211,30 @@ def backward(q, k, v, o, do, lse, causal: bool = False, block_mask=None, scale=N
     _check(library().fa_bwd_ex(_DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
                                _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, _scale(scale, d), int(bool(causal)),
                                _ptr(mask), mstride, _ptr(ws), nbytes, _stream(q.device)), "fa_bwd")
+    return dq, dk, dv
+
+
+def backward_qk(q, k, v, o, do, lse, causal: bool = False, scale=None, workspace=None, dq=None, dk=None, dv=None):
+    """Gradients of forward_decode's result: q, o, do [B, H, Nq, d]; k, v [B, H, Nk, d];
+    lse [B, H, Nq]. causal uses the bottom-right alignment. Returns (dq, dk, dv)."""
+    if q.dim() != 4 or k.dim() != 4 or k.shape != v.shape:
+        raise ValueError("q: [B, H, Nq, d]; k, v: [B, H, Nk, d]")
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if k.shape[:2] != (B, H) or k.shape[3] != d or o.shape != q.shape or do.shape != q.shape:
+        raise ValueError("k, v share q's B, H and d; o and do have q's shape")
+    for t in (q, k, v, o, do):
+        if not t.is_cuda or t.dtype != q.dtype or not t.is_contiguous() or t.device != q.device:
+            raise ValueError("q, k, v, o, do must be contiguous CUDA tensors of one type and device")
+    if q.dtype not in _DTYPES:
+        raise ValueError("q, k, v must be bf16 or fp16")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws, nbytes = _workspace(B, H, Nq, d, q.device, workspace)
+    _check(library().fa_bwd_qk(_DTYPES[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                               _ptr(dq), _ptr(dk), _ptr(dv), B, H, Nq, Nk, d, _scale(scale, d), int(bool(causal)),
+                               _ptr(ws), nbytes, _stream(q.device)), "fa_bwd_qk")
     return dq, dk, dv
 
 

@@ -70,7 +70,7 @@ fa_status check_common(int B, int H, int N, int d, float scale, bool allow_d256 
   if (B <= 0 || H <= 0 || N <= 0 || !isfinite(scale)) return FA_ERR_INVALID;
   if (d != 64 && d != 128 && !(allow_d256 && d == 256)) return FA_ERR_UNSUPPORTED;
   const long long BH = (long long)B * H;
-  if (BH > 65535) return FA_ERR_UNSUPPORTED;               // grid.y limit
+  if (BH > 0x7fffffffll) return FA_ERR_UNSUPPORTED;        // TMA head coordinate (int32)
   if ((long long)N * d > (1ll << 31) / 2) return FA_ERR_UNSUPPORTED;  // per-head elements
   return FA_OK;
 }
@@ -133,6 +133,7 @@ fa_status fa_fwd_ex(int dtype, const void* q, const void* k, const void* v, void
       !encode_bhnd(&tv, v, BH, N, d, f16) || !encode_bhnd(&to, o, BH, N, d, f16))
     return FA_ERR_CUDA;
   fa::FwdParams p;
+  p.BH = BH;
   p.lse = lse;
   p.block_mask = block_mask;
   p.mask_stride = block_mask_head_stride;
@@ -150,7 +151,7 @@ fa_status fa_fwd_ex(int dtype, const void* q, const void* k, const void* v, void
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
   p.f16 = f16;
-  return from_cuda(fa::launch_fwd(d, tq, tk, tv, to, p, (int)BH, static_cast<cudaStream_t>(stream)));
+  return from_cuda(fa::launch_fwd(d, tq, tk, tv, to, p, BH, static_cast<cudaStream_t>(stream)));
 }
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
@@ -205,7 +206,7 @@ fa_status check_decode(int B, int H, int Nq, int Nk, int d, float scale, int nsp
   // would turn into NaN. So the scale must be positive, as in the backward.
   if (!(scale > 0.f)) return FA_ERR_UNSUPPORTED;
   const long long BH = (long long)B * H;
-  if (BH > 65535) return FA_ERR_UNSUPPORTED;
+  if (BH > 0x7fffffffll) return FA_ERR_UNSUPPORTED;  // TMA head coordinate (int32)
   if ((long long)Nq * d > (1ll << 31) / 2 || (long long)Nk * d > (1ll << 31) / 2) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
@@ -237,6 +238,7 @@ fa_status fa_fwd_decode(int dtype, const void* q, const void* k, const void* v, 
       !encode_bhnd(&tv, v, BH, Nk, d, f16) || !encode_bhnd(&to, o, BH, Nq, d, f16))
     return FA_ERR_CUDA;
   fa::FwdParams p;
+  p.BH = BH;
   p.lse = lse;
   p.block_mask = nullptr;
   p.mask_stride = 0;
@@ -255,7 +257,7 @@ fa_status fa_fwd_decode(int dtype, const void* q, const void* k, const void* v, 
   p.timeout_ns = kWaitLimitNs;
   p.f16 = f16;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = fa::launch_fwd(d, tq, tk, tv, to, p, (int)BH, s);
+  cudaError_t e = fa::launch_fwd(d, tq, tk, tv, to, p, BH, s);
   if (e != cudaSuccess || ns == 1) return from_cuda(e);
   fa::FwdMergeParams m;
   m.o_part = w.o_part;
@@ -276,30 +278,179 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d) {
   return layout(nullptr, B, H, N, d).bytes;
 }
 
-fa_status fa_bwd_preprocess_ex(int dtype, const void* o, const void* dO, const float* lse, int B, int H, int N,
-                                  int d, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+// ------------------------------------------------------------------------- backward plans
+// Each stage of the backward is validated and prepared (parameter block, tensor maps) by a
+// plan function that enqueues nothing; the entry points launch only after every plan they
+// need has succeeded, so an argument error never leaves a stage half-run.
+namespace {
+
+// Shapes of one backward problem: N_q query rows and N_k keys per head (N_q = N_k = N for
+// the square calls), causal alignment offset (key j visible to query i iff j <= i + off).
+struct BwdShape {
+  int B, H, Nq, Nk, d;
+  int causal_off;
+};
+
+fa_status check_bwd_shape(const BwdShape& sh, float scale) {
+  fa_status st = check_common(sh.B, sh.H, sh.Nq, sh.d, scale);
+  if (st != FA_OK) return st;
+  st = check_common(sh.B, sh.H, sh.Nk, sh.d, scale);
+  if (st != FA_OK) return st;
+  if (!(scale > 0.f)) return FA_ERR_UNSUPPORTED;  // the backward folds log2(scale) into P
+  return FA_OK;
+}
+
+fa_status plan_bwd_pre(int dtype, const void* o, const void* dO, const float* lse, const BwdShape& sh, float scale,
+                       void* workspace, size_t workspace_bytes, fa::BwdPreParams* p) {
   if (!valid_dtype(dtype)) return FA_ERR_INVALID;
   if (!o || !dO || !lse) return FA_ERR_INVALID;
   if (!aligned16(o) || !aligned16(dO) || !aligned16(lse)) return FA_ERR_INVALID;
-  fa_status st = check_common(B, H, N, d, scale);
+  fa_status st = check_bwd_shape(sh, scale);
   if (st != FA_OK) return st;
-  if (!(scale > 0.f)) return FA_ERR_UNSUPPORTED;  // the backward folds log2(scale) into P
   if (!workspace || !aligned16(workspace)) return FA_ERR_WORKSPACE;
-  Workspace w = layout(workspace, B, H, N, d);
+  Workspace w = layout(workspace, sh.B, sh.H, sh.Nq, sh.d);
   if (workspace_bytes < w.bytes) return FA_ERR_WORKSPACE;
-  fa::BwdPreParams p;
-  p.o = static_cast<const uint16_t*>(o);
-  p.dout = static_cast<const uint16_t*>(dO);
-  p.lse = lse;
+  p->o = static_cast<const uint16_t*>(o);
+  p->dout = static_cast<const uint16_t*>(dO);
+  p->lse = lse;
+  p->delta = w.delta;
+  p->lse2 = w.lse2;
+  p->dq_acc = w.dq_acc;
+  p->rows = (long long)sh.B * sh.H * sh.Nq;
+  p->N = sh.Nq;
+  p->Np = (sh.Nq + 127) / 128 * 128;
+  p->D = sh.d;
+  p->log2_scale = log2f(scale);
+  p->f16 = dtype == FA_DTYPE_F16;
+  return FA_OK;
+}
+
+struct BwdMainPlan {
+  alignas(64) CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdqa;
+  fa::BwdParams p;
+  long long BH;
+  int d;
+};
+
+fa_status plan_bwd_main(int dtype, const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                        const BwdShape& sh, float scale, int causal, const uint8_t* block_mask,
+                        long long block_mask_head_stride, void* workspace, size_t workspace_bytes,
+                        BwdMainPlan* m) {
+  if (!valid_dtype(dtype)) return FA_ERR_INVALID;
+  if (block_mask != nullptr && sh.Nq != sh.Nk) return FA_ERR_INVALID;  // masks are square
+  if (!mask_stride_ok(block_mask, block_mask_head_stride, sh.Nq)) return FA_ERR_INVALID;
+  const int f16 = dtype == FA_DTYPE_F16;
+  if (!q || !k || !v || !dO || !dk || !dv) return FA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_INVALID;
+  fa_status st = check_bwd_shape(sh, scale);
+  if (st != FA_OK) return st;
+  const long long BH = (long long)sh.B * sh.H;
+  const int Np = (sh.Nq + 127) / 128 * 128;
+  if (BH * Np > 0x7fffffffll) return FA_ERR_UNSUPPORTED;  // TMA row coordinate of the dQ accumulator
+  if (!workspace || !aligned16(workspace)) return FA_ERR_WORKSPACE;
+  Workspace w = layout(workspace, sh.B, sh.H, sh.Nq, sh.d);
+  if (workspace_bytes < w.bytes) return FA_ERR_WORKSPACE;
+  if (!get_encoder()) return FA_ERR_CUDA;
+  if (!encode_bhnd(&m->tq, q, BH, sh.Nq, sh.d, f16) || !encode_bhnd(&m->tk, k, BH, sh.Nk, sh.d, f16) ||
+      !encode_bhnd(&m->tv, v, BH, sh.Nk, sh.d, f16) || !encode_bhnd(&m->tdo, dO, BH, sh.Nq, sh.d, f16) ||
+      !encode_bhnd(&m->tdk, dk, BH, sh.Nk, sh.d, f16) || !encode_bhnd(&m->tdv, dv, BH, sh.Nk, sh.d, f16) ||
+      !encode_dq_acc(&m->tdqa, w.dq_acc, BH * Np, sh.d))
+    return FA_ERR_CUDA;
+  fa::BwdParams& p = m->p;
+  p.BH = BH;
   p.delta = w.delta;
   p.lse2 = w.lse2;
   p.dq_acc = w.dq_acc;
-  p.rows = (long long)B * H * N;
-  p.N = N;
-  p.Np = (N + 127) / 128 * 128;
-  p.D = d;
-  p.log2_scale = log2f(scale);
-  p.f16 = dtype == FA_DTYPE_F16;
+  p.block_mask = block_mask;
+  p.mask_stride = block_mask_head_stride;
+  p.N = sh.Nq;
+  p.Np = Np;
+  p.nb = (sh.Nq + 127) / 128;
+  p.Nk = sh.Nk;
+  p.nbk = (sh.Nk + 127) / 128;
+  p.causal = causal ? 1 : 0;
+  p.causal_off = sh.causal_off;
+  p.inv_scale = 1.0f / scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = kWaitLimitNs;
+  p.f16 = f16;
+  m->BH = BH;
+  m->d = sh.d;
+  return FA_OK;
+}
+
+cudaError_t launch_plan(const BwdMainPlan& m, cudaStream_t s) {
+  return fa::launch_bwd_main(m.d, m.tq, m.tk, m.tv, m.tdo, m.tdk, m.tdv, m.tdqa, m.p, m.BH, s);
+}
+
+fa_status plan_dq_finish(int dtype, void* dq, const BwdShape& sh, void* workspace, size_t workspace_bytes,
+                         fa::DqFinishParams* p) {
+  if (!valid_dtype(dtype)) return FA_ERR_INVALID;
+  if (!dq || !aligned16(dq)) return FA_ERR_INVALID;
+  fa_status st = check_bwd_shape(sh, 1.0f);
+  if (st != FA_OK) return st;
+  if (!workspace || !aligned16(workspace)) return FA_ERR_WORKSPACE;
+  Workspace w = layout(workspace, sh.B, sh.H, sh.Nq, sh.d);
+  if (workspace_bytes < w.bytes) return FA_ERR_WORKSPACE;
+  p->dq_acc = w.dq_acc;
+  p->dq = static_cast<uint16_t*>(dq);
+  p->rows = (long long)sh.B * sh.H * sh.Nq;
+  p->N = sh.Nq;
+  p->Np = (sh.Nq + 127) / 128 * 128;
+  p->D = sh.d;
+  p->scale = 1.0f;  // the accumulated dQ already carries the scale (the main kernel folds it into P)
+  p->f16 = dtype == FA_DTYPE_F16;
+  return FA_OK;
+}
+
+// Null and alignment checks of every tensor pointer of a whole backward call (pure host
+// logic, no CUDA call), so that a bad pointer of any stage is refused first.
+fa_status bwd_check_pointers(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                             const float* lse, const void* dq, const void* dk, const void* dv) {
+  const void* ptrs[9] = {q, k, v, o, dO, lse, dq, dk, dv};
+  for (const void* x : ptrs)
+    if (x == nullptr || !aligned16(x)) return FA_ERR_INVALID;
+  return FA_OK;
+}
+
+// The whole backward: every stage planned first, then the three launches.
+fa_status bwd_all(int dtype, const void* q, const void* k, const void* v, const void* o, const void* dO,
+                  const float* lse, void* dq, void* dk, void* dv, const BwdShape& sh, float scale, int causal,
+                  const uint8_t* block_mask, long long block_mask_head_stride, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  fa_status st = bwd_check_pointers(q, k, v, o, dO, lse, dq, dk, dv);
+  if (st != FA_OK) return st;
+  fa::BwdPreParams pre;
+  st = plan_bwd_pre(dtype, o, dO, lse, sh, scale, workspace, workspace_bytes, &pre);
+  if (st != FA_OK) return st;
+  BwdMainPlan m;
+  st = plan_bwd_main(dtype, q, k, v, dO, dk, dv, sh, scale, causal, block_mask, block_mask_head_stride, workspace,
+                     workspace_bytes, &m);
+  if (st != FA_OK) return st;
+  fa::DqFinishParams fin;
+  st = plan_dq_finish(dtype, dq, sh, workspace, workspace_bytes, &fin);
+  if (st != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = fa::launch_bwd_pre(pre, s);
+  if (e == cudaSuccess) e = launch_plan(m, s);
+  if (e == cudaSuccess) e = fa::launch_dq_finish(fin, s);
+  return from_cuda(e);
+}
+
+BwdShape square(int B, int H, int N, int d) { return BwdShape{B, H, N, N, d, 0}; }
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_bwd_preprocess_ex(int dtype, const void* o, const void* dO, const float* lse, int B, int H, int N,
+                               int d, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  fa::BwdPreParams p;
+  fa_status st = plan_bwd_pre(dtype, o, dO, lse, square(B, H, N, d), scale, workspace, workspace_bytes, &p);
+  if (st != FA_OK) return st;
   return from_cuda(fa::launch_bwd_pre(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -311,43 +462,11 @@ fa_status fa_bwd_preprocess(const void* o, const void* dO, const float* lse, int
 fa_status fa_bwd_main_ex(int dtype, const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
                          int B, int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
                          long long block_mask_head_stride, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!valid_dtype(dtype)) return FA_ERR_INVALID;
-  if (!mask_stride_ok(block_mask, block_mask_head_stride, N)) return FA_ERR_INVALID;
-  const int f16 = dtype == FA_DTYPE_F16;
-  if (!q || !k || !v || !dO || !dk || !dv) return FA_ERR_INVALID;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) || !aligned16(dv))
-    return FA_ERR_INVALID;
-  fa_status st = check_common(B, H, N, d, scale);
+  BwdMainPlan m;
+  fa_status st = plan_bwd_main(dtype, q, k, v, dO, dk, dv, square(B, H, N, d), scale, causal, block_mask,
+                               block_mask_head_stride, workspace, workspace_bytes, &m);
   if (st != FA_OK) return st;
-  if (!(scale > 0.f)) return FA_ERR_UNSUPPORTED;  // the backward folds log2(scale) into P
-  if ((long long)B * H * ((N + 127) / 128 * 128) > 0x7fffffffll) return FA_ERR_UNSUPPORTED;  // TMA row coordinate
-  if (!workspace || !aligned16(workspace)) return FA_ERR_WORKSPACE;
-  Workspace w = layout(workspace, B, H, N, d);
-  if (workspace_bytes < w.bytes) return FA_ERR_WORKSPACE;
-  if (!get_encoder()) return FA_ERR_CUDA;
-  const long long BH = (long long)B * H;
-  alignas(64) CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdqa;
-  if (!encode_bhnd(&tq, q, BH, N, d, f16) || !encode_bhnd(&tk, k, BH, N, d, f16) ||
-      !encode_bhnd(&tv, v, BH, N, d, f16) || !encode_bhnd(&tdo, dO, BH, N, d, f16) ||
-      !encode_bhnd(&tdk, dk, BH, N, d, f16) || !encode_bhnd(&tdv, dv, BH, N, d, f16) ||
-      !encode_dq_acc(&tdqa, w.dq_acc, BH * ((N + 127) / 128 * 128), d))
-    return FA_ERR_CUDA;
-  fa::BwdParams p;
-  p.delta = w.delta;
-  p.lse2 = w.lse2;
-  p.dq_acc = w.dq_acc;
-  p.block_mask = block_mask;
-  p.mask_stride = block_mask_head_stride;
-  p.N = N;
-  p.Np = (N + 127) / 128 * 128;
-  p.nb = (N + 127) / 128;
-  p.causal = causal ? 1 : 0;
-  p.inv_scale = 1.0f / scale;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.timeout_ns = kWaitLimitNs;
-  p.f16 = f16;
-  return from_cuda(
-      fa::launch_bwd_main(d, tq, tk, tv, tdo, tdk, tdv, tdqa, p, (int)BH, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_plan(m, static_cast<cudaStream_t>(stream)));
 }
 
 fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B,
@@ -358,23 +477,10 @@ fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* d
 }
 
 fa_status fa_bwd_dq_finish_ex(int dtype, void* dq, int B, int H, int N, int d, void* workspace,
-                                 size_t workspace_bytes, void* stream) {
-  if (!valid_dtype(dtype)) return FA_ERR_INVALID;
-  if (!dq || !aligned16(dq)) return FA_ERR_INVALID;
-  fa_status st = check_common(B, H, N, d, 1.0f);
-  if (st != FA_OK) return st;
-  if (!workspace || !aligned16(workspace)) return FA_ERR_WORKSPACE;
-  Workspace w = layout(workspace, B, H, N, d);
-  if (workspace_bytes < w.bytes) return FA_ERR_WORKSPACE;
+                              size_t workspace_bytes, void* stream) {
   fa::DqFinishParams p;
-  p.dq_acc = w.dq_acc;
-  p.dq = static_cast<uint16_t*>(dq);
-  p.rows = (long long)B * H * N;
-  p.N = N;
-  p.Np = (N + 127) / 128 * 128;
-  p.D = d;
-  p.scale = 1.0f;  // the accumulated dQ already carries the scale (fa_bwd_main folds it into P)
-  p.f16 = dtype == FA_DTYPE_F16;
+  fa_status st = plan_dq_finish(dtype, dq, square(B, H, N, d), workspace, workspace_bytes, &p);
+  if (st != FA_OK) return st;
   return from_cuda(fa::launch_dq_finish(p, static_cast<cudaStream_t>(stream)));
 }
 
@@ -387,15 +493,8 @@ fa_status fa_bwd_ex(int dtype, const void* q, const void* k, const void* v, cons
                     const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale,
                     int causal, const uint8_t* block_mask, long long block_mask_head_stride, void* workspace,
                     size_t workspace_bytes, void* stream) {
-  if (!valid_dtype(dtype)) return FA_ERR_INVALID;
-  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID;
-  if (!mask_stride_ok(block_mask, block_mask_head_stride, N)) return FA_ERR_INVALID;
-  fa_status st = fa_bwd_preprocess_ex(dtype, o, dO, lse, B, H, N, d, scale, workspace, workspace_bytes, stream);
-  if (st != FA_OK) return st;
-  st = fa_bwd_main_ex(dtype, q, k, v, dO, dk, dv, B, H, N, d, scale, causal, block_mask, block_mask_head_stride,
-                      workspace, workspace_bytes, stream);
-  if (st != FA_OK) return st;
-  return fa_bwd_dq_finish_ex(dtype, dq, B, H, N, d, workspace, workspace_bytes, stream);
+  return bwd_all(dtype, q, k, v, o, dO, lse, dq, dk, dv, square(B, H, N, d), scale, causal, block_mask,
+                 block_mask_head_stride, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
@@ -403,6 +502,14 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  const uint8_t* block_mask, void* workspace, size_t workspace_bytes, void* stream) {
   return fa_bwd_ex(FA_DTYPE_BF16, q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, block_mask, 0,
                    workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_qk(int dtype, const void* q, const void* k, const void* v, const void* o, const void* dO,
+                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d, float scale,
+                    int causal, void* workspace, size_t workspace_bytes, void* stream) {
+  const BwdShape sh{B, H, Nq, Nk, d, Nk - Nq};  // bottom-right alignment, as fa_fwd_decode
+  return bwd_all(dtype, q, k, v, o, dO, lse, dq, dk, dv, sh, scale, causal, nullptr, 0, workspace, workspace_bytes,
+                 stream);
 }
 
 fa_status fa_last_device_status(void* stream) {

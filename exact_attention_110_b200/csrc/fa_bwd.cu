@@ -94,10 +94,12 @@ struct BwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// bmask: this (b, h)'s block mask (or null).
+// bmask: this (b, h)'s block mask (or null), [query tiles][key tiles]. Causal: key tile j is
+// active for query tile i when its first key is visible to the tile's last row
+// (128j <= 128i + 127 + causal_off; i >= j for the square problem).
 __device__ __forceinline__ bool bwd_tile_active(const BwdParams& p, const uint8_t* bmask, int i, int j) {
-  if (p.causal && i < j) return false;
-  if (bmask != nullptr && bmask[i * p.nb + j] == 0) return false;
+  if (p.causal && 128 * j > 128 * i + 127 + p.causal_off) return false;
+  if (bmask != nullptr && bmask[i * p.nbk + j] == 0) return false;
   return true;
 }
 
@@ -159,10 +161,14 @@ __global__ void __launch_bounds__(512, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   AbortState* ab = reinterpret_cast<AbortState*>(smem + C::OFF_MISC + 4);
 
-  const int bh = blockIdx.y;
+  const long long bh_l = cta_bh();
+  if (bh_l >= p.BH) return;  // past the last head (head counts above 65535 round the grid up)
+  const int bh = (int)bh_l;
   const uint8_t* bmask = p.block_mask == nullptr ? nullptr : p.block_mask + (size_t)bh * p.mask_stride;
   const int j = blockIdx.x;  // key tile (causal: j = 0 has the most work and starts first)
-  const int i_begin = p.causal ? j : 0;
+  // causal: the first query tile whose last row sees key tile j's first key
+  const int i_first = 128 * j - 127 - p.causal_off;
+  const int i_begin = (p.causal && i_first > 0) ? (i_first + 127) / 128 : 0;
   const uint64_t lim = p.timeout_ns;
 
   if (warp == 0 && lane == 0) {
@@ -396,10 +402,13 @@ __global__ void __launch_bounds__(512, 1)
       const int s = it % NS;
       const float* nlse2 = reinterpret_cast<const float*>(smem + C::OFF_LSE + s * 512) + 64 * h;
       const float* ndel = reinterpret_cast<const float*>(smem + C::OFF_DEL + s * 512) + 64 * h;
-      const bool diag = p.causal && i == j;
-      // Keys of a partial last tile beyond N (zero rows from TMA) take no part: P = 0 there, so
-      // nothing non-finite can reach dQ through them.
-      const bool kpad = 128 * j + kr >= p.N;
+      // Causal band: key 128j+kr is visible to query 128i+q iff 128j+kr <= 128i+q+causal_off,
+      // i.e. q >= qmin (q >= kr on the diagonal tile of the square problem).
+      const bool diag = p.causal && (128 * j + 127 > 128 * i + p.causal_off);
+      const int qmin = kr + 128 * (j - i) - p.causal_off;
+      // Keys of a partial last tile beyond N_k (zero rows from TMA) take no part: P = 0 there,
+      // so nothing non-finite can reach dQ through them.
+      const bool kpad = 128 * j + kr >= p.Nk;
       const int qoff = 64 * h;  // query index of column 0 of this group
 
       // ---- P phase: P^T = exp2(S^T * scale*log2e - LSE*log2e), back into TMEM as bf16
@@ -442,12 +451,12 @@ __global__ void __launch_bounds__(512, 1)
               p2 = ex2(x2);
               p3 = ex2(x3);
             }
-            if (diag) {  // key kr is visible to query qoff+q iff kr <= qoff+q
+            if (diag) {  // key kr is visible to query qoff+q iff qoff+q >= qmin
               const int qq = qoff + q;
-              if (qq < kr) p0 = 0.f;
-              if (qq + 1 < kr) p1 = 0.f;
-              if (qq + 2 < kr) p2 = 0.f;
-              if (qq + 3 < kr) p3 = 0.f;
+              if (qq < qmin) p0 = 0.f;
+              if (qq + 1 < qmin) p1 = 0.f;
+              if (qq + 2 < qmin) p2 = 0.f;
+              if (qq + 3 < qmin) p3 = 0.f;
             }
             if (kpad) p0 = p1 = p2 = p3 = 0.f;
             pf[q] = p0;
@@ -611,19 +620,19 @@ __global__ void __launch_bounds__(512, 1)
 template <int D, bool F16>
 static cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
-                                const CUtensorMap& tdqa, const BwdParams& p, int BH, cudaStream_t stream) {
+                                const CUtensorMap& tdqa, const BwdParams& p, long long BH, cudaStream_t stream) {
   using C = BwdCfg<D>;
   cudaError_t e =
       cudaFuncSetAttribute(fa_bwd_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.nb, BH);
+  const dim3 grid = grid_bh(p.nbk, BH);
   fa_bwd_kernel<D, F16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdk, tdv, tdqa, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
-                            const CUtensorMap& tdqa, const BwdParams& p, int BH, cudaStream_t stream) {
+                            const CUtensorMap& tdqa, const BwdParams& p, long long BH, cudaStream_t stream) {
   if (p.f16) {
     if (D == 64) return launch_bwd_t<64, true>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
     return launch_bwd_t<128, true>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);

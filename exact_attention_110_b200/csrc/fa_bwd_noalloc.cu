@@ -49,6 +49,9 @@ void* scratch_for_current_device(fa_status* st) {
 extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
                                     const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                                     float scale, int causal, const uint8_t* block_mask, void* stream) {
+  // Pointer errors first, before the scratch array's address is looked up (a CUDA call).
+  const fa_status pst = bwd_check_pointers(q, k, v, o, dO, lse, dq, dk, dv);
+  if (pst != FA_OK) return pst;
   const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
   if (need == 0) {  // sizes fa_bwd rejects: let it report the precise reason
     return fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, B, H, N, d, scale, causal, block_mask, nullptr, 0, stream);

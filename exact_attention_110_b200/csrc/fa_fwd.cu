@@ -210,7 +210,9 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   AbortState* ab = reinterpret_cast<AbortState*>(smem + C::OFF_MISC + 4);
 
-  const int bh = blockIdx.y;
+  const long long bh_l = cta_bh();
+  if (bh_l >= p.BH) return;  // past the last head (head counts above 65535 round the grid up)
+  const int bh = (int)bh_l;
   const uint8_t* bmask = p.block_mask == nullptr ? nullptr : p.block_mask + (size_t)bh * p.mask_stride;
   // blockIdx.x = pair index * nsplit + split; causal grids start with the heaviest pairs
   const int pi = (int)blockIdx.x / p.nsplit, split = (int)blockIdx.x - pi * p.nsplit;
@@ -814,19 +816,19 @@ int fwd_tiles_per_cta(int D, int nb) { return fwd_one_tile(D, nb) ? 1 : 2; }
 
 template <int D, bool F16, bool ONE>
 static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream) {
+                                const CUtensorMap& to, const FwdParams& p, long long BH, cudaStream_t stream) {
   using C = FwdCfg<D, ONE>;
   cudaError_t e =
       cudaFuncSetAttribute(fa_fwd_kernel<D, F16, ONE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.nb + C::TILES - 1) / C::TILES * p.nsplit, BH);
+  const dim3 grid = grid_bh((p.nb + C::TILES - 1) / C::TILES * p.nsplit, BH);
   fa_fwd_kernel<D, F16, ONE><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
 
 template <bool F16>
 static cudaError_t launch_fwd_dtype(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                    const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream) {
+                                    const CUtensorMap& to, const FwdParams& p, long long BH, cudaStream_t stream) {
   if (D == 256) return launch_fwd_t<256, F16, true>(tq, tk, tv, to, p, BH, stream);
   const bool one = fwd_one_tile(D, p.nb);
   if (D == 64)
@@ -837,7 +839,7 @@ static cudaError_t launch_fwd_dtype(int D, const CUtensorMap& tq, const CUtensor
 }
 
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream) {
+                       const CUtensorMap& to, const FwdParams& p, long long BH, cudaStream_t stream) {
   return p.f16 ? launch_fwd_dtype<true>(D, tq, tk, tv, to, p, BH, stream)
                : launch_fwd_dtype<false>(D, tq, tk, tv, to, p, BH, stream);
 }

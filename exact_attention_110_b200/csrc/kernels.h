@@ -23,8 +23,18 @@ enum WaitSite : int {
   WAIT_SELFTEST = 0x7700,
 };
 
+// (b, h) of this CTA. Up to 65535 heads the grid's y index is the head; beyond that the
+// heads are spread over y and z (grid_bh), and CTAs past the last head exit at once.
+__device__ __forceinline__ long long cta_bh() { return (long long)blockIdx.z * gridDim.y + blockIdx.y; }
+inline dim3 grid_bh(unsigned x, long long BH) {
+  const unsigned z = (unsigned)((BH + 65534) / 65535);
+  const unsigned y = (unsigned)((BH + z - 1) / z);
+  return dim3(x, y, z);
+}
+
 struct FwdParams {
   float* lse;                  // [BH][N]
+  long long BH;                // heads (B * H)
   const uint8_t* block_mask;   // [nb][nb] (or one per (b, h), mask_stride apart) or null
   long long mask_stride;       // elements between consecutive (b, h) masks; 0 = one shared mask
   int N;                       // query rows per head
@@ -57,13 +67,16 @@ struct BwdPreParams {
 };
 
 struct BwdParams {
+  long long BH;          // heads (B * H)
   const float* delta;    // [BH][Np]  -D
   const float* lse2;     // [BH][Np]  -LSE * log2(e) + log2(scale)
   float* dq_acc;         // [BH][Np][D]
   const uint8_t* block_mask;
   long long mask_stride; // elements between consecutive (b, h) masks; 0 = one shared mask
-  int N, Np, nb;
+  int N, Np, nb;         // query rows, padded to 128, query tiles
+  int Nk, nbk;           // keys, key tiles (N_k = N for the square problem)
   int causal;
+  int causal_off;        // causal: key j is visible to query i iff j <= i + causal_off
   float inv_scale;       // 1 / scale (dV epilogue: P carries the scale)
   float scale_log2;      // scale * log2(e)
   unsigned long long timeout_ns;
@@ -105,7 +118,7 @@ inline int device_sm_count() {
 
 // Launchers (return the launch error, if any).
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& to, const FwdParams& p, int BH, cudaStream_t stream);
+                       const CUtensorMap& to, const FwdParams& p, long long BH, cudaStream_t stream);
 cudaError_t launch_fwd_merge(const FwdMergeParams& p, cudaStream_t stream);
 // Whether the forward runs one 128-row query tile per CTA (head dimension D, nb query tiles),
 // and the tiles per CTA that follow (1 or 2).
@@ -114,7 +127,7 @@ int fwd_tiles_per_cta(int D, int nb);
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
-                            const CUtensorMap& tdqa, const BwdParams& p, int BH, cudaStream_t stream);
+                            const CUtensorMap& tdqa, const BwdParams& p, long long BH, cudaStream_t stream);
 cudaError_t launch_dq_finish(const DqFinishParams& p, cudaStream_t stream);
 
 }  // namespace fa

@@ -32,8 +32,12 @@
  *    backward's dK and dV accumulators would not fit tensor memory). N is any positive length;
  *    a partial last 128-row tile is handled inside the kernels (rows and keys beyond N take no
  *    part and are never written).
+ *  - B*H may be any positive count up to 2^31 - 1 (heads beyond 65535 are spread over two
+ *    grid dimensions); the backward also needs B*H*ceil(N/128)*128 < 2^31.
  *  - stream is a cudaStream_t (NULL = legacy default stream). All calls are asynchronous
- *    on it; argument errors are reported synchronously, before anything is enqueued.
+ *    on it; argument errors are reported synchronously, before anything is enqueued: a
+ *    call that runs several kernels (fa_bwd and its variants) checks every argument of
+ *    every stage before the first launch.
  *  - Not re-entrant on the same output buffers; distinct calls on distinct buffers may run
  *    concurrently on different streams.
  */
@@ -195,6 +199,24 @@ size_t fa_fwd_decode_workspace_bytes(int B, int H, int Nq, int Nk, int d, int ns
 fa_status fa_fwd_decode(int dtype, const void* q, const void* k, const void* v, void* o,
                         float* lse, int B, int H, int Nq, int Nk, int d, float scale, int causal,
                         int nsplit, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward pass for N_q query rows against N_k keys per head: the gradient of the forward that
+ * fa_fwd_decode computes (the problem statement of [P3] §2.1/§2.2 gives Q and K/V their own
+ * lengths), by the same recomputation as fa_bwd ([P3] §4.2; [P1] §主要操作, backward).
+ *   in : q, o, dO  [B][H][Nq][d];  k, v  [B][H][Nk][d]  (dtype as for fa_bwd_ex)
+ *        lse       fp32 [B][H][Nq] from fa_fwd_decode with the same causal flag and scale
+ *   out: dq [B][H][Nq][d];  dk, dv [B][H][Nk][d]
+ *   causal: bottom-right alignment as in fa_fwd_decode (key j visible to query i iff
+ *           j <= i + Nk - Nq). Rows that see no key (Nq > Nk) have LSE = -inf and O = 0;
+ *           they contribute nothing and get dq = 0. No block mask.
+ *   workspace: fa_bwd_workspace_bytes(B, H, Nq, d) bytes (it depends on the query rows only).
+ * Errors as for fa_bwd. With Nq = Nk it computes exactly what fa_bwd_ex computes.
+ */
+fa_status fa_bwd_qk(int dtype, const void* q, const void* k, const void* v, const void* o,
+                    const void* dO, const float* lse, void* dq, void* dk, void* dv, int B, int H,
+                    int Nq, int Nk, int d, float scale, int causal, void* workspace,
+                    size_t workspace_bytes, void* stream);
 
 #define FA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,

@@ -55,7 +55,7 @@ def test_fwd_argument_checks(lib):
     assert fwd(lib, d=512) == 2                  # (d = 256 is a supported forward head dim)
     assert lib.fa_bwd_workspace_bytes(1, 1, 128, 256) == 0   # ... but not a backward one
     assert fwd(lib, N=0) == 1                    # empty sequence -> INVALID
-    assert fwd(lib, B=65536) == 2 and fwd(lib, B=256, H=256) == 2  # B*H above the grid's y limit
+    assert fwd(lib, B=65536, H=65536) == 2      # B*H above the TMA head coordinate's range
 
 
 def test_workspace_size_and_checks(lib):
@@ -188,3 +188,38 @@ def test_decode_piece_choice(lib):
     # N_q = 200 is two query tiles: one CTA per head at d = 128, two at d = 256
     assert pieces(4, 16, 200, 16384, 128) == 2
     assert pieces(4, 16, 200, 16384, 256) == 1
+
+
+def test_backward_checks_every_stage_before_launching(lib):
+    # A misaligned dq (needed only by the last stage) must be refused before the first stage is
+    # enqueued: no CUDA call is made, so this runs without a GPU.
+    need = lib.fa_bwd_workspace_bytes(1, 1, 128, 64)
+    vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.fa_bwd_noalloc.restype = i32
+    lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, f32, i32, vp, vp]
+    args = [FAKE] * 9
+    for i in range(9):
+        bad = list(args)
+        bad[i] = FAKE + 8
+        st = lib.fa_bwd(*bad, 1, 1, 128, 64, 0.125, 0, None, FAKE, need, None)
+        assert st == 1, (i, st)
+        st = lib.fa_bwd_noalloc(*bad, 1, 1, 128, 64, 0.125, 0, None, None)
+        assert st == 1, (i, st)
+        bad[i] = None
+        assert lib.fa_bwd(*bad, 1, 1, 128, 64, 0.125, 0, None, FAKE, need, None) == 1
+
+
+def test_general_shape_backward_argument_checks(lib):
+    i32 = ctypes.c_int
+    f = lib.fa_bwd_qk
+    f.restype = i32
+    need = lib.fa_bwd_workspace_bytes(1, 1, 100, 64)
+
+    def call(Nq=100, Nk=300, d=64, scale=0.125, ws=FAKE, nbytes=need, dq=FAKE, dtype=0):
+        return f(dtype, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, dq, FAKE, FAKE, 1, 1, Nq, Nk, d,
+                 ctypes.c_float(scale), 1, ws, ctypes.c_size_t(nbytes), None)
+    assert call(dq=FAKE + 4) == 1
+    assert call(Nq=0) == 1 and call(Nk=0) == 1
+    assert call(d=96) == 2 and call(scale=-1.0) == 2 and call(scale=0.0) == 2
+    assert call(nbytes=need - 1) == 5 and call(ws=None) == 5
+    assert call(dtype=7) == 1

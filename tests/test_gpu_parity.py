@@ -240,20 +240,88 @@ def test_config_block_sparse(fa, oracle_mod):
 @pytest.mark.parametrize("N", [512, 1024, 2048, 4096, 8192, 16384])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
-def test_config_seqlen_sweep_forward_rows(fa, oracle_mod, N, d, causal):
-    # 16k tokens, hidden 2048: B = 16384 / N, H = 2048 / d. Forward checked on sampled rows of
-    # sampled heads (the oracle computes those rows one by one).
+def test_config_seqlen_sweep_forward_and_backward(fa, oracle_mod, N, d, causal):
+    # 16k tokens, hidden 2048: B = 16384 / N, H = 2048 / d, one launch of each kernel over the
+    # whole batch as the benchmark runs it. One sampled head is compared with the oracle in
+    # full: O and LSE, and dQ, dK, dV of the recomputation backward ([P3] §4.2: the same
+    # gradients as the standard backward).
     B, Hh = 16384 // N, 2048 // d
-    gpu, ref = H.make_case(B, Hh, N, d, seed=synth.BASE_SEED + 7, with_do=False)
+    gpu, ref = H.make_case(B, Hh, N, d, seed=synth.BASE_SEED + 7)
     scale = 1.0 / np.sqrt(d)
     o, lse = run_fwd(fa, gpu, causal, None, scale)
-    o64, l64 = H.to_f64(o), H.to_f64(lse)
-    rng = np.random.default_rng(N + d + causal)
-    for (b, h) in sampled_heads(B, Hh, 2, N + d):
-        rows = np.unique(np.concatenate([[0, 127, 128, N - 1], rng.choice(N, 60, replace=False)]))
-        o_ref, l_ref = oracle_mod.attention_fwd_rows(ref["q"][b, h], ref["k"][b, h], ref["v"][b, h], rows, scale,
-                                                     causal=causal)
-        H.assert_fwd_close(o64[b, h, rows], l64[b, h, rows], o_ref, l_ref, f"N={N} d={d} head {b},{h}")
+    dq, dk, dv = run_bwd(fa, gpu, o, lse, causal, None, scale)
+    for (b, h) in sampled_heads(B, Hh, 1, N + d + causal):
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        outs = [H.to_f64(x[sl]) for x in (o, lse, dq, dk, dv)]
+        args = [ref[k][sl] for k in ("q", "k", "v")]
+        o_ref, l_ref = oracle_mod.attention_fwd(*args, scale, causal=causal)
+        H.assert_fwd_close(outs[0], outs[1], o_ref, l_ref, f"N={N} d={d} causal={causal} head {b},{h}")
+        g_ref = oracle_mod.attention_bwd(*args, ref["do"][sl], scale, causal=causal)[:3]
+        H.assert_grads_close(outs[2:], g_ref, f"N={N} d={d} causal={causal} head {b},{h}")
+
+
+GENERAL_BWD = [
+    # B, H, Nq, Nk, d, causal, dtype: the backward of N_q queries against N_k keys
+    (1, 2, 128, 512, 64, False, "bf16"),
+    (1, 2, 200, 700, 128, True, "bf16"),     # ragged, bottom-right causal: rows see different key counts
+    (2, 1, 300, 200, 64, True, "bf16"),      # more queries than keys: 100 rows see nothing
+    (1, 1, 1, 1000, 128, True, "bf16"),      # one query (a decode step's gradient)
+    (1, 2, 640, 256, 128, False, "bf16"),
+    (1, 2, 384, 1000, 64, True, "f16"),
+    (1, 1, 512, 512, 128, True, "bf16"),     # N_q = N_k through the general entry point
+]
+
+
+@pytest.mark.parametrize("B,Hh,Nq,Nk,d,causal,dtype", GENERAL_BWD)
+def test_general_shape_backward(fa, oracle_mod, B, Hh, Nq, Nk, d, causal, dtype):
+    seed = synth.BASE_SEED + 13 * Nq + Nk
+    gq, rq = H.make_case(B, Hh, Nq, d, seed=seed, dtype=dtype)
+    gk, rk = H.make_case(B, Hh, Nk, d, seed=seed + 500, with_do=False, dtype=dtype)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = fa.forward_decode(gq["q"], gk["k"], gk["v"], causal=causal, scale=scale)
+    dq, dk, dv = fa.backward_qk(gq["q"], gk["k"], gk["v"], o, gq["do"], lse, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.last_device_status() == 0
+    assert dq.shape == gq["q"].shape and dk.shape == dv.shape == gk["k"].shape
+    o_ref, l_ref = oracle_mod.attention_fwd_qk(rq["q"], rk["k"], rk["v"], scale, causal=causal)
+    H.assert_fwd_close(H.to_f64(o), H.to_f64(lse), o_ref, l_ref, f"general fwd {B,Hh,Nq,Nk,d,causal}")
+    g_ref = oracle_mod.attention_bwd_qk(rq["q"], rk["k"], rk["v"], rq["do"], scale, causal=causal)[:3]
+    H.assert_grads_close([H.to_f64(x) for x in (dq, dk, dv)], g_ref, f"general bwd {B,Hh,Nq,Nk,d,causal}")
+    if causal and Nq > Nk:  # rows that see no key: dQ exactly zero
+        assert torch.all(dq[:, :, :Nq - Nk] == 0)
+
+
+def test_general_shape_backward_equals_square_backward(fa):
+    # N_q = N_k: the general entry point runs the same kernels as fa_bwd, so dK and dV are
+    # bit-identical; dQ differs at most by the order in which key tiles' shares were added.
+    gpu, _ = H.make_case(1, 2, 640, 128, seed=synth.BASE_SEED + 78)
+    for causal in (False, True):
+        o, lse = run_fwd(fa, gpu, causal, None, 0.0884)
+        dq1, dk1, dv1 = run_bwd(fa, gpu, o, lse, causal, None, 0.0884)
+        dq2, dk2, dv2 = fa.backward_qk(gpu["q"], gpu["k"], gpu["v"], o, gpu["do"], lse, causal=causal, scale=0.0884)
+        torch.cuda.synchronize()
+        assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+        assert (dq1.float() - dq2.float()).abs().max().item() < 2e-3
+
+
+def test_misaligned_dq_leaves_outputs_untouched(fa):
+    # Every argument of every backward stage is checked before the first launch: a bad dq
+    # (used only by the last stage) must not let the first two stages write dK and dV.
+    import ctypes
+    gpu, _ = H.make_case(1, 1, 256, 64, seed=synth.BASE_SEED + 79)
+    o, lse = run_fwd(fa, gpu, False, None, 0.125)
+    dk = torch.full_like(gpu["q"], 3.0)
+    dv = torch.full_like(gpu["q"], -2.0)
+    dq_buf = torch.zeros(gpu["q"].numel() + 8, dtype=gpu["q"].dtype, device="cuda")
+    ws = torch.empty(fa.bwd_workspace_bytes(1, 1, 256, 64), dtype=torch.uint8, device="cuda")
+    lib = fa.library()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    st = lib.fa_bwd(gpu["q"].data_ptr(), gpu["k"].data_ptr(), gpu["v"].data_ptr(), o.data_ptr(), gpu["do"].data_ptr(),
+                    lse.data_ptr(), dq_buf.data_ptr() + 2, dk.data_ptr(), dv.data_ptr(), 1, 1, 256, 64, 0.125, 0,
+                    None, ws.data_ptr(), ws.numel(), stream)
+    torch.cuda.synchronize()
+    assert st == 1
+    assert torch.all(dk == 3.0) and torch.all(dv == -2.0)
 
 
 def test_masked_blocks_do_not_influence_output(fa):
@@ -348,14 +416,16 @@ def test_bench_workload_backward_full_size(fa, oracle_mod):
     assert ((dv_sum - do_sum).norm(dim=-1) / do_sum.norm(dim=-1)).max().item() < 2e-2
 
 
-def test_largest_head_count(fa, oracle_mod):
-    # B*H = 65535 (the grid's y limit) with one 128-row tile per head, forward and backward.
-    # Heads are independent: the bulk is seeded device-side random data, and five heads across
-    # the range carry synth's draws, which the oracle gets bit for bit.
-    B, N, d, scale = 65535, 128, 64, 0.125
+@pytest.mark.parametrize("B", [65535, 70001])
+def test_largest_head_count(fa, oracle_mod, B):
+    # B*H = 65535 (one grid dimension's limit) and 70001 (heads spread over two grid
+    # dimensions, the last row of CTAs partly past the last head), one 128-row tile per head,
+    # forward and backward. Heads are independent: the bulk is seeded device-side random data,
+    # and five heads across the range carry synth's draws, which the oracle gets bit for bit.
+    N, d, scale = 128, 64, 0.125
     g = torch.Generator(device="cuda").manual_seed(synth.BASE_SEED)
     gpu = {k: torch.randn(B, 1, N, d, device="cuda", dtype=torch.bfloat16, generator=g) for k in ("q", "k", "v", "do")}
-    sample = (0, 1, 32767, 65533, 65534)
+    sample = (0, 1, 32767, 65534, B - 1) if B > 65535 else (0, 1, 32767, 65533, 65534)
     small, ref = H.make_case(len(sample), 1, N, d, seed=synth.BASE_SEED + 9)
     for x, b in enumerate(sample):
         for k in gpu:
