@@ -314,6 +314,103 @@ def _stream(seed: int, n: int, dtype: str = "bf16"):
     return synth.normal_bits(seed, n, dtype)
 
 
+SWEEP_POINTS = [(n, dd, c) for dd in (64, 128) for c in (False, True) for n in (512, 1024, 2048, 4096, 8192, 16384)]
+# The other configurations the metric is quoted on (block-sparse: diagonal on, others Bernoulli(0.25)).
+NAMED_CONFIGS = {
+    "bert_large_shape": dict(B=16, H=16, N=512, d=64, causal=False, block_sparse=False),
+    "gpt2_shape_causal": dict(B=8, H=12, N=1024, d=64, causal=True, block_sparse=False),
+    "block_sparse": dict(B=4, H=16, N=4096, d=64, causal=False, block_sparse=True),
+}
+
+
+def time_kernels(fa, t, shape, causal, mask, scale, steps, warmup):
+    """Per-kernel CUDA-event times (ms, mean over `steps`) of one fwd+bwd step on the views in
+    `t` (q, k, v, do, o, dq, dk, dv of `shape`; lse; ws), after `warmup` untimed steps, and the
+    whole-loop time per step."""
+    import torch
+    q, k, v, do, o, dq, dk, dv = (t[x] for x in ("q", "k", "v", "do", "o", "dq", "dk", "dv"))
+    lse, ws = t["lse"], t["ws"]
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record()
+        fa.forward(q, k, v, causal=causal, block_mask=mask, scale=scale, out=o, lse=lse)
+        if evs is not None:
+            evs[1].record()
+        fa.bwd_preprocess(o, do, lse, scale=scale, workspace=ws)
+        if evs is not None:
+            evs[2].record()
+        fa.bwd_main(q, k, v, do, ws, causal=causal, block_mask=mask, scale=scale, dk=dk, dv=dv)
+        if evs is not None:
+            evs[3].record()
+        fa.bwd_dq_finish(ws, shape, q.device, dq=dq)
+        if evs is not None:
+            evs[4].record()
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for e in evs:
+        step(e)
+    end.record()
+    torch.cuda.synchronize()
+    k_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(4)]
+    return k_ms, start.elapsed_time(end) / steps
+
+
+def run_sweep(fa, dev, dtype, steps, warmup, peaks):
+    """The metric's curve: every sequence-length sweep point (16k tokens, hidden 2048; N x d x
+    causal) and the named configurations, each timed on its own with CUDA events. All sweep
+    points have 16384 x 2048 elements per tensor, so one set of device buffers serves them all
+    (viewed as [B, H, N, d]); the named configurations use prefixes of the same buffers."""
+    import torch
+    import synth
+    n = TOKENS * HIDDEN
+    base = {x: synth.to_torch(_stream(synth.BASE_SEED + off, n, dtype), dtype, dev)
+            for x, off in (("q", synth.SEED_Q), ("k", synth.SEED_K), ("v", synth.SEED_V), ("do", synth.SEED_DO))}
+    for x in ("o", "dq", "dk", "dv"):
+        base[x] = torch.empty_like(base["q"])
+    lse_all = torch.empty(n // 64, dtype=torch.float32, device=dev)
+    ws_all = torch.empty(max(fa.bwd_workspace_bytes(TOKENS // N, HIDDEN // dd, N, dd) for N, dd, _ in SWEEP_POINTS),
+                         dtype=torch.uint8, device=dev)
+
+    def views(B, H, N, d):
+        m = B * H * N * d
+        t = {x: base[x][:m].view(B, H, N, d) for x in ("q", "k", "v", "do", "o", "dq", "dk", "dv")}
+        t["lse"] = lse_all[:B * H * N].view(B, H, N)
+        t["ws"] = ws_all
+        return t
+
+    def entry(B, H, N, d, causal, mask_np):
+        mask = None if mask_np is None else torch.from_numpy(mask_np).to(dev)
+        density = float(mask_np.mean()) if mask_np is not None else 1.0
+        (f_ms, p_ms, m_ms, d_ms), step_ms = time_kernels(fa, views(B, H, N, d), (B, H, N, d), causal, mask,
+                                                          1.0 / math.sqrt(d), steps, warmup)
+        ff = fwd_flops(B, H, N, d, causal, density)
+        fwd_t = ff / (f_ms * 1e-3) / 1e12
+        fb_t = 3.5 * ff / (step_ms * 1e-3) / 1e12
+        return {"B": B, "H": H, "N": N, "d": d, "causal": causal, "block_density": round(density, 4),
+                "fwd_ms": round(f_ms, 4), "bwd_ms": round(p_ms + m_ms + d_ms, 4), "step_ms": round(step_ms, 4),
+                "fwd_tflops": round(fwd_t, 1), "fwd_bwd_tflops": round(fb_t, 1),
+                "bwd_main_tflops": round(2.5 * ff / (m_ms * 1e-3) / 1e12, 1),
+                "pct_of_peak_fwd": round(100 * fwd_t / peaks["bf16_tflops"], 2),
+                "pct_of_peak_fwd_bwd": round(100 * fb_t / peaks["bf16_tflops"], 2)}
+
+    points = []
+    for (N, d, c) in SWEEP_POINTS:
+        points.append(entry(TOKENS // N, HIDDEN // d, N, d, c, None))
+    named = {}
+    for name, c in NAMED_CONFIGS.items():
+        mask_np = synth.block_mask_for(c["N"]) if c["block_sparse"] else None
+        named[name] = entry(c["B"], c["H"], c["N"], c["d"], c["causal"], mask_np)
+    if fa.last_device_status(dev) != 0:
+        raise RuntimeError("device wait timed out in the sweep")
+    return points, named
+
+
 def run_gpu(args, wl, rank, world, local_rank, dist_on):
     import numpy as np
     import torch
@@ -456,6 +553,16 @@ def run_gpu(args, wl, rank, world, local_rank, dist_on):
         "gpu_launches": 4 * args.steps,
         "clocks": clk.summary(),
     }
+    if not args.no_sweep:
+        with ClockSampler(physical_gpu(local_rank)) as sclk:
+            time.sleep(0.3)
+            points, named = run_sweep(fa, dev, args.dtype, args.sweep_steps, args.warmup, peaks)
+        line["sweep"] = {"unit": UNIT, "peak": peaks["bf16_tflops"],
+                         "peak_kind": f"bf16 dense burst ({peaks['source']})",
+                         "steps": args.sweep_steps, "warmup": args.warmup, "dtype": args.dtype,
+                         "workload": "16k tokens, hidden 2048: B = 16384/N, H = 2048/d, bf16 N(0,1); "
+                                     "per-GPU figures on this rank",
+                         "points": points, "configs": named, "clocks": sclk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         nh = heads_for_seconds(wl, 12.0)
         f, t, cores = oracle_sample(wl, nh, 3000, args.dtype)
@@ -479,6 +586,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the sequence-length curve (24 points + named configs) in the headline line")
+    ap.add_argument("--sweep-steps", type=int, default=5, help="timed steps per point of that curve")
     ap.add_argument("--sweep", action="store_true", help="one JSON line per sweep point (N x d x causal)")
     ap.add_argument("--block-density", type=float, default=0.25,
                     help="with --block-sparse: probability that an off-diagonal 128x128 block is on")
@@ -515,7 +625,7 @@ def main(argv=None):
             return run_forward_only(args, workload(args.seqlen, args.headdim, args.causal, False),
                                     rank, world, local_rank, dist_on)
         if args.density_sweep:
-            args.no_cpu_baseline, args.no_e2e = True, True
+            args.no_cpu_baseline, args.no_e2e, args.no_sweep = True, True, True
             for p_on in (0.05, 0.1, 0.25, 0.5, 1.0):
                 run_gpu(args, workload(args.seqlen, args.headdim, False, True, p_on), rank, world, local_rank, dist_on)
             return 0
@@ -524,7 +634,7 @@ def main(argv=None):
         for (n, dd, c) in points:
             wl = workload(n, dd, c, args.block_sparse, args.block_density)
             if args.sweep:
-                args.no_cpu_baseline, args.no_e2e = True, True
+                args.no_cpu_baseline, args.no_e2e, args.no_sweep = True, True, True
             run_gpu(args, wl, rank, world, local_rank, dist_on)
     finally:
         if dist_on:

@@ -43,6 +43,17 @@ def test_step_line_with_e2e():
     assert e2e["d2h_bytes_per_step"] == 4 * B * H * N * d * 2 + B * H * N * 4  # o, dq, dk, dv, lse
     assert 0 < e2e["value"] < line["value"]  # the host copies make the end-to-end step slower
     assert set(line["kernels"]) == {"fwd", "bwd_preprocess", "bwd_main", "bwd_dq_finish"}
+    # the metric's curve: every sweep point and the named configurations, each timed on its own
+    sw = line["sweep"]
+    pts = {(p["N"], p["d"], p["causal"]) for p in sw["points"]}
+    assert pts == {(n, d, c) for n in (512, 1024, 2048, 4096, 8192, 16384) for d in (64, 128) for c in (False, True)}
+    for p in sw["points"]:
+        assert p["B"] * p["N"] == 16384 and p["H"] * p["d"] == 2048
+        assert 0 < p["fwd_tflops"] and 0 < p["fwd_bwd_tflops"]
+        assert abs(p["pct_of_peak_fwd"] - 100 * p["fwd_tflops"] / sw["peak"]) < 0.1
+    assert set(sw["configs"]) == {"bert_large_shape", "gpt2_shape_causal", "block_sparse"}
+    assert 0.2 < sw["configs"]["block_sparse"]["block_density"] < 0.35
+    assert "sm_mhz" in sw["clocks"]
 
 
 @pytest.mark.gpu
