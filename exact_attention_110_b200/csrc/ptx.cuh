@@ -397,18 +397,25 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Coefficients of the cubic 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 on f in [-0.5, 0.5] used by the
+// FMA-pipe exp2 below: the fp32-rounded minimax fit of the relative error (Lawson's
+// iteratively reweighted least squares), exactly as printed by
+// `python -m exact_attention_110_b200.fit_ex2_poly`; max relative error 7.5e-5 in fp32 Horner
+// form, far below the bf16 rounding P receives.
+constexpr float kEx2C0 = 0.9999280571937561f;
+constexpr float kEx2C1 = 0.6932610273361206f;
+constexpr float kEx2C2 = 0.24261121451854706f;
+constexpr float kEx2C3 = 0.05517137795686722f;
+
 // 2^x evaluated on the FMA pipe, to take load off the special-function unit. x = n + f with
-// n = round(x) (added into the exponent field) and f in [-0.5, 0.5], 2^f by a cubic whose
-// coefficients were fitted for this library (iteratively reweighted least squares on the
-// relative error over [-0.5, 0.5]; max relative error 7.5e-5 in fp32 Horner form, far below
-// the bf16 rounding P receives). Inputs at or below -125 (including -inf) return exactly 0.
+// n = round(x) (added into the exponent field) and f in [-0.5, 0.5], 2^f by the cubic above.
+// Inputs at or below -125 (including -inf) return exactly 0.
 __device__ __forceinline__ float ex2_poly(float x) {
   const float xc = fmaxf(x, -125.f);
   const float t = __fadd_rn(xc, 12582912.f);  // 1.5 * 2^23: the integer part lands in the low bits
   const int n = __float_as_int(t) - 0x4B400000;
   const float f = __fsub_rn(xc, __fsub_rn(t, 12582912.f));
-  const float p = fmaf(fmaf(fmaf(0.05517132207751274f, f, 0.24261054396629333f), f, 0.6932609677314758f), f,
-                       0.9999281167984009f);
+  const float p = fmaf(fmaf(fmaf(kEx2C3, f, kEx2C2), f, kEx2C1), f, kEx2C0);
   const float r = __int_as_float(__float_as_int(p) + (n << 23));
   return x > -125.f ? r : 0.f;
 }
@@ -455,10 +462,10 @@ __device__ __forceinline__ Ex2PolyConsts ex2_poly_consts() {
   k.magic = f2_pack(12582912.f, 12582912.f);
   k.neg_magic = f2_pack(-12582912.f, -12582912.f);
   k.neg_one = f2_pack(-1.f, -1.f);
-  k.c0 = f2_pack(0.9999281167984009f, 0.9999281167984009f);
-  k.c1 = f2_pack(0.6932609677314758f, 0.6932609677314758f);
-  k.c2 = f2_pack(0.24261054396629333f, 0.24261054396629333f);
-  k.c3 = f2_pack(0.05517132207751274f, 0.05517132207751274f);
+  k.c0 = f2_pack(kEx2C0, kEx2C0);
+  k.c1 = f2_pack(kEx2C1, kEx2C1);
+  k.c2 = f2_pack(kEx2C2, kEx2C2);
+  k.c3 = f2_pack(kEx2C3, kEx2C3);
   return k;
 }
 __device__ __forceinline__ uint64_t ex2_poly2(uint64_t x2, const Ex2PolyConsts& k) {
