@@ -258,9 +258,8 @@ def run_decode(args, rank, world, local_rank, dist_on):
 
 
 def run_forward_only(args, wl, rank, world, local_rank, dist_on):
-    """Forward pass alone on the sweep's workload (the one line for head dimension 256, which
-    has a forward but no backward). Metric: forward TFLOPS (4·N²·d per head, halved when
-    causal) against the measured dense bf16 peak."""
+    """Forward pass alone on the sweep's workload. Metric: forward TFLOPS (4·N²·d per head,
+    halved when causal) against the measured dense bf16 peak."""
     import torch
     import exact_attention_110_b200 as fa
     import synth
@@ -320,6 +319,9 @@ NAMED_CONFIGS = {
     "bert_large_shape": dict(B=16, H=16, N=512, d=64, causal=False, block_sparse=False),
     "gpt2_shape_causal": dict(B=8, H=12, N=1024, d=64, causal=True, block_sparse=False),
     "block_sparse": dict(B=4, H=16, N=4096, d=64, causal=False, block_sparse=True),
+    # the same 16k tokens x hidden 2048 at head dimension 256
+    "head_dim_256": dict(B=4, H=8, N=4096, d=256, causal=False, block_sparse=False),
+    "head_dim_256_causal": dict(B=4, H=8, N=4096, d=256, causal=True, block_sparse=False),
 }
 
 
@@ -596,8 +598,7 @@ def main(argv=None):
                     help="block-sparse config at densities 0.05..1: runtime should follow the blocks that are on")
     ap.add_argument("--decode", type=int, default=0, metavar="NQ",
                     help="decode-shaped forward: NQ queries per head against --seqlen keys (B=8)")
-    ap.add_argument("--forward-only", action="store_true",
-                    help="time the forward alone (the only pass built at head dimension 256)")
+    ap.add_argument("--forward-only", action="store_true", help="time the forward alone")
     ap.add_argument("--dtype", choices=["bf16", "f16"], default="bf16",
                     help="element type of q, k, v, o, dO and the gradients (fp32 accumulation either way)")
     args = ap.parse_args(argv)

@@ -10,7 +10,7 @@ the library is missing, every call raises -- there is no fallback implementation
     o, lse = forward_decode(q, k, v, causal=False, scale=None, num_splits=0)   # Nq != Nk
     dq, dk, dv = backward_qk(q, k, v, o, do, lse, causal=False, scale=None)     # its gradients
 
-q, k, v, o, do: bf16 (or fp16) CUDA tensors [B, H, N, d] of one type, contiguous, d in {64, 128},
+q, k, v, o, do: bf16 (or fp16) CUDA tensors [B, H, N, d] of one type, contiguous, d in {64, 128, 256},
 any N >= 1.
 lse: fp32 [B, H, N]. block_mask: uint8 CUDA tensor [nb, nb] shared by every head, or one mask per
 head [B, H, nb, nb] (nb = ceil(N/128)), or None.

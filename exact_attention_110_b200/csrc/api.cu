@@ -64,11 +64,10 @@ bool mask_stride_ok(const uint8_t* mask, long long stride, int N) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Head dimensions: 64 and 128 everywhere; 256 in the forward only (its backward's dK and dV
-// accumulators alone would fill the 512 TMEM columns).
-fa_status check_common(int B, int H, int N, int d, float scale, bool allow_d256 = false) {
+// Head dimensions: 64, 128 and 256 in every pass.
+fa_status check_common(int B, int H, int N, int d, float scale) {
   if (B <= 0 || H <= 0 || N <= 0 || !isfinite(scale)) return FA_ERR_INVALID;
-  if (d != 64 && d != 128 && !(allow_d256 && d == 256)) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   const long long BH = (long long)B * H;
   if (BH > 0x7fffffffll) return FA_ERR_UNSUPPORTED;        // TMA head coordinate (int32)
   if ((long long)N * d > (1ll << 31) / 2) return FA_ERR_UNSUPPORTED;  // per-head elements
@@ -123,7 +122,7 @@ fa_status fa_fwd_ex(int dtype, const void* q, const void* k, const void* v, void
   const int f16 = dtype == FA_DTYPE_F16;
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID;
-  fa_status st = check_common(B, H, N, d, scale, true);
+  fa_status st = check_common(B, H, N, d, scale);
   if (st != FA_OK) return st;
   if (!(scale > 0.f)) return FA_ERR_UNSUPPORTED;  // see check_decode
   if (!get_encoder()) return FA_ERR_CUDA;

@@ -59,20 +59,29 @@ namespace fa {
 template <int D>
 struct BwdCfg {
   static constexpr int THREADS = 512;
-  static constexpr int NS = (D == 128) ? 2 : 3;     // Q ring depth (with -LSE*log2e and -D)
+  // d = 256: two CTAs per key tile, CTA `hh` owning the 128-column half hh of d for dK, dV
+  // and its dQ share (S^T and dP^T still contract over all 256 columns). Its accumulators then
+  // fill TMEM exactly as at d = 128. K_j stays in shared memory; Q_i, dO_i and V_j stream as
+  // 64-column panels through one FIFO ring (see the producer), since the four full 64 KB tiles
+  // the two contractions read would not fit.
+  static constexpr bool SPLIT = (D == 256);
+  static constexpr int DH = SPLIT ? 128 : D;       // accumulator width per CTA (dK, dV, dQ share)
+  static constexpr int NS = (D == 64) ? 3 : 2;     // Q ring depth (with -LSE*log2e and -D); SPLIT: vector ring
   // d = 128: dO is single-buffered to make room for the dQ staging buffer. dO_i is last read by
   // dV_i and next needed by dP_{i+1}, three MMA groups later, which covers the load.
-  static constexpr int NS_DO = (D == 128) ? 1 : NS;
-  static constexpr int DQ_CHUNKS = D / 32;         // 32-column dQ chunks per query tile
+  static constexpr int NS_DO = (D == 128) ? 1 : (SPLIT ? 0 : NS);
+  static constexpr int RING = SPLIT ? 6 : 0;       // SPLIT: 64-column panel slots
+  static constexpr int DQ_CHUNKS = DH / 32;        // 32-column dQ chunks per query tile
   static constexpr int DQ_SLOTS = 2;                // staging slots: one filling, one being reduced
   static constexpr int DQ_SLOT_BYTES = 128 * 32 * 4;
   static constexpr int PANEL_BYTES = 128 * 128;
-  static constexpr int PANELS = D / 64;
+  static constexpr int PANELS = D / 64;            // panels of a whole 128 x D tile
+  static constexpr int PANELS_H = DH / 64;         // panels of this CTA's dK / dV columns
   static constexpr int TILE_BYTES = PANELS * PANEL_BYTES;
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + TILE_BYTES;
-  static constexpr int OFF_Q = OFF_V + TILE_BYTES;
-  static constexpr int OFF_DO = OFF_Q + NS * TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + TILE_BYTES;                              // not SPLIT
+  static constexpr int OFF_Q = SPLIT ? OFF_K + TILE_BYTES : OFF_V + TILE_BYTES;  // SPLIT: the panel ring
+  static constexpr int OFF_DO = SPLIT ? OFF_Q + RING * PANEL_BYTES : OFF_Q + NS * TILE_BYTES;
   static constexpr int OFF_DS = OFF_DO + NS_DO * TILE_BYTES;  // 128 keys x 128 queries bf16
   static constexpr int DS_BYTES = 2 * PANEL_BYTES;
   static constexpr int OFF_DQS = OFF_DS + DS_BYTES;           // dQ staging [DQ_SLOTS][128][32] fp32
@@ -80,18 +89,23 @@ struct BwdCfg {
   static constexpr int OFF_LSE = OFF_DQS + DQS_BYTES;         // [NS][128] fp32: -LSE*log2e
   static constexpr int OFF_DEL = OFF_LSE + NS * 512;          // [NS][128] fp32: -D
   static constexpr int OFF_BAR = OFF_DEL + NS * 512;
-  static constexpr int NBAR = 1 + 2 * NS + 2 * NS_DO + 9;
+  static constexpr int NQB = SPLIT ? RING : NS;               // full/empty barrier pairs of the Q ring
+  static constexpr int NBAR = 1 + 2 * NQB + 2 * NS_DO + 9;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int TMEM_COLS = 512;
-  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
-  static constexpr bool DQ_ALIAS = (D == 128);           // dQ reuses the dP^T columns
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + DH;
+  static constexpr bool DQ_ALIAS = (DH == 128);          // dQ reuses the dP^T columns
   static constexpr uint32_t T_DQ = DQ_ALIAS ? T_DP : 384u;
   // setmaxnreg split of the launch allocation (512 x 128, checked by the build script):
   // control warpgroup (TMA, MMA, 2 idle warps), two P/dS warpgroups, dQ-drain warpgroup.
   static constexpr int REGS_CTRL = FA_BWD_REGS_CTRL, REGS_PDS = FA_BWD_REGS_PDS, REGS_DQ = FA_BWD_REGS_DQ;
   static_assert(128 * (REGS_CTRL + 2 * REGS_PDS + REGS_DQ) <= 512 * 128, "setmaxnreg split exceeds the launch");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  // SPLIT: the vectors of query tile i+2 land in tile i's vector slot together with Q_{i+2}'s
+  // first panel, which sits 12 panels after Q_i's first dK panel in the ring order; with at
+  // most 12 slots that load cannot start before dK_i, i.e. before tile i's dS phase is done.
+  static_assert(RING <= 12, "vector slot reuse needs a ring of at most 12 panels");
 };
 
 // bmask: this (b, h)'s block mask (or null), [query tiles][key tiles]. Causal: key tile j is
@@ -134,7 +148,7 @@ __global__ void __launch_bounds__(512, 1)
                   const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                   const __grid_constant__ CUtensorMap tmdQa, const BwdParams p) {
   using C = BwdCfg<D>;
-  constexpr int NS = C::NS, NS_DO = C::NS_DO;
+  constexpr int NS = C::NS, NS_DO = C::NS_DO, NQB = C::NQB;
   extern __shared__ __align__(1024) uint8_t smem[];
 
   const uint32_t warp = warp_id(), lane = lane_id();
@@ -145,9 +159,9 @@ __global__ void __launch_bounds__(512, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* bar_kv = bars;               // K_j, V_j landed
-  uint64_t* bar_qf = bars + 1;           // [NS] Q_i, -LSE2_i, -D_i landed
-  uint64_t* bar_qe = bar_qf + NS;        // [NS] Q stage free (after dK_i)
-  uint64_t* bar_dof = bar_qe + NS;       // [NS_DO] dO_i landed
+  uint64_t* bar_qf = bars + 1;           // [NQB] Q_i, -LSE2_i, -D_i landed (SPLIT: ring slot full)
+  uint64_t* bar_qe = bar_qf + NQB;       // [NQB] Q stage free after dK_i (SPLIT: ring slot free)
+  uint64_t* bar_dof = bar_qe + NQB;      // [NS_DO] dO_i landed
   uint64_t* bar_doe = bar_dof + NS_DO;   // [NS_DO] dO stage free (after dV_i)
   uint64_t* bar_s = bar_doe + NS_DO;     // S^T_i ready in TMEM
   uint64_t* bar_dp = bar_s + 1;          // dP^T_i ready in TMEM
@@ -165,7 +179,9 @@ __global__ void __launch_bounds__(512, 1)
   if (bh_l >= p.BH) return;  // past the last head (head counts above 65535 round the grid up)
   const int bh = (int)bh_l;
   const uint8_t* bmask = p.block_mask == nullptr ? nullptr : p.block_mask + (size_t)bh * p.mask_stride;
-  const int j = blockIdx.x;  // key tile (causal: j = 0 has the most work and starts first)
+  // key tile (causal: j = 0 has the most work and starts first); SPLIT: and the half of d
+  const int j = C::SPLIT ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int hh = C::SPLIT ? (int)(blockIdx.x & 1) : 0;
   // causal: the first query tile whose last row sees key tile j's first key
   const int i_first = 128 * j - 127 - p.causal_off;
   const int i_begin = (p.causal && i_first > 0) ? (i_first + 127) / 128 : 0;
@@ -173,7 +189,7 @@ __global__ void __launch_bounds__(512, 1)
 
   if (warp == 0 && lane == 0) {
     mbar_init(bar_kv, 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NQB; ++s) {
       mbar_init(&bar_qf[s], 1);
       mbar_init(&bar_qe[s], 1);
     }
@@ -213,57 +229,118 @@ __global__ void __launch_bounds__(512, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmdO);
-      mbar_arrive_expect_tx(bar_kv, 2 * C::TILE_BYTES);
-      for (int pn = 0; pn < C::PANELS; ++pn) {
-        tma_load_3d(smem + C::OFF_K + pn * C::PANEL_BYTES, &tmK, bar_kv, pn * 64, j * 128, bh);
-        tma_load_3d(smem + C::OFF_V + pn * C::PANEL_BYTES, &tmV, bar_kv, pn * 64, j * 128, bh);
-      }
-      int it = 0;
-      int issued[NS], issued_do[NS_DO];
-      for (int s = 0; s < NS; ++s) issued[s] = -1;
-      for (int s = 0; s < NS_DO; ++s) issued_do[s] = -1;
-      bool ok = true;
-      for (int i = i_begin; i < p.nb; ++i) {
-        if (!bwd_tile_active(p, bmask, i, j)) continue;
-        // Q_i first: its stage frees at dK_{i-NS}, before dO_i's stage frees at dV_{i-NS_DO}.
-        const int s = it % NS;
-        const uint32_t ph = (it / NS) & 1;
-        ok = mbar_wait(&bar_qe[s], ph ^ 1, ab, lim, WAIT_BWD_LOAD + 1);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&bar_qf[s], C::TILE_BYTES + 1024);
+      if constexpr (!C::SPLIT) {
+        mbar_arrive_expect_tx(bar_kv, 2 * C::TILE_BYTES);
+        for (int pn = 0; pn < C::PANELS; ++pn) {
+          tma_load_3d(smem + C::OFF_K + pn * C::PANEL_BYTES, &tmK, bar_kv, pn * 64, j * 128, bh);
+          tma_load_3d(smem + C::OFF_V + pn * C::PANEL_BYTES, &tmV, bar_kv, pn * 64, j * 128, bh);
+        }
+        int it = 0;
+        int issued[NS], issued_do[NS_DO];
+        for (int s = 0; s < NS; ++s) issued[s] = -1;
+        for (int s = 0; s < NS_DO; ++s) issued_do[s] = -1;
+        bool ok = true;
+        for (int i = i_begin; i < p.nb; ++i) {
+          if (!bwd_tile_active(p, bmask, i, j)) continue;
+          // Q_i first: its stage frees at dK_{i-NS}, before dO_i's stage frees at dV_{i-NS_DO}.
+          const int s = it % NS;
+          const uint32_t ph = (it / NS) & 1;
+          ok = mbar_wait(&bar_qe[s], ph ^ 1, ab, lim, WAIT_BWD_LOAD + 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bar_qf[s], C::TILE_BYTES + 1024);
+          for (int pn = 0; pn < C::PANELS; ++pn)
+            tma_load_3d(smem + C::OFF_Q + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &bar_qf[s], pn * 64, i * 128,
+                        bh);
+          const size_t vec = (size_t)bh * p.Np + (size_t)i * 128;
+          bulk_load(smem + C::OFF_LSE + s * 512, p.lse2 + vec, 512, &bar_qf[s]);
+          bulk_load(smem + C::OFF_DEL + s * 512, p.delta + vec, 512, &bar_qf[s]);
+          issued[s] = ph;
+          const int sd = it % NS_DO;
+          const uint32_t phd = (it / NS_DO) & 1;
+          ok = mbar_wait(&bar_doe[sd], phd ^ 1, ab, lim, WAIT_BWD_LOAD + 4);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bar_dof[sd], C::TILE_BYTES);
+          for (int pn = 0; pn < C::PANELS; ++pn)
+            tma_load_3d(smem + C::OFF_DO + sd * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmdO, &bar_dof[sd], pn * 64,
+                        i * 128, bh);
+          issued_do[sd] = phd;
+          ++it;
+        }
+        AbortState none{0};
+        if (!ok) {
+          for (int s = 0; s < NS; ++s)
+            if (issued[s] >= 0) mbar_wait(&bar_qf[s], issued[s], &none, lim, WAIT_BWD_LOAD + 2);
+          for (int s = 0; s < NS_DO; ++s)
+            if (issued_do[s] >= 0) mbar_wait(&bar_dof[s], issued_do[s], &none, lim, WAIT_BWD_LOAD + 5);
+        }
+      } else {
+        // K_j (all four panels) stays; everything else streams through the panel ring in the
+        // order the MMA issuer consumes it. First tile i0: Q(i0) panels 0-3 (S^T), then V and
+        // dO(i0) panels p = 0-3 in pairs (dP^T). Then per tile i (next active tile i'):
+        // dO(i) panels of half hh (dV), Q(i') panels 0-3 (S^T of i'), Q(i) panels of half hh
+        // (dK), V / dO(i') panel pairs (dP^T of i'). Q's first panel carries the tile's -LSE2
+        // and -D vectors into vector slot (active tile index) & 1.
+        mbar_arrive_expect_tx(bar_kv, C::TILE_BYTES);
         for (int pn = 0; pn < C::PANELS; ++pn)
-          tma_load_3d(smem + C::OFF_Q + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &bar_qf[s], pn * 64, i * 128,
-                      bh);
-        const size_t vec = (size_t)bh * p.Np + (size_t)i * 128;
-        bulk_load(smem + C::OFF_LSE + s * 512, p.lse2 + vec, 512, &bar_qf[s]);
-        bulk_load(smem + C::OFF_DEL + s * 512, p.delta + vec, 512, &bar_qf[s]);
-        issued[s] = ph;
-        const int sd = it % NS_DO;
-        const uint32_t phd = (it / NS_DO) & 1;
-        ok = mbar_wait(&bar_doe[sd], phd ^ 1, ab, lim, WAIT_BWD_LOAD + 4);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&bar_dof[sd], C::TILE_BYTES);
-        for (int pn = 0; pn < C::PANELS; ++pn)
-          tma_load_3d(smem + C::OFF_DO + sd * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmdO, &bar_dof[sd], pn * 64,
-                      i * 128, bh);
-        issued_do[sd] = phd;
-        ++it;
+          tma_load_3d(smem + C::OFF_K + pn * C::PANEL_BYTES, &tmK, bar_kv, pn * 64, j * 128, bh);
+        int issued[C::RING];
+        for (int s = 0; s < C::RING; ++s) issued[s] = -1;
+        int npush = 0, vit = 0;
+        bool ok = true;
+        auto push = [&](const CUtensorMap* map, int x, int y, int vec_tile) -> bool {
+          const int s = npush % C::RING;
+          const uint32_t ph = (uint32_t)(npush / C::RING) & 1u;
+          if (!mbar_wait(&bar_qe[s], ph ^ 1u, ab, lim, WAIT_BWD_LOAD + 1)) return false;
+          mbar_arrive_expect_tx(&bar_qf[s], C::PANEL_BYTES + (vec_tile >= 0 ? 1024 : 0));
+          tma_load_3d(smem + C::OFF_Q + s * C::PANEL_BYTES, map, &bar_qf[s], x, y, bh);
+          if (vec_tile >= 0) {
+            const int vs = vit & 1;
+            const size_t vec = (size_t)bh * p.Np + (size_t)vec_tile * 128;
+            bulk_load(smem + C::OFF_LSE + vs * 512, p.lse2 + vec, 512, &bar_qf[s]);
+            bulk_load(smem + C::OFF_DEL + vs * 512, p.delta + vec, 512, &bar_qf[s]);
+            ++vit;
+          }
+          issued[s] = (int)ph;
+          ++npush;
+          return true;
+        };
+        auto push_s = [&](int i) -> bool {  // Q(i) panels 0-3, vectors with the first
+          for (int pn = 0; pn < C::PANELS; ++pn)
+            if (!push(&tmQ, pn * 64, i * 128, pn == 0 ? i : -1)) return false;
+          return true;
+        };
+        auto push_dp = [&](int i) -> bool {  // V_j and dO(i) panel pairs
+          for (int pn = 0; pn < C::PANELS; ++pn)
+            if (!push(&tmV, pn * 64, j * 128, -1) || !push(&tmdO, pn * 64, i * 128, -1)) return false;
+          return true;
+        };
+        int i = i_begin;
+        while (i < p.nb && !bwd_tile_active(p, bmask, i, j)) ++i;
+        if (i < p.nb) ok = push_s(i) && push_dp(i);
+        while (ok && i < p.nb) {
+          int inext = i + 1;
+          while (inext < p.nb && !bwd_tile_active(p, bmask, inext, j)) ++inext;
+          const bool has_next = inext < p.nb;
+          ok = push(&tmdO, 128 * hh, i * 128, -1) && push(&tmdO, 128 * hh + 64, i * 128, -1);
+          if (ok && has_next) ok = push_s(inext);
+          if (ok) ok = push(&tmQ, 128 * hh, i * 128, -1) && push(&tmQ, 128 * hh + 64, i * 128, -1);
+          if (ok && has_next) ok = push_dp(inext);
+          i = inext;
+        }
+        AbortState none{0};
+        if (!ok)
+          for (int s = 0; s < C::RING; ++s)
+            if (issued[s] >= 0) mbar_wait(&bar_qf[s], issued[s], &none, lim, WAIT_BWD_LOAD + 2);
       }
       AbortState none{0};
-      if (!ok) {
-        for (int s = 0; s < NS; ++s)
-          if (issued[s] >= 0) mbar_wait(&bar_qf[s], issued[s], &none, lim, WAIT_BWD_LOAD + 2);
-        for (int s = 0; s < NS_DO; ++s)
-          if (issued_do[s] >= 0) mbar_wait(&bar_dof[s], issued_do[s], &none, lim, WAIT_BWD_LOAD + 5);
-      }
       mbar_wait(bar_kv, 0, &none, lim, WAIT_BWD_LOAD + 3);  // K/V landed before the CTA can exit
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_f32acc(128, 128, 0, 0, F16);  // K/V (A) and Q/dO (B), K-major
-      constexpr uint32_t IDESC_KV = idesc_f32acc(128, D, 0, 1, F16);   // dV, dK: B = dO / Q MN-major
-      constexpr uint32_t IDESC_Q = idesc_f32acc(128, D, 1, 1, F16);    // dQ = dS K: A = dS^T, B = K, MN-major
+      constexpr uint32_t IDESC_KV = idesc_f32acc(128, C::DH, 0, 1, F16);  // dV, dK: B = dO / Q MN-major
+      constexpr uint32_t IDESC_Q = idesc_f32acc(128, C::DH, 1, 1, F16);   // dQ = dS K: A = dS^T, B = K, MN-major
       constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
       const uint32_t tS = tmem + C::T_S, tDP = tmem + C::T_DP, tDV = tmem + C::T_DV, tDK = tmem + C::T_DK;
       const uint32_t tDQ = tmem + C::T_DQ;
@@ -278,103 +355,209 @@ __global__ void __launch_bounds__(512, 1)
       const uint64_t dS_mn = sdesc_sw128(sDS, C::PANEL_BYTES, 1024); // dS^T read MN-major (dQ)
       bool ok = mbar_wait_spin(bar_kv, 0, ab, lim, WAIT_BWD_MMA + 1);
 
-      auto issue_s = [&](int st) {
-        const uint64_t b = dQ_k + (uint64_t)(st * TILE16);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
-          umma_ss(tS, dK_k + off16, b + off16, IDESC_S, kk > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_dp = [&](int st) {
-        const uint64_t b = dO_k + (uint64_t)(st * TILE16);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
-          umma_ss(tDP, dV_k + off16, b + off16, IDESC_S, kk > 0 ? 1u : 0u);
-        }
-      };
+      if constexpr (!C::SPLIT) {
+        auto issue_s = [&](int st) {
+          const uint64_t b = dQ_k + (uint64_t)(st * TILE16);
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
+            umma_ss(tS, dK_k + off16, b + off16, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+        };
+        auto issue_dp = [&](int st) {
+          const uint64_t b = dO_k + (uint64_t)(st * TILE16);
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
+            umma_ss(tDP, dV_k + off16, b + off16, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+        };
 
-      int i = i_begin;
-      while (i < p.nb && !bwd_tile_active(p, bmask, i, j)) ++i;
-      int it = 0;
-      if (ok && i < p.nb) {
-        ok = mbar_wait_spin(&bar_qf[0], 0, ab, lim, WAIT_BWD_MMA + 2);
-        if (ok) {
-          tc_fence_after();
-          issue_s(0);
-          umma_commit(bar_s);
-          ok = mbar_wait_spin(&bar_dof[0], 0, ab, lim, WAIT_BWD_MMA + 9);
+        int i = i_begin;
+        while (i < p.nb && !bwd_tile_active(p, bmask, i, j)) ++i;
+        int it = 0;
+        if (ok && i < p.nb) {
+          ok = mbar_wait_spin(&bar_qf[0], 0, ab, lim, WAIT_BWD_MMA + 2);
+          if (ok) {
+            tc_fence_after();
+            issue_s(0);
+            umma_commit(bar_s);
+            ok = mbar_wait_spin(&bar_dof[0], 0, ab, lim, WAIT_BWD_MMA + 9);
+          }
+          if (ok) {
+            tc_fence_after();
+            issue_dp(0);
+            umma_commit(bar_dp);
+          }
         }
-        if (ok) {
-          tc_fence_after();
-          issue_dp(0);
-          umma_commit(bar_dp);
-        }
-      }
-      while (ok && i < p.nb) {
-        const int s = it % NS;
-        int inext = i + 1;
-        while (inext < p.nb && !bwd_tile_active(p, bmask, inext, j)) ++inext;
-        const bool has_next = inext < p.nb;
-        const int sn = (it + 1) % NS;
-        const int sd = it % NS_DO, sdn = (it + 1) % NS_DO;
-        const uint32_t acc = it > 0 ? 1u : 0u;
-        const uint64_t dOs = dO_mn + (uint64_t)(sd * TILE16), dQs = dQ_mn + (uint64_t)(s * TILE16);
+        while (ok && i < p.nb) {
+          const int s = it % NS;
+          int inext = i + 1;
+          while (inext < p.nb && !bwd_tile_active(p, bmask, inext, j)) ++inext;
+          const bool has_next = inext < p.nb;
+          const int sn = (it + 1) % NS;
+          const int sd = it % NS_DO, sdn = (it + 1) % NS_DO;
+          const uint32_t acc = it > 0 ? 1u : 0u;
+          const uint64_t dOs = dO_mn + (uint64_t)(sd * TILE16), dQs = dQ_mn + (uint64_t)(s * TILE16);
 
-        // dV += P^T dO_i (reduction over the 128 queries of tile i), A = P^T from TMEM
-        ok = mbar_wait_spin(bar_p, it & 1, ab, lim, WAIT_BWD_MMA + 3);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, dOs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV,
-                  kk > 0 ? 1u : acc);
-        umma_commit(&bar_doe[sd]);  // dO_i read by dP_i and dV_i
-        // S^T_{i+1} over P^T_i (the dV MMAs above read it first: tcgen05.mma runs in order)
-        if (has_next) {
-          ok = mbar_wait_spin(&bar_qf[sn], ((it + 1) / NS) & 1, ab, lim, WAIT_BWD_MMA + 4);
+          // dV += P^T dO_i (reduction over the 128 queries of tile i), A = P^T from TMEM
+          ok = mbar_wait_spin(bar_p, it & 1, ab, lim, WAIT_BWD_MMA + 3);
           if (!ok) break;
           tc_fence_after();
-          issue_s(sn);
-          umma_commit(bar_s);
-        }
-        ok = mbar_wait_spin(bar_ds, it & 1, ab, lim, WAIT_BWD_MMA + 5);
-        if (!ok) break;
-        if (!C::DQ_ALIAS && it > 0) {  // d = 64: the dQ columns must have been drained
-          ok = mbar_wait_spin(bar_dqfree, (it - 1) & 1, ab, lim, WAIT_BWD_MMA + 6);
+  #pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, dOs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV,
+                    kk > 0 ? 1u : acc);
+          umma_commit(&bar_doe[sd]);  // dO_i read by dP_i and dV_i
+          // S^T_{i+1} over P^T_i (the dV MMAs above read it first: tcgen05.mma runs in order)
+          if (has_next) {
+            ok = mbar_wait_spin(&bar_qf[sn], ((it + 1) / NS) & 1, ab, lim, WAIT_BWD_MMA + 4);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(sn);
+            umma_commit(bar_s);
+          }
+          ok = mbar_wait_spin(bar_ds, it & 1, ab, lim, WAIT_BWD_MMA + 5);
           if (!ok) break;
-        }
-        tc_fence_after();
-        // dQ_i (d = 128: into the dP^T columns, already read by the dS phase)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // reduction over the 128 keys of tile j
-          const uint64_t kdesc = dK_mn + (uint64_t)(kk * (2048 >> 4)), sdesc = dS_mn + (uint64_t)(kk * (2048 >> 4));
-          umma_ss(tDQ, sdesc, kdesc, IDESC_Q, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar_dq);
-        // dK += dS^T Q_i
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
-          umma_ss(tDK, dS_k + aoff16, dQs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV, kk > 0 ? 1u : acc);
-        }
-        umma_commit(bar_dsfree);
-        umma_commit(&bar_qe[s]);
-        // dP^T_{i+1}
-        if (has_next) {
-          if (C::DQ_ALIAS) {  // the dP^T columns hold dQ_i until the drain warps have read it
-            ok = mbar_wait_spin(bar_dqfree, it & 1, ab, lim, WAIT_BWD_MMA + 7);
+          if (!C::DQ_ALIAS && it > 0) {  // d = 64: the dQ columns must have been drained
+            ok = mbar_wait_spin(bar_dqfree, (it - 1) & 1, ab, lim, WAIT_BWD_MMA + 6);
             if (!ok) break;
           }
-          ok = mbar_wait_spin(&bar_dof[sdn], ((it + 1) / NS_DO) & 1, ab, lim, WAIT_BWD_MMA + 10);
+          tc_fence_after();
+          // dQ_i (d = 128: into the dP^T columns, already read by the dS phase)
+  #pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {  // reduction over the 128 keys of tile j
+            const uint64_t kdesc = dK_mn + (uint64_t)(kk * (2048 >> 4)), sdesc = dS_mn + (uint64_t)(kk * (2048 >> 4));
+            umma_ss(tDQ, sdesc, kdesc, IDESC_Q, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar_dq);
+          // dK += dS^T Q_i
+  #pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t aoff16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
+            umma_ss(tDK, dS_k + aoff16, dQs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV, kk > 0 ? 1u : acc);
+          }
+          umma_commit(bar_dsfree);
+          umma_commit(&bar_qe[s]);
+          // dP^T_{i+1}
+          if (has_next) {
+            if (C::DQ_ALIAS) {  // the dP^T columns hold dQ_i until the drain warps have read it
+              ok = mbar_wait_spin(bar_dqfree, it & 1, ab, lim, WAIT_BWD_MMA + 7);
+              if (!ok) break;
+            }
+            ok = mbar_wait_spin(&bar_dof[sdn], ((it + 1) / NS_DO) & 1, ab, lim, WAIT_BWD_MMA + 10);
+            if (!ok) break;
+            tc_fence_after();
+            issue_dp(sdn);
+            umma_commit(bar_dp);
+          }
+          i = inext;
+          ++it;
+        }
+      } else {
+        // Panels come off the ring in the producer's order; each is released by a commit right
+        // after the MMAs that read it (commits track every earlier MMA, so release is in order).
+        // dV and dK take one 64-column panel of this CTA's half at a time (two N = 64 groups).
+        constexpr uint32_t IDESC_H64 = idesc_f32acc(128, 64, 0, 1, F16);
+        const uint64_t ring_k = sdesc_sw128(sQ, 16, 1024);               // a panel as K-major operand
+        const uint64_t ring_mn = sdesc_sw128(sQ, C::PANEL_BYTES, 1024);  // a panel as MN-major B
+        constexpr uint32_t P16 = C::PANEL_BYTES >> 4;
+        int npop = 0;
+        auto pop = [&](int where) -> int {  // next ring slot, once its panel has landed; -1: abort
+          const int sl = npop % C::RING;
+          const uint32_t ph = (uint32_t)(npop / C::RING) & 1u;
+          ++npop;
+          return mbar_wait_spin(&bar_qf[sl], ph, ab, lim, where) ? sl : -1;
+        };
+        auto issue_s = [&]() -> bool {  // S^T = sum over the four panels of K_j[:, p] Q_i[:, p]^T
+          for (int pn = 0; pn < C::PANELS; ++pn) {
+            const int sl = pop(WAIT_BWD_MMA + 2);
+            if (sl < 0) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_ss(tS, dK_k + (uint64_t)((pn * C::PANEL_BYTES + kk * 32) >> 4),
+                      ring_k + (uint64_t)(sl * P16 + ((kk * 32) >> 4)), IDESC_S, (pn > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(&bar_qe[sl]);
+          }
+          umma_commit(bar_s);
+          return true;
+        };
+        auto issue_dp = [&]() -> bool {  // dP^T = sum over the panels of V_j[:, p] dO_i[:, p]^T
+          for (int pn = 0; pn < C::PANELS; ++pn) {
+            const int sv = pop(WAIT_BWD_MMA + 9);
+            const int sd = sv < 0 ? -1 : pop(WAIT_BWD_MMA + 9);
+            if (sd < 0) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_ss(tDP, ring_k + (uint64_t)(sv * P16 + ((kk * 32) >> 4)),
+                      ring_k + (uint64_t)(sd * P16 + ((kk * 32) >> 4)), IDESC_S, (pn > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(&bar_qe[sv]);
+            umma_commit(&bar_qe[sd]);
+          }
+          umma_commit(bar_dp);
+          return true;
+        };
+        int i = i_begin;
+        while (i < p.nb && !bwd_tile_active(p, bmask, i, j)) ++i;
+        int it = 0;
+        if (ok && i < p.nb) ok = issue_s() && issue_dp();
+        while (ok && i < p.nb) {
+          int inext = i + 1;
+          while (inext < p.nb && !bwd_tile_active(p, bmask, inext, j)) ++inext;
+          const bool has_next = inext < p.nb;
+          const uint32_t acc = it > 0 ? 1u : 0u;
+          // dV_hh += P^T dO_i[:, half hh], A = P^T from TMEM, one 64-column panel at a time
+          ok = mbar_wait_spin(bar_p, it & 1, ab, lim, WAIT_BWD_MMA + 3);
+          for (int q = 0; q < 2 && ok; ++q) {
+            const int sl = pop(WAIT_BWD_MMA + 4);
+            if (sl < 0) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_ts(tDV + 64u * q, tS + (kk >> 2) * 64 + (kk & 3) * 8,
+                      ring_mn + (uint64_t)(sl * P16 + kk * (2048 >> 4)), IDESC_H64, kk > 0 ? 1u : acc);
+            umma_commit(&bar_qe[sl]);
+          }
+          if (!ok) break;
+          // S^T_{i+1} over P^T_i (the dV MMAs above read it first: tcgen05.mma runs in order)
+          if (has_next && !issue_s()) { ok = false; break; }
+          ok = mbar_wait_spin(bar_ds, it & 1, ab, lim, WAIT_BWD_MMA + 5);
           if (!ok) break;
           tc_fence_after();
-          issue_dp(sdn);
-          umma_commit(bar_dp);
+          // dQ_i[:, half hh] = dS_i K_j[:, half hh] into the dP^T columns (already read)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t kdesc = dK_mn + (uint64_t)(((2 * hh) * C::PANEL_BYTES) >> 4) + (uint64_t)(kk * (2048 >> 4));
+            const uint64_t sdesc = dS_mn + (uint64_t)(kk * (2048 >> 4));
+            umma_ss(tDQ, sdesc, kdesc, IDESC_Q, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar_dq);
+          // dK_hh += dS^T Q_i[:, half hh], one panel at a time
+          for (int q = 0; q < 2 && ok; ++q) {
+            const int sl = pop(WAIT_BWD_MMA + 6);
+            if (sl < 0) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t aoff16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
+              umma_ss(tDK + 64u * q, dS_k + aoff16, ring_mn + (uint64_t)(sl * P16 + kk * (2048 >> 4)), IDESC_H64,
+                      kk > 0 ? 1u : acc);
+            }
+            umma_commit(&bar_qe[sl]);
+          }
+          if (!ok) break;
+          umma_commit(bar_dsfree);
+          // dP^T_{i+1}: the dP^T columns hold dQ_i until the drain warps have read it
+          if (has_next) {
+            ok = mbar_wait_spin(bar_dqfree, it & 1, ab, lim, WAIT_BWD_MMA + 7);
+            if (ok) ok = issue_dp();
+            if (!ok) break;
+          }
+          i = inext;
+          ++it;
         }
-        i = inext;
-        ++it;
       }
       umma_commit(bar_acc);
       umma_commit(bar_done);
@@ -522,7 +705,7 @@ __global__ void __launch_bounds__(512, 1)
     // -------------------------------------------------------------- epilogue: dV (group h: panel h)
     if (ok) ok = warp_wait(bar_acc, 0, ab, lim, WAIT_BWD_EPILOGUE + 1);
     uint8_t* stage = smem + C::OFF_Q;  // Q ring stage 0 is free once every MMA retired
-    if (ok && h < C::PANELS) {
+    if (ok && h < C::PANELS_H) {
       tc_fence_after();
       stage_row16<64, F16>(tmem + lane_off + C::T_DV + 64u * h, smem_u32(stage + h * C::PANEL_BYTES), kr, p.inv_scale,
                          it == 0);
@@ -530,7 +713,8 @@ __global__ void __launch_bounds__(512, 1)
     }
     named_bar_sync(1, 256);
     if (warp == 4 && lane == 0 && *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
-      for (int pn = 0; pn < C::PANELS; ++pn) tma_store_3d(&tmdV, stage + pn * C::PANEL_BYTES, pn * 64, j * 128, bh);
+      for (int pn = 0; pn < C::PANELS_H; ++pn)
+        tma_store_3d(&tmdV, stage + pn * C::PANEL_BYTES, C::DH * hh + pn * 64, j * 128, bh);
       bulk_commit_group();
       bulk_wait_group_read0();
     }
@@ -557,9 +741,9 @@ __global__ void __launch_bounds__(512, 1)
       // Read the whole row and release the TMEM columns before anything else (at d = 128 the
       // next dP^T is written there). When aborting (!ok) the values are not used; the columns
       // stay allocated until every role has left.
-      uint32_t u[D];
+      uint32_t u[C::DH];
       tc_fence_after();
-      if constexpr (D == 128) {
+      if constexpr (C::DH == 128) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32_async(tDQ_row + c * 32, *reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
 #pragma unroll
@@ -585,7 +769,7 @@ __global__ void __launch_bounds__(512, 1)
         fence_proxy_async_smem();
         named_bar_sync(3, 128);  // slot written
         if (issuer) {
-          tma_reduce_add_2d(&tmdQa, slot, 32 * c, row0);
+          tma_reduce_add_2d(&tmdQa, slot, C::DH * hh + 32 * c, row0);
           bulk_commit_group();
         }
       }
@@ -594,15 +778,17 @@ __global__ void __launch_bounds__(512, 1)
     if (issuer) bulk_wait_group0();  // every reduction complete before the CTA exits
     // -------------------------------------------------------------- epilogue: dK (dS carries the scale)
     if (ok) ok = warp_wait(bar_acc, 0, ab, lim, WAIT_BWD_EPILOGUE + 2);
-    uint8_t* stage = smem + C::OFF_DO;  // dO ring stage 0, free once every MMA retired
+    // dO ring stage 0 (SPLIT: panel slots 2-3), free once every MMA retired
+    uint8_t* stage = smem + (C::SPLIT ? C::OFF_Q + 2 * C::PANEL_BYTES : C::OFF_DO);
     if (ok) {
       tc_fence_after();
-      stage_row16<D, F16>(tmem + lane_off + C::T_DK, smem_u32(stage), ln, 1.f, it == 0);
+      stage_row16<C::DH, F16>(tmem + lane_off + C::T_DK, smem_u32(stage), ln, 1.f, it == 0);
       fence_proxy_async_smem();
     }
     named_bar_sync(2, 128);
     if (wq == 0 && lane == 0 && *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
-      for (int pn = 0; pn < C::PANELS; ++pn) tma_store_3d(&tmdK, stage + pn * C::PANEL_BYTES, pn * 64, j * 128, bh);
+      for (int pn = 0; pn < C::PANELS_H; ++pn)
+        tma_store_3d(&tmdK, stage + pn * C::PANEL_BYTES, C::DH * hh + pn * 64, j * 128, bh);
       bulk_commit_group();
       bulk_wait_group_read0();
     }
@@ -625,7 +811,7 @@ static cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   cudaError_t e =
       cudaFuncSetAttribute(fa_bwd_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const dim3 grid = grid_bh(p.nbk, BH);
+  const dim3 grid = grid_bh(p.nbk * (C::SPLIT ? 2 : 1), BH);  // SPLIT: two CTAs (halves of d) per key tile
   fa_bwd_kernel<D, F16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdk, tdv, tdqa, p);
   return cudaGetLastError();
 }
@@ -635,9 +821,11 @@ cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk,
                             const CUtensorMap& tdqa, const BwdParams& p, long long BH, cudaStream_t stream) {
   if (p.f16) {
     if (D == 64) return launch_bwd_t<64, true>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+    if (D == 256) return launch_bwd_t<256, true>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
     return launch_bwd_t<128, true>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
   }
   if (D == 64) return launch_bwd_t<64, false>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+  if (D == 256) return launch_bwd_t<256, false>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
   return launch_bwd_t<128, false>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
 }
 

@@ -86,6 +86,9 @@ cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream) {
   const int grid = device_sm_count() * 8;  // 8 resident 256-thread blocks per SM
   if (p.D == 64)
     p.f16 ? fa_bwd_pre_kernel<64, true><<<grid, 256, 0, stream>>>(p) : fa_bwd_pre_kernel<64, false><<<grid, 256, 0, stream>>>(p);
+  else if (p.D == 256)
+    p.f16 ? fa_bwd_pre_kernel<256, true><<<grid, 256, 0, stream>>>(p)
+          : fa_bwd_pre_kernel<256, false><<<grid, 256, 0, stream>>>(p);
   else
     p.f16 ? fa_bwd_pre_kernel<128, true><<<grid, 256, 0, stream>>>(p)
           : fa_bwd_pre_kernel<128, false><<<grid, 256, 0, stream>>>(p);
@@ -97,6 +100,9 @@ cudaError_t launch_dq_finish(const DqFinishParams& p, cudaStream_t stream) {
   if (p.D == 64)
     p.f16 ? fa_dq_finish_kernel<64, true><<<grid, 256, 0, stream>>>(p)
           : fa_dq_finish_kernel<64, false><<<grid, 256, 0, stream>>>(p);
+  else if (p.D == 256)
+    p.f16 ? fa_dq_finish_kernel<256, true><<<grid, 256, 0, stream>>>(p)
+          : fa_dq_finish_kernel<256, false><<<grid, 256, 0, stream>>>(p);
   else
     p.f16 ? fa_dq_finish_kernel<128, true><<<grid, 256, 0, stream>>>(p)
           : fa_dq_finish_kernel<128, false><<<grid, 256, 0, stream>>>(p);

@@ -27,9 +27,10 @@
  *  - All pointers are device memory owned by the caller. The library allocates no device
  *    memory apart from one static device status word and the fixed scratch array that
  *    fa_bwd_noalloc uses.
- *  - Every pointer must be 16-byte aligned. d must be 64 or 128, or 256 in the forward calls
- *    (fa_fwd, fa_fwd_ex, fa_fwd_decode: one 128-row query tile per thread block there; the
- *    backward's dK and dV accumulators would not fit tensor memory). N is any positive length;
+ *  - Every pointer must be 16-byte aligned. d must be 64, 128 or 256 (at 256 the forward runs
+ *    one 128-row query tile per thread block and the backward two thread blocks per key tile,
+ *    one per 128-column half of d, because the dK and dV accumulators of a whole tile would not
+ *    fit tensor memory together). N is any positive length;
  *    a partial last 128-row tile is handled inside the kernels (rows and keys beyond N take no
  *    part and are never written).
  *  - B*H may be any positive count up to 2^31 - 1 (heads beyond 65535 are spread over two
@@ -54,8 +55,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID = 1,     /* null/misaligned pointer, non-positive size, non-finite scale */
-  FA_ERR_UNSUPPORTED = 2, /* valid but not implemented: d not in {64,128} (256: forward only);
-                             scale <= 0 */
+  FA_ERR_UNSUPPORTED = 2, /* valid but not implemented: d not in {64,128,256}; scale <= 0 */
   FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call or a kernel launch failed */
   FA_ERR_TIMEOUT = 4,     /* a device-side bounded wait gave up (see fa_last_device_status) */
   FA_ERR_WORKSPACE = 5    /* workspace pointer null or smaller than fa_bwd_workspace_bytes */
@@ -133,7 +133,7 @@ fa_status fa_bwd_dq_finish(void* dq, int B, int H, int N, int d, void* workspace
  * from a fixed array of FA_NOALLOC_SCRATCH_BYTES in the library's device memory, reserved
  * on every GPU that loads the library until the process exits. Problems whose
  * fa_bwd_workspace_bytes exceed it return FA_ERR_WORKSPACE (about (d+2)*4 bytes per query
- * row: B*H*N up to ~129k rows at d = 128, ~254k at d = 64). Allocates nothing.
+ * row: B*H*N up to ~65k rows at d = 256, ~129k at d = 128, ~254k at d = 64). Allocates nothing.
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress)
  * with that device current; make that first call before any stream capture. All calls share
  * the one array: calls whose kernels overlap on the GPU (different streams, no ordering)

@@ -52,8 +52,8 @@ def test_fwd_argument_checks(lib):
     assert fwd(lib, B=0) == 1 and fwd(lib, H=-1) == 1 and fwd(lib, N=0) == 1
     assert fwd(lib, scale=math.nan) == 1 and fwd(lib, scale=math.inf) == 1
     assert fwd(lib, d=96) == 2                   # unsupported head dim
-    assert fwd(lib, d=512) == 2                  # (d = 256 is a supported forward head dim)
-    assert lib.fa_bwd_workspace_bytes(1, 1, 128, 256) == 0   # ... but not a backward one
+    assert fwd(lib, d=512) == 2                  # (d = 256 is supported)
+    assert lib.fa_bwd_workspace_bytes(1, 1, 128, 256) == 2 * 512 + 128 * 256 * 4  # and a backward one
     assert fwd(lib, N=0) == 1                    # empty sequence -> INVALID
     assert fwd(lib, B=65536, H=65536) == 2      # B*H above the TMA head coordinate's range
 

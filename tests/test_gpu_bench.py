@@ -51,7 +51,8 @@ def test_step_line_with_e2e():
         assert p["B"] * p["N"] == 16384 and p["H"] * p["d"] == 2048
         assert 0 < p["fwd_tflops"] and 0 < p["fwd_bwd_tflops"]
         assert abs(p["pct_of_peak_fwd"] - 100 * p["fwd_tflops"] / sw["peak"]) < 0.1
-    assert set(sw["configs"]) == {"bert_large_shape", "gpt2_shape_causal", "block_sparse"}
+    assert set(sw["configs"]) == {"bert_large_shape", "gpt2_shape_causal", "block_sparse", "head_dim_256",
+                                  "head_dim_256_causal"}
     assert 0.2 < sw["configs"]["block_sparse"]["block_density"] < 0.35
     assert "sm_mhz" in sw["clocks"]
 

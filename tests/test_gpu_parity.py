@@ -135,20 +135,52 @@ def test_per_head_block_masks(fa, oracle_mod, B, Hh, N, d, causal):
             H.assert_grads_close([x[sl] for x in outs[2:]], g_ref, f"head {b},{h}")
 
 
-@pytest.mark.parametrize("B,Hh,N,causal,mask", [(1, 2, 384, False, None), (2, 1, 333, True, None),
-                                                (1, 1, 640, False, "bernoulli")])
-def test_forward_head_dim_256(fa, oracle_mod, B, Hh, N, causal, mask):
-    # d = 256: one 128-row query tile per thread block (forward only)
+HEAD_DIM_256 = [
+    # B, H, N, causal, mask, dtype: d = 256 (forward: one query tile per CTA; backward: two CTAs
+    # per key tile, one per 128-column half of d, Q/dO/V streamed as 64-column panels)
+    (1, 2, 384, False, None, "bf16"),
+    (2, 1, 333, True, None, "bf16"),       # ragged, causal
+    (1, 1, 640, False, "bernoulli", "bf16"),
+    (1, 2, 128, True, None, "bf16"),       # a single tile
+    (1, 1, 1000, True, None, "bf16"),      # many query tiles per key tile: the ring wraps often
+    (1, 2, 520, False, None, "f16"),
+]
+
+
+@pytest.mark.parametrize("B,Hh,N,causal,mask,dtype", HEAD_DIM_256)
+def test_head_dim_256(fa, oracle_mod, B, Hh, N, causal, mask, dtype):
     d = 256
-    gpu, ref = H.make_case(B, Hh, N, d, seed=synth.BASE_SEED + N + 256, with_do=False)
+    gpu, ref = H.make_case(B, Hh, N, d, seed=synth.BASE_SEED + N + 256, dtype=dtype)
     scale = 1.0 / np.sqrt(d)
     m = mask_for(mask, N)
     mt = None if m is None else torch.from_numpy(m).cuda()
     o, lse = run_fwd(fa, gpu, causal, mt, scale)
     o_ref, l_ref = oracle_mod.attention_fwd(ref["q"], ref["k"], ref["v"], scale, causal=causal, mask=m)
-    H.assert_fwd_close(H.to_f64(o), H.to_f64(lse), o_ref, l_ref, f"d=256 {B,Hh,N,causal,mask}")
-    with pytest.raises(fa.FAError):  # no backward at d = 256
-        fa.backward(gpu["q"], gpu["k"], gpu["v"], o, gpu["q"], lse, causal=causal, block_mask=mt, scale=scale)
+    H.assert_fwd_close(H.to_f64(o), H.to_f64(lse), o_ref, l_ref, f"d=256 fwd {B,Hh,N,causal,mask,dtype}")
+    dq, dk, dv = run_bwd(fa, gpu, o, lse, causal, mt, scale)
+    g_ref = oracle_mod.attention_bwd(ref["q"], ref["k"], ref["v"], ref["do"], scale, causal=causal, mask=m)[:3]
+    H.assert_grads_close([H.to_f64(x) for x in (dq, dk, dv)], g_ref, f"d=256 bwd {B,Hh,N,causal,mask,dtype}")
+
+
+def test_head_dim_256_sweep_shape(fa, oracle_mod):
+    # The sweep's 16k-token, hidden-2048 batch at d = 256 (B = 4, H = 8, N = 4096) in one launch
+    # of each kernel; one sampled head against the oracle in full.
+    check_heads(fa, oracle_mod, 4, 8, 4096, 256, True, None, nheads=1, seed=synth.BASE_SEED + 256)
+
+
+def test_head_dim_256_general_shape(fa, oracle_mod):
+    # d = 256 through the general-shape backward (N_q != N_k, bottom-right causal)
+    B, Hh, Nq, Nk, d = 1, 2, 200, 450, 256
+    seed = synth.BASE_SEED + 4
+    gq, rq = H.make_case(B, Hh, Nq, d, seed=seed)
+    gk, rk = H.make_case(B, Hh, Nk, d, seed=seed + 500, with_do=False)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = fa.forward_decode(gq["q"], gk["k"], gk["v"], causal=True, scale=scale)
+    dq, dk, dv = fa.backward_qk(gq["q"], gk["k"], gk["v"], o, gq["do"], lse, causal=True, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.last_device_status() == 0
+    g_ref = oracle_mod.attention_bwd_qk(rq["q"], rk["k"], rk["v"], rq["do"], scale, causal=True)[:3]
+    H.assert_grads_close([H.to_f64(x) for x in (dq, dk, dv)], g_ref, "d=256 general bwd")
 
 
 DECODE = [
