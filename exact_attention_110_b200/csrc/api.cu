@@ -150,6 +150,8 @@ fa_status fa_fwd_ex(int dtype, const void* q, const void* k, const void* v, void
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
   p.f16 = f16;
+  const int items = (p.nb + fa::fwd_tiles_per_cta(d, p.nb) - 1) / fa::fwd_tiles_per_cta(d, p.nb);
+  p.order_group = fa::causal_group(p.causal, items, BH, fa::device_sm_count());
   return from_cuda(fa::launch_fwd(d, tq, tk, tv, to, p, BH, static_cast<cudaStream_t>(stream)));
 }
 
@@ -255,6 +257,8 @@ fa_status fa_fwd_decode(int dtype, const void* q, const void* k, const void* v, 
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
   p.f16 = f16;
+  const int tpc = fa::fwd_tiles_per_cta(d, p.nb);
+  p.order_group = fa::causal_group(p.causal, (p.nb + tpc - 1) / tpc * ns, BH, fa::device_sm_count());
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = fa::launch_fwd(d, tq, tk, tv, to, p, BH, s);
   if (e != cudaSuccess || ns == 1) return from_cuda(e);
@@ -372,6 +376,7 @@ fa_status plan_bwd_main(int dtype, const void* q, const void* k, const void* v, 
   p.nbk = (sh.Nk + 127) / 128;
   p.causal = causal ? 1 : 0;
   p.causal_off = sh.causal_off;
+  p.order_group = fa::causal_group(p.causal, p.nbk * (sh.d == 256 ? 2 : 1), BH, fa::device_sm_count());
   p.inv_scale = 1.0f / scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;

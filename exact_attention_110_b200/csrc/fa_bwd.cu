@@ -175,13 +175,11 @@ __global__ void __launch_bounds__(512, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   AbortState* ab = reinterpret_cast<AbortState*>(smem + C::OFF_MISC + 4);
 
-  const long long bh_l = cta_bh();
-  if (bh_l >= p.BH) return;  // past the last head (head counts above 65535 round the grid up)
-  const int bh = (int)bh_l;
+  int bh, xj;  // head and work item: key tile j (SPLIT: 2j + half of d); causal: j = 0 is the heaviest
+  if (!cta_work(p.BH, p.nbk * (C::SPLIT ? 2 : 1), p.order_group, bh, xj)) return;
   const uint8_t* bmask = p.block_mask == nullptr ? nullptr : p.block_mask + (size_t)bh * p.mask_stride;
-  // key tile (causal: j = 0 has the most work and starts first); SPLIT: and the half of d
-  const int j = C::SPLIT ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-  const int hh = C::SPLIT ? (int)(blockIdx.x & 1) : 0;
+  const int j = C::SPLIT ? (xj >> 1) : xj;
+  const int hh = C::SPLIT ? (xj & 1) : 0;
   // causal: the first query tile whose last row sees key tile j's first key
   const int i_first = 128 * j - 127 - p.causal_off;
   const int i_begin = (p.causal && i_first > 0) ? (i_first + 127) / 128 : 0;
@@ -358,7 +356,7 @@ __global__ void __launch_bounds__(512, 1)
       if constexpr (!C::SPLIT) {
         auto issue_s = [&](int st) {
           const uint64_t b = dQ_k + (uint64_t)(st * TILE16);
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
             umma_ss(tS, dK_k + off16, b + off16, IDESC_S, kk > 0 ? 1u : 0u);
@@ -366,7 +364,7 @@ __global__ void __launch_bounds__(512, 1)
         };
         auto issue_dp = [&](int st) {
           const uint64_t b = dO_k + (uint64_t)(st * TILE16);
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
             umma_ss(tDP, dV_k + off16, b + off16, IDESC_S, kk > 0 ? 1u : 0u);
@@ -404,7 +402,7 @@ __global__ void __launch_bounds__(512, 1)
           ok = mbar_wait_spin(bar_p, it & 1, ab, lim, WAIT_BWD_MMA + 3);
           if (!ok) break;
           tc_fence_after();
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             umma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, dOs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV,
                     kk > 0 ? 1u : acc);
@@ -425,14 +423,14 @@ __global__ void __launch_bounds__(512, 1)
           }
           tc_fence_after();
           // dQ_i (d = 128: into the dP^T columns, already read by the dS phase)
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk) {  // reduction over the 128 keys of tile j
             const uint64_t kdesc = dK_mn + (uint64_t)(kk * (2048 >> 4)), sdesc = dS_mn + (uint64_t)(kk * (2048 >> 4));
             umma_ss(tDQ, sdesc, kdesc, IDESC_Q, kk > 0 ? 1u : 0u);
           }
           umma_commit(bar_dq);
           // dK += dS^T Q_i
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t aoff16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
             umma_ss(tDK, dS_k + aoff16, dQs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV, kk > 0 ? 1u : acc);
@@ -811,7 +809,7 @@ static cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   cudaError_t e =
       cudaFuncSetAttribute(fa_bwd_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const dim3 grid = grid_bh(p.nbk * (C::SPLIT ? 2 : 1), BH);  // SPLIT: two CTAs (halves of d) per key tile
+  const dim3 grid = grid_work(p.nbk * (C::SPLIT ? 2 : 1), BH, p.order_group);  // SPLIT: two CTAs per key tile
   fa_bwd_kernel<D, F16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdk, tdv, tdqa, p);
   return cudaGetLastError();
 }

@@ -210,13 +210,11 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   AbortState* ab = reinterpret_cast<AbortState*>(smem + C::OFF_MISC + 4);
 
-  const long long bh_l = cta_bh();
-  if (bh_l >= p.BH) return;  // past the last head (head counts above 65535 round the grid up)
-  const int bh = (int)bh_l;
+  const int npairs = (p.nb + C::TILES - 1) / C::TILES;
+  int bh, xi;  // head and work item = pair index * nsplit + split; causal: the heaviest pairs first
+  if (!cta_work(p.BH, npairs * p.nsplit, p.order_group, bh, xi)) return;
   const uint8_t* bmask = p.block_mask == nullptr ? nullptr : p.block_mask + (size_t)bh * p.mask_stride;
-  // blockIdx.x = pair index * nsplit + split; causal grids start with the heaviest pairs
-  const int pi = (int)blockIdx.x / p.nsplit, split = (int)blockIdx.x - pi * p.nsplit;
-  const int npairs = (int)gridDim.x / p.nsplit;
+  const int pi = xi / p.nsplit, split = xi - pi * p.nsplit;
   const int pair = p.causal ? npairs - 1 - pi : pi;
   const int qb0 = C::TILES * pair;  // 128-row tile index of tile 0
   // this CTA's key tiles: its split's range, cut at the last key the pair's last row sees
@@ -821,7 +819,7 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   cudaError_t e =
       cudaFuncSetAttribute(fa_fwd_kernel<D, F16, ONE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const dim3 grid = grid_bh((p.nb + C::TILES - 1) / C::TILES * p.nsplit, BH);
+  const dim3 grid = grid_work((p.nb + C::TILES - 1) / C::TILES * p.nsplit, BH, p.order_group);
   fa_fwd_kernel<D, F16, ONE><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }

@@ -356,6 +356,25 @@ def test_misaligned_dq_leaves_outputs_untouched(fa):
     assert torch.all(dk == 3.0) and torch.all(dv == -2.0)
 
 
+@pytest.mark.parametrize("N,d", [(256, 64), (640, 128), (300, 256)])
+def test_causal_grid_order_with_a_partial_last_group(fa, oracle_mod, N, d):
+    # Causal grids enumerate heads in groups (longest work items first within a group); with
+    # 300 heads the last group is partial. Heads at both ends and inside the partial group must
+    # match the oracle in both passes.
+    B, Hh = 100, 3
+    gpu, ref = H.make_case(B, Hh, N, d, seed=synth.BASE_SEED + 300 + N)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = run_fwd(fa, gpu, True, None, scale)
+    dq, dk, dv = run_bwd(fa, gpu, o, lse, True, None, scale)
+    for (b, h) in ((0, 0), (49, 1), (98, 2), (99, 0), (99, 2)):
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        args = [ref[k][sl] for k in ("q", "k", "v")]
+        o_ref, l_ref = oracle_mod.attention_fwd(*args, scale, causal=True)
+        H.assert_fwd_close(H.to_f64(o[sl]), H.to_f64(lse[sl]), o_ref, l_ref, f"head {b},{h}")
+        g_ref = oracle_mod.attention_bwd(*args, ref["do"][sl], scale, causal=True)[:3]
+        H.assert_grads_close([H.to_f64(x[sl]) for x in (dq, dk, dv)], g_ref, f"head {b},{h}")
+
+
 def test_masked_blocks_do_not_influence_output(fa):
     # Keys/values in blocks that are off (or in the causal future) must not change O at all.
     N, d = 512, 64
