@@ -387,6 +387,7 @@ def run_sweep(fa, dev, dtype, steps, warmup, peaks):
         return t
 
     def entry(B, H, N, d, causal, mask_np):
+        time.sleep(0.25)  # each point starts from an idle GPU, as a burst measurement does
         mask = None if mask_np is None else torch.from_numpy(mask_np).to(dev)
         density = float(mask_np.mean()) if mask_np is not None else 1.0
         (f_ms, p_ms, m_ms, d_ms), step_ms = time_kernels(fa, views(B, H, N, d), (B, H, N, d), causal, mask,

@@ -111,9 +111,14 @@ struct BwdCfg {
 // bmask: this (b, h)'s block mask (or null), [query tiles][key tiles]. Causal: key tile j is
 // active for query tile i when its first key is visible to the tile's last row
 // (128j <= 128i + 127 + causal_off; i >= j for the square problem).
-__device__ __forceinline__ bool bwd_tile_active(const BwdParams& p, const uint8_t* bmask, int i, int j) {
-  if (p.causal && 128 * j > 128 * i + 127 + p.causal_off) return false;
-  if (bmask != nullptr && bmask[i * p.nbk + j] == 0) return false;
+// The fields are copied out of the kernel parameters once per thread (see fa_fwd.cu, TileTest).
+struct BwdTiles {
+  int nb, nbk, Nk, causal, causal_off;
+  const uint8_t* bmask;
+};
+__device__ __forceinline__ bool bwd_tile_active(const BwdTiles& tt, int i, int j) {
+  if (tt.causal && 128 * j > 128 * i + 127 + tt.causal_off) return false;
+  if (tt.bmask != nullptr && tt.bmask[i * tt.nbk + j] == 0) return false;
   return true;
 }
 
@@ -178,6 +183,7 @@ __global__ void __launch_bounds__(512, 1)
   int bh, xj;  // head and work item: key tile j (SPLIT: 2j + half of d); causal: j = 0 is the heaviest
   if (!cta_work(p.BH, p.nbk * (C::SPLIT ? 2 : 1), p.order_group, bh, xj)) return;
   const uint8_t* bmask = p.block_mask == nullptr ? nullptr : p.block_mask + (size_t)bh * p.mask_stride;
+  const BwdTiles tt{p.nb, p.nbk, p.Nk, p.causal, p.causal_off, bmask};
   const int j = C::SPLIT ? (xj >> 1) : xj;
   const int hh = C::SPLIT ? (xj & 1) : 0;
   // causal: the first query tile whose last row sees key tile j's first key
@@ -238,8 +244,8 @@ __global__ void __launch_bounds__(512, 1)
         for (int s = 0; s < NS; ++s) issued[s] = -1;
         for (int s = 0; s < NS_DO; ++s) issued_do[s] = -1;
         bool ok = true;
-        for (int i = i_begin; i < p.nb; ++i) {
-          if (!bwd_tile_active(p, bmask, i, j)) continue;
+        for (int i = i_begin; i < tt.nb; ++i) {
+          if (!bwd_tile_active(tt, i, j)) continue;
           // Q_i first: its stage frees at dK_{i-NS}, before dO_i's stage frees at dV_{i-NS_DO}.
           const int s = it % NS;
           const uint32_t ph = (it / NS) & 1;
@@ -313,12 +319,12 @@ __global__ void __launch_bounds__(512, 1)
           return true;
         };
         int i = i_begin;
-        while (i < p.nb && !bwd_tile_active(p, bmask, i, j)) ++i;
-        if (i < p.nb) ok = push_s(i) && push_dp(i);
-        while (ok && i < p.nb) {
+        while (i < tt.nb && !bwd_tile_active(tt, i, j)) ++i;
+        if (i < tt.nb) ok = push_s(i) && push_dp(i);
+        while (ok && i < tt.nb) {
           int inext = i + 1;
-          while (inext < p.nb && !bwd_tile_active(p, bmask, inext, j)) ++inext;
-          const bool has_next = inext < p.nb;
+          while (inext < tt.nb && !bwd_tile_active(tt, inext, j)) ++inext;
+          const bool has_next = inext < tt.nb;
           ok = push(&tmdO, 128 * hh, i * 128, -1) && push(&tmdO, 128 * hh + 64, i * 128, -1);
           if (ok && has_next) ok = push_s(inext);
           if (ok) ok = push(&tmQ, 128 * hh, i * 128, -1) && push(&tmQ, 128 * hh + 64, i * 128, -1);
@@ -372,9 +378,9 @@ __global__ void __launch_bounds__(512, 1)
         };
 
         int i = i_begin;
-        while (i < p.nb && !bwd_tile_active(p, bmask, i, j)) ++i;
+        while (i < tt.nb && !bwd_tile_active(tt, i, j)) ++i;
         int it = 0;
-        if (ok && i < p.nb) {
+        if (ok && i < tt.nb) {
           ok = mbar_wait_spin(&bar_qf[0], 0, ab, lim, WAIT_BWD_MMA + 2);
           if (ok) {
             tc_fence_after();
@@ -388,11 +394,11 @@ __global__ void __launch_bounds__(512, 1)
             umma_commit(bar_dp);
           }
         }
-        while (ok && i < p.nb) {
+        while (ok && i < tt.nb) {
           const int s = it % NS;
           int inext = i + 1;
-          while (inext < p.nb && !bwd_tile_active(p, bmask, inext, j)) ++inext;
-          const bool has_next = inext < p.nb;
+          while (inext < tt.nb && !bwd_tile_active(tt, inext, j)) ++inext;
+          const bool has_next = inext < tt.nb;
           const int sn = (it + 1) % NS;
           const int sd = it % NS_DO, sdn = (it + 1) % NS_DO;
           const uint32_t acc = it > 0 ? 1u : 0u;
@@ -498,13 +504,13 @@ __global__ void __launch_bounds__(512, 1)
           return true;
         };
         int i = i_begin;
-        while (i < p.nb && !bwd_tile_active(p, bmask, i, j)) ++i;
+        while (i < tt.nb && !bwd_tile_active(tt, i, j)) ++i;
         int it = 0;
-        if (ok && i < p.nb) ok = issue_s() && issue_dp();
-        while (ok && i < p.nb) {
+        if (ok && i < tt.nb) ok = issue_s() && issue_dp();
+        while (ok && i < tt.nb) {
           int inext = i + 1;
-          while (inext < p.nb && !bwd_tile_active(p, bmask, inext, j)) ++inext;
-          const bool has_next = inext < p.nb;
+          while (inext < tt.nb && !bwd_tile_active(tt, inext, j)) ++inext;
+          const bool has_next = inext < tt.nb;
           const uint32_t acc = it > 0 ? 1u : 0u;
           // dV_hh += P^T dO_i[:, half hh], A = P^T from TMEM, one 64-column panel at a time
           ok = mbar_wait_spin(bar_p, it & 1, ab, lim, WAIT_BWD_MMA + 3);
@@ -578,18 +584,18 @@ __global__ void __launch_bounds__(512, 1)
     const Ex2PolyConsts ek = ex2_poly_consts();
     bool ok = true;
     int it = 0;
-    for (int i = i_begin; i < p.nb; ++i) {
-      if (!bwd_tile_active(p, bmask, i, j)) continue;
+    for (int i = i_begin; i < tt.nb; ++i) {
+      if (!bwd_tile_active(tt, i, j)) continue;
       const int s = it % NS;
       const float* nlse2 = reinterpret_cast<const float*>(smem + C::OFF_LSE + s * 512) + 64 * h;
       const float* ndel = reinterpret_cast<const float*>(smem + C::OFF_DEL + s * 512) + 64 * h;
       // Causal band: key 128j+kr is visible to query 128i+q iff 128j+kr <= 128i+q+causal_off,
       // i.e. q >= qmin (q >= kr on the diagonal tile of the square problem).
-      const bool diag = p.causal && (128 * j + 127 > 128 * i + p.causal_off);
-      const int qmin = kr + 128 * (j - i) - p.causal_off;
+      const bool diag = tt.causal && (128 * j + 127 > 128 * i + tt.causal_off);
+      const int qmin = kr + 128 * (j - i) - tt.causal_off;
       // Keys of a partial last tile beyond N_k (zero rows from TMA) take no part: P = 0 there,
       // so nothing non-finite can reach dQ through them.
-      const bool kpad = 128 * j + kr >= p.Nk;
+      const bool kpad = 128 * j + kr >= tt.Nk;
       const int qoff = 64 * h;  // query index of column 0 of this group
 
       // ---- P phase: P^T = exp2(S^T * scale*log2e - LSE*log2e), back into TMEM as bf16
@@ -733,8 +739,8 @@ __global__ void __launch_bounds__(512, 1)
     bool ok = true;
     int it = 0;
     uint32_t nred = 0;  // bulk reductions issued so far (staging slot = nred % DQ_SLOTS)
-    for (int i = i_begin; i < p.nb; ++i) {
-      if (!bwd_tile_active(p, bmask, i, j)) continue;
+    for (int i = i_begin; i < tt.nb; ++i) {
+      if (!bwd_tile_active(tt, i, j)) continue;
       ok = warp_wait(bar_dq, it & 1, ab, lim, WAIT_BWD_DQ + 1);
       // Read the whole row and release the TMEM columns before anything else (at d = 128 the
       // next dP^T is written there). When aborting (!ok) the values are not used; the columns

@@ -88,12 +88,21 @@ struct FwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// bmask: this (b, h)'s block mask (or null). Causal: tile j is active when the last row of
-// tile qb sees its first key (128j <= 128qb + 127 + causal_off; j <= qb for the square problem).
-__device__ __forceinline__ bool fwd_tile_active(const FwdParams& p, const uint8_t* bmask, int qb, int j) {
-  if (qb >= p.nb) return false;
-  if (p.causal && 128 * j > 128 * qb + 127 + p.causal_off) return false;
-  if (bmask != nullptr && bmask[qb * p.nbk + j] == 0) return false;
+// What the tile test needs, copied out of the kernel parameters once per thread. The test runs
+// between inline-asm statements that clobber memory (MMA issue, barrier waits); read straight
+// from the parameters, every test after such a statement reloads them from constant space as
+// a chain of dependent loads (measured: ~500 cycles per step of the MMA-issuing thread).
+// bmask: this (b, h)'s block mask (or null).
+struct TileTest {
+  int nb, nbk, Nk, causal, causal_off;
+  const uint8_t* bmask;
+};
+// Causal: tile j is active when the last row of tile qb sees its first key
+// (128j <= 128qb + 127 + causal_off; j <= qb for the square problem).
+__device__ __forceinline__ bool fwd_tile_active(const TileTest& tt, int qb, int j) {
+  if (qb >= tt.nb) return false;
+  if (tt.causal && 128 * j > 128 * qb + 127 + tt.causal_off) return false;
+  if (tt.bmask != nullptr && tt.bmask[qb * tt.nbk + j] == 0) return false;
   return true;
 }
 
@@ -214,6 +223,7 @@ __global__ void __launch_bounds__(384, 1)
   int bh, xi;  // head and work item = pair index * nsplit + split; causal: the heaviest pairs first
   if (!cta_work(p.BH, npairs * p.nsplit, p.order_group, bh, xi)) return;
   const uint8_t* bmask = p.block_mask == nullptr ? nullptr : p.block_mask + (size_t)bh * p.mask_stride;
+  const TileTest tt{p.nb, p.nbk, p.Nk, p.causal, p.causal_off, bmask};
   const int pi = xi / p.nsplit, split = xi - pi * p.nsplit;
   const int pair = p.causal ? npairs - 1 - pi : pi;
   const int qb0 = C::TILES * pair;  // 128-row tile index of tile 0
@@ -295,7 +305,7 @@ __global__ void __launch_bounds__(384, 1)
           return true;
         };
         for (int j = j_begin; j < j_end && ok; ++j) {
-          if (!fwd_tile_active(p, bmask, qb0, j)) continue;
+          if (!fwd_tile_active(tt, qb0, j)) continue;
           const int ks = a % NS;
           const uint32_t kph = (uint32_t)(a / NS) & 1u;
           ok = mbar_wait(&bar_ke[ks], kph ^ 1u, ab, lim, WAIT_FWD_LOAD + 1);
@@ -313,7 +323,7 @@ __global__ void __launch_bounds__(384, 1)
         if (ok && a >= 2) ok = load_v(j_prev, a - 1);
       }
       for (int j = j_begin; C::TILES == 2 && j < j_end && ok; ++j) {
-        if (!fwd_tile_active(p, bmask, qb0, j) && !fwd_tile_active(p, bmask, qb0 + 1, j)) continue;
+        if (!fwd_tile_active(tt, qb0, j) && !fwd_tile_active(tt, qb0 + 1, j)) continue;
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
         ok = mbar_wait(&bar_ke[s], ph ^ 1, ab, lim, WAIT_FWD_LOAD + 1);
@@ -382,7 +392,7 @@ __global__ void __launch_bounds__(384, 1)
         };
         int a = 0;
         for (int j = j_begin; j < j_end && ok; ++j) {
-          if (!fwd_tile_active(p, bmask, qb0, j)) continue;
+          if (!fwd_tile_active(tt, qb0, j)) continue;
           if (a >= 2) ok = issue_pv(a - 2);
           const int ks = a % NS;
           if (ok) ok = mbar_wait_spin(&bar_kf[ks], (uint32_t)(a / NS) & 1u, ab, lim, WAIT_FWD_MMA + 2);
@@ -409,8 +419,8 @@ __global__ void __launch_bounds__(384, 1)
       int it = 0;
 
       for (int j = j_begin; C::TILES == 2 && j < j_end && ok; ++j) {
-        const bool act0 = fwd_tile_active(p, bmask, qb0, j);
-        const bool act1 = fwd_tile_active(p, bmask, qb0 + 1, j);
+        const bool act0 = fwd_tile_active(tt, qb0, j);
+        const bool act1 = fwd_tile_active(tt, qb0 + 1, j);
         if (!act0 && !act1) continue;
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
@@ -513,11 +523,11 @@ __global__ void __launch_bounds__(384, 1)
       int a = 0;                // active KV tiles so far
 
       for (int j = j_begin; tvalid && j < j_end; ++j) {
-        if (!fwd_tile_active(p, bmask, qb, j)) continue;
+        if (!fwd_tile_active(tt, qb, j)) continue;
         const uint32_t b = (uint32_t)(a & 1);
         const uint32_t tS = tS_row + b * 128u;
-        const bool diag = p.causal && (128 * j + 127 > 128 * qb + p.causal_off);
-        const bool masked = diag || (128 * j + 128 > p.Nk);
+        const bool diag = tt.causal && (128 * j + 127 > 128 * qb + tt.causal_off);
+        const bool masked = diag || (128 * j + 128 > tt.Nk);
         uint32_t su[64];  // this row's scores of this half (fp32 bits)
         float mh = -INFINITY;
         if (ok) ok = warp_wait(&bar_s[b], (uint32_t)(a >> 1) & 1u, ab, lim, WAIT_FWD_SOFTMAX + 1);
@@ -525,7 +535,7 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
           tmem_ld64(tS + 64u * h, su);
           if (masked) {  // same rule as two tiles, for key columns 64h..64h+63
-            const int lim_c = min(diag ? 128 * (qb - j) + r + p.causal_off + 1 : 128, p.Nk - 128 * j) - 64 * h;
+            const int lim_c = min(diag ? 128 * (qb - j) + r + tt.causal_off + 1 : 128, tt.Nk - 128 * j) - 64 * h;
 #pragma unroll
             for (int c = 0; c < 64; ++c)
               if (c >= lim_c) su[c] = 0xff800000u;  // -inf
@@ -674,7 +684,7 @@ __global__ void __launch_bounds__(384, 1)
 
       if (tvalid) {
         for (int j = j_begin; j < j_end; ++j) {
-          if (!fwd_tile_active(p, bmask, qb, j)) continue;
+          if (!fwd_tile_active(tt, qb, j)) continue;
           ok = warp_wait(&bar_s[t], s_phase, ab, lim, WAIT_FWD_SOFTMAX + 1);
           if (!ok) break;
           s_phase ^= 1u;
@@ -685,10 +695,10 @@ __global__ void __launch_bounds__(384, 1)
           // Elementwise mask: on the causal diagonal band key 128j+c is visible to row 128qb+r iff
           // 128j+c <= 128qb+r+causal_off (c <= r for the square problem); in a partial last key
           // tile keys 128j+c >= Nk do not exist (TMA filled zeros).
-          const bool diag = p.causal && (128 * j + 127 > 128 * qb + p.causal_off);
-          const bool masked = diag || (128 * j + 128 > p.Nk);
+          const bool diag = tt.causal && (128 * j + 127 > 128 * qb + tt.causal_off);
+          const bool masked = diag || (128 * j + 128 > tt.Nk);
           if (masked) {
-            const int lim = min(diag ? 128 * (qb - j) + r + p.causal_off + 1 : 128, p.Nk - 128 * j);
+            const int lim = min(diag ? 128 * (qb - j) + r + tt.causal_off + 1 : 128, tt.Nk - 128 * j);
 #pragma unroll
             for (int c = 0; c < 128; ++c)
               if (c >= lim) su[c] = 0xff800000u;  // -inf
