@@ -88,10 +88,9 @@ struct FwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-// What the tile test needs, copied out of the kernel parameters once per thread. The test runs
-// between inline-asm statements that clobber memory (MMA issue, barrier waits); read straight
-// from the parameters, every test after such a statement reloads them from constant space as
-// a chain of dependent loads (measured: ~500 cycles per step of the MMA-issuing thread).
+// What the tile test needs, copied out of the kernel parameters once per thread: the test runs
+// between inline-asm statements that clobber memory (MMA issue, barrier waits), after which
+// fields read straight from the parameters would be reloaded from constant space.
 // bmask: this (b, h)'s block mask (or null).
 struct TileTest {
   int nb, nbk, Nk, causal, causal_off;
