@@ -485,37 +485,71 @@ def run_gpu(args, wl, rank, world, local_rank, dist_on):
     peaks = load_peaks()
 
     # ---- end to end through the public API with pinned host buffers
+    # Every step copies its inputs (q, k, v, dO) in from pinned host memory and its results
+    # (o, lse, dq, dk, dv) back out. Steps are pipelined over three streams with two sets of
+    # device buffers, as a training loop would overlap its transfers: step k's compute runs while
+    # step k+1's inputs arrive and step k-1's results leave; events order each buffer's reuse.
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
-        ho, hdq, hdk, hdv = (torch.empty(shape, dtype=q.dtype).pin_memory() for _ in range(4))
-        hl = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+        hin = [t.cpu().pin_memory() for t in (q, k, v, do)]
+        hout = [torch.empty(shape, dtype=q.dtype).pin_memory() for _ in range(4)] + \
+               [torch.empty((B, H, N), dtype=torch.float32).pin_memory()]
+        din = [[torch.empty_like(t) for t in (q, k, v, do)] for _ in range(2)]
+        dout = [[torch.empty_like(q) for _ in range(4)] + [torch.empty((B, H, N), device=dev, dtype=torch.float32)]
+                for _ in range(2)]
+        s_in, s_c, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_c = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        issued = [False, False]
 
-        def e2e_step():
-            q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True); do.copy_(hdo, non_blocking=True)
-            fa.forward(q, k, v, causal=causal, block_mask=mask, scale=scale, out=o, lse=lse)
-            fa.backward(q, k, v, o, do, lse, causal=causal, block_mask=mask, scale=scale, workspace=ws,
-                        dq=dq, dk=dk, dv=dv)
-            ho.copy_(o, non_blocking=True); hl.copy_(lse, non_blocking=True)
-            hdq.copy_(dq, non_blocking=True); hdk.copy_(dk, non_blocking=True); hdv.copy_(dv, non_blocking=True)
+        def e2e_step(i):
+            b = i % 2
+            xq, xk, xv, xdo = din[b]
+            xo, xdq, xdk, xdv, xl = dout[b]
+            with torch.cuda.stream(s_in):
+                if issued[b]:
+                    s_in.wait_event(ev_c[b])  # the compute two steps back has read these inputs
+                for dst, src in zip(din[b], hin):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[b].record(s_in)
+            with torch.cuda.stream(s_c):
+                s_c.wait_event(ev_in[b])
+                if issued[b]:
+                    s_c.wait_event(ev_out[b])  # the results two steps back have left
+                fa.forward(xq, xk, xv, causal=causal, block_mask=mask, scale=scale, out=xo, lse=xl)
+                fa.backward(xq, xk, xv, xo, xdo, xl, causal=causal, block_mask=mask, scale=scale, workspace=ws,
+                            dq=xdq, dk=xdk, dv=xdv)
+                ev_c[b].record(s_c)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_c[b])
+                for dst, src in zip(hout, (xo, xdq, xdk, xdv, xl)):
+                    dst.copy_(src, non_blocking=True)
+                ev_out[b].record(s_out)
+            issued[b] = True
 
-        for _ in range(2):
-            e2e_step()
+        for i in range(4):
+            e2e_step(i)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if dist_on:
             torch.distributed.barrier()
-        e0.record()
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record()
         torch.cuda.synchronize()
+        e0.record(s_in)
+        for i in range(args.steps):
+            e2e_step(i)
+        s_out.wait_stream(s_in)
+        s_out.wait_stream(s_c)
+        e1.record(s_out)
+        torch.cuda.synchronize()
+        if fa.last_device_status(dev) != 0:
+            raise RuntimeError("device wait timed out in the end-to-end loop")
         e2e_ms = reduce_max(e0.elapsed_time(e1), dist_on, dev) / args.steps
         nb = B * H * N * d * 2
         e2e = {"value": world * 3.5 * f_fwd / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": 4 * nb, "d2h_bytes_per_step": 4 * nb + B * H * N * 4,
-               "ms_per_step": e2e_ms}
+               "ms_per_step": e2e_ms,
+               "pipeline": "3 streams (copy in, compute, copy out), 2 device buffer sets, pinned host memory"}
 
     # ---- roofline of the dominant kernel (bwd main: 5 of the 7 matmuls of a step)
     main_flops = 2.5 * f_fwd
