@@ -38,6 +38,9 @@
 #include "kernels.h"
 #include "ptx.cuh"
 
+#ifndef FA_FWD_SOLO_MAX_NB
+#define FA_FWD_SOLO_MAX_NB 8
+#endif
 #ifndef FA_FWD_EXP_EMU_MASK
 #define FA_FWD_EXP_EMU_MASK 0x0u
 #endif
@@ -819,7 +822,15 @@ __global__ void __launch_bounds__(384, 1)
 
 bool fwd_one_tile(int D, int nb) { return D == 256 || nb == 1; }
 
-int fwd_tiles_per_cta(int D, int nb) { return fwd_one_tile(D, nb) ? 1 : 2; }
+// Short sequences (few query tiles per head) run one query tile per CTA, two CTAs per SM
+// (fa_fwd_solo.cu), so that one CTA's prologue and epilogue overlap the other's KV steps.
+bool fwd_solo(int D, int nb) { return !fwd_one_tile(D, nb) && nb <= FA_FWD_SOLO_MAX_NB; }
+
+int fwd_tiles_per_cta(int D, int nb) { return (fwd_one_tile(D, nb) || fwd_solo(D, nb)) ? 1 : 2; }
+
+template <int D, bool F16>
+cudaError_t launch_fwd_solo(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& to, const FwdParams& p, long long BH, cudaStream_t stream);
 
 template <int D, bool F16, bool ONE>
 static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -837,6 +848,9 @@ template <bool F16>
 static cudaError_t launch_fwd_dtype(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                     const CUtensorMap& to, const FwdParams& p, long long BH, cudaStream_t stream) {
   if (D == 256) return launch_fwd_t<256, F16, true>(tq, tk, tv, to, p, BH, stream);
+  if (fwd_solo(D, p.nb))
+    return D == 64 ? launch_fwd_solo<64, F16>(tq, tk, tv, to, p, BH, stream)
+                   : launch_fwd_solo<128, F16>(tq, tk, tv, to, p, BH, stream);
   const bool one = fwd_one_tile(D, p.nb);
   if (D == 64)
     return one ? launch_fwd_t<64, F16, true>(tq, tk, tv, to, p, BH, stream)

@@ -2,6 +2,7 @@
 // (defined in api.cu), so they are compiled together instead of with relocatable device code.
 #include "api.cu"
 #include "fa_fwd.cu"
+#include "fa_fwd_solo.cu"
 #include "fa_fwd_merge.cu"
 #include "fa_bwd.cu"
 #include "fa_bwd_aux.cu"

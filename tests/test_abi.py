@@ -166,8 +166,9 @@ def test_decode_argument_checks_and_workspace(lib):
 def test_decode_piece_choice(lib):
     """The library's piece count (num_splits = 0): enough (b, h, CTA) units for about three
     quarters of a 148-SM wave, at least two 128-key tiles per piece. A CTA holds one query tile
-    when there is only one (N_q <= 128) or d = 256, else two. (Without a GPU the SM count falls
-    back to 148, the B200's.)"""
+    when there is only one (N_q <= 128), when d = 256, or when there are at most eight
+    (N_q <= 1024: two such CTAs share an SM), else two. (Without a GPU the SM count falls back to
+    148, the B200's.)"""
     lib.fa_fwd_decode_workspace_bytes.restype = ctypes.c_size_t
     ws = lib.fa_fwd_decode_workspace_bytes
 
@@ -185,9 +186,11 @@ def test_decode_piece_choice(lib):
     assert pieces(1, 1, 1, 16384, 128) == 64                    # 111 wanted, capped at 128 key tiles / 2
     assert pieces(1, 1, 1, 65536, 128) == target                # 512 key tiles: 111 pieces
     assert pieces(1, 1, 1, 1024, 128) == 4                      # capped: 8 key tiles / 2
-    # N_q = 200 is two query tiles: one CTA per head at d = 128, two at d = 256
-    assert pieces(4, 16, 200, 16384, 128) == 2
+    # N_q = 200 is two query tiles, one per CTA: 128 CTAs already
+    assert pieces(4, 16, 200, 16384, 128) == 1
     assert pieces(4, 16, 200, 16384, 256) == 1
+    # N_q = 2000 is 16 query tiles, two per CTA: 8 CTAs per head, 32 for 4 heads
+    assert pieces(1, 4, 2000, 16384, 128) == -(-target // 32)
 
 
 def test_backward_checks_every_stage_before_launching(lib):
