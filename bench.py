@@ -203,6 +203,17 @@ def run_reference(args, wl, rank, world):
     return 0
 
 
+def fwd_kernel_name(d: int, nq: int) -> str:
+    """The forward kernel the library launches for nq query rows at head dimension d (a label
+    for the roofline object; the choice itself is made in the library)."""
+    nb = -(-nq // 128)
+    if d == 256 or (d == 128 and nb == 1):
+        return "fa_fwd_kernel (one tile per CTA)"
+    if nb <= 8:
+        return "fa_fwd_solo_kernel" + (" (query rows copied per lane quarter)" if d == 64 and nq <= 64 else "")
+    return "fa_fwd_kernel"
+
+
 # ----------------------------------------------------------------------------- decode arm
 def run_decode(args, rank, world, local_rank, dist_on):
     """Decode-shaped forward: args.decode queries per head against --seqlen keys, B=8, H=16
@@ -250,7 +261,7 @@ def run_decode(args, rank, world, local_rank, dist_on):
                        "workspace_bytes": need},
             "tflops": world * fwd_flops(B, H, 1, d) * nq * nk / (ms * 1e-3) / 1e12,
             "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / world / peaks["hbm_gbs"], "traffic": None, "kernel": "fa_fwd_kernel"},
+                         "frac": gbs / world / peaks["hbm_gbs"], "traffic": None, "kernel": fwd_kernel_name(d, nq)},
             "gpu_launches": args.steps * (2 if need > 0 else 1), "clocks": clk.summary()}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -297,7 +308,7 @@ def run_forward_only(args, wl, rank, world, local_rank, dist_on):
             "config": {"workload": wl["name"] + ", forward only", "B": B, "H": H, "N": N, "d": d,
                        "causal": causal},
             "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": tflops / peaks["bf16_tflops"], "traffic": None, "kernel": "fa_fwd_kernel"},
+                         "frac": tflops / peaks["bf16_tflops"], "traffic": None, "kernel": fwd_kernel_name(d, N)},
             "gpu_launches": args.steps, "clocks": clk.summary()}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -26,11 +26,12 @@ bool get_encoder() {
   return g_encode != nullptr;
 }
 
-// [BH][N][D] bf16 (or fp16) viewed as a 3-D tensor {D, N, BH}; box 64 x 128 x 1, 128-byte swizzle.
-bool encode_bhnd(CUtensorMap* map, const void* base, long long BH, int N, int D, int f16) {
+// [BH][N][D] bf16 (or fp16) viewed as a 3-D tensor {D, N, BH}; box 64 x rows x 1 (rows = 128,
+// or 128 / k for a query tile loaded as k copies of its first 128 / k rows), 128-byte swizzle.
+bool encode_bhnd(CUtensorMap* map, const void* base, long long BH, int N, int D, int f16, int rows = 128) {
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   const CUtensorMapDataType dt = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUresult r = g_encode(map, dt, 3, const_cast<void*>(base), dims, strides, box,
@@ -128,7 +129,7 @@ fa_status fa_fwd_ex(int dtype, const void* q, const void* k, const void* v, void
   if (!get_encoder()) return FA_ERR_CUDA;
   const long long BH = (long long)B * H;
   alignas(64) CUtensorMap tq, tk, tv, to;
-  if (!encode_bhnd(&tq, q, BH, N, d, f16) || !encode_bhnd(&tk, k, BH, N, d, f16) ||
+  if (!encode_bhnd(&tq, q, BH, N, d, f16, 128 / fa::fwd_rep(d, N)) || !encode_bhnd(&tk, k, BH, N, d, f16) ||
       !encode_bhnd(&tv, v, BH, N, d, f16) || !encode_bhnd(&to, o, BH, N, d, f16))
     return FA_ERR_CUDA;
   fa::FwdParams p;
@@ -235,7 +236,7 @@ fa_status fa_fwd_decode(int dtype, const void* q, const void* k, const void* v, 
   if (ns > 1 && (!workspace || !aligned16(workspace) || workspace_bytes < w.bytes)) return FA_ERR_WORKSPACE;
   if (!get_encoder()) return FA_ERR_CUDA;
   alignas(64) CUtensorMap tq, tk, tv, to;
-  if (!encode_bhnd(&tq, q, BH, Nq, d, f16) || !encode_bhnd(&tk, k, BH, Nk, d, f16) ||
+  if (!encode_bhnd(&tq, q, BH, Nq, d, f16, 128 / fa::fwd_rep(d, Nq)) || !encode_bhnd(&tk, k, BH, Nk, d, f16) ||
       !encode_bhnd(&tv, v, BH, Nk, d, f16) || !encode_bhnd(&to, o, BH, Nq, d, f16))
     return FA_ERR_CUDA;
   fa::FwdParams p;

@@ -820,7 +820,10 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-bool fwd_one_tile(int D, int nb) { return D == 256 || nb == 1; }
+// The one-tile kernel (one CTA per SM) runs d = 256, and a single query tile (decode) at d = 128;
+// a single tile at d = 64 goes to the two-CTAs-per-SM kernel below, whose second CTA hides
+// the first one's chain (decode at Nq <= 128, 16384 keys: K/V read 3.3 -> 3.8 TB/s).
+bool fwd_one_tile(int D, int nb) { return D == 256 || (nb == 1 && D == 128); }
 
 // Short sequences (few query tiles per head) run one query tile per CTA, two CTAs per SM
 // (fa_fwd_solo.cu), so that one CTA's prologue and epilogue overlap the other's KV steps.
@@ -828,7 +831,12 @@ bool fwd_solo(int D, int nb) { return !fwd_one_tile(D, nb) && nb <= FA_FWD_SOLO_
 
 int fwd_tiles_per_cta(int D, int nb) { return (fwd_one_tile(D, nb) || fwd_solo(D, nb)) ? 1 : 2; }
 
-template <int D, bool F16>
+// At most 32 (64) query rows and d = 64 (decode): the tile's lane quarters hold four (two)
+// copies of those rows and split each KV step's keys between them, so the softmax warps share
+// the step's exponentials instead of the quarters holding the real rows doing them all.
+int fwd_rep(int D, int Nq) { return D != 64 ? 1 : Nq <= 32 ? 4 : Nq <= 64 ? 2 : 1; }
+
+template <int D, bool F16, int REP>
 cudaError_t launch_fwd_solo(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& to, const FwdParams& p, long long BH, cudaStream_t stream);
 
@@ -849,8 +857,10 @@ static cudaError_t launch_fwd_dtype(int D, const CUtensorMap& tq, const CUtensor
                                     const CUtensorMap& to, const FwdParams& p, long long BH, cudaStream_t stream) {
   if (D == 256) return launch_fwd_t<256, F16, true>(tq, tk, tv, to, p, BH, stream);
   if (fwd_solo(D, p.nb))
-    return D == 64 ? launch_fwd_solo<64, F16>(tq, tk, tv, to, p, BH, stream)
-                   : launch_fwd_solo<128, F16>(tq, tk, tv, to, p, BH, stream);
+    return D == 128                 ? launch_fwd_solo<128, F16, 1>(tq, tk, tv, to, p, BH, stream)
+           : fwd_rep(D, p.N) == 4 ? launch_fwd_solo<64, F16, 4>(tq, tk, tv, to, p, BH, stream)
+           : fwd_rep(D, p.N) == 2 ? launch_fwd_solo<64, F16, 2>(tq, tk, tv, to, p, BH, stream)
+                                  : launch_fwd_solo<64, F16, 1>(tq, tk, tv, to, p, BH, stream);
   const bool one = fwd_one_tile(D, p.nb);
   if (D == 64)
     return one ? launch_fwd_t<64, F16, true>(tq, tk, tv, to, p, BH, stream)

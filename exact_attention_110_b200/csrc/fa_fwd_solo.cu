@@ -11,6 +11,12 @@
 // CTAs are resident per SM: the tensor core and the special-function unit interleave the two
 // CTAs' chains (the ping-pong of the two-tile kernel, across CTAs) and one CTA's prologue and
 // epilogue overlap the other's KV steps.
+// Decode form (REP = 4 or 2: d = 64, at most 32 or 64 query rows): a tile with one real row
+// still costs a whole 128-row softmax per KV step, all of it in the warp that holds the row.
+// Here the query tile is loaded as REP copies of its first 128 / REP rows (four copies: one
+// per TMEM lane quarter), and copy c scores only keys (128 / REP) c .. of each step (P of the
+// row's other keys is zero in its lanes), so the warps share the exponentials; the copies' O
+// are combined at the end like the partial results of a key-range split (LSE-weighted).
 // Roles (192 threads, so two CTAs keep 168 registers per thread): warps 0-3 the softmax
 // (thread = row = TMEM lane), warp 4 the TMA producer, warp 5 the MMA issuer (one thread),
 // which also allocates and frees the tensor memory.
@@ -37,7 +43,7 @@ struct FwdSoloCfg {
   static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
 };
 
-template <int D, bool F16>
+template <int D, bool F16, int REP>
 __global__ void __launch_bounds__(192, 2)
     fa_fwd_solo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -115,7 +121,9 @@ __global__ void __launch_bounds__(192, 2)
       tma_prefetch_desc(&tmO);
       mbar_arrive_expect_tx(bar_q, C::TILE_BYTES);
       for (int pn = 0; pn < C::PANELS; ++pn)
-        tma_load_3d(smem + C::OFF_Q + pn * C::PANEL_BYTES, &tmQ, bar_q, pn * 64, qb * 128, bh);
+        for (int w = 0; w < REP; ++w)  // REP copies of the tile's first 128 / REP rows (tmQ's box height)
+          tma_load_3d(smem + C::OFF_Q + pn * C::PANEL_BYTES + w * (128 / REP) * 128, &tmQ, bar_q, pn * 64, qb * 128,
+                      bh);
       int it = 0;
       int issued_k[NS], issued_v[NS];
       for (int s = 0; s < NS; ++s) issued_k[s] = issued_v[s] = -1;
@@ -213,7 +221,13 @@ __global__ void __launch_bounds__(192, 2)
   } else {
     // ------------------------------------------------------------------ softmax warpgroup
     const uint32_t wq = warp & 3;  // TMEM lane quarter this warp may touch
-    const int r = wq * 32 + lane;  // row inside the tile
+    // The tile's lanes hold REP copies of its first 128 / REP rows (REP = 1: all 128 rows, thread
+    // = row). Copy cp = wq / QPR scores keys W cp .. W cp + W - 1 of each step; the copies'
+    // partial softmaxes are combined in the epilogue.
+    constexpr int W = 128 / REP;   // keys of a step this warp scores
+    constexpr int QPR = 4 / REP;   // lane quarters per copy
+    const int r = (int)((wq % QPR) * 32 + lane);  // row inside the tile
+    const int c0 = (int)(wq / QPR) * W;          // first of this warp's keys in a step
     const uint32_t lane_off = (wq * 32u) << 16;
     const uint32_t tS_row = tmem + lane_off;
     const uint32_t tO_row = tmem + lane_off + 128u;
@@ -231,26 +245,44 @@ __global__ void __launch_bounds__(192, 2)
       if (!ok) break;
       s_phase ^= 1u;
       tc_fence_after();
-      uint32_t su[128];
-      tmem_ld128(tS_row, su);
+      uint32_t su[W];
+      if constexpr (REP == 1)
+        tmem_ld128(tS_row, su);
+      else if constexpr (REP == 2)
+        tmem_ld64(tS_row + c0, su);
+      else
+        tmem_ld32(tS_row + c0, su);
       // causal band and the keys >= Nk of a partial last key tile, as in the two-tile kernel
       const bool diag = tt.causal && (128 * j + 127 > 128 * qb + tt.causal_off);
       const bool masked = diag || (128 * j + 128 > tt.Nk);
       if (masked) {
-        const int lim_c = min(diag ? 128 * (qb - j) + r + tt.causal_off + 1 : 128, tt.Nk - 128 * j);
+        const int lim_c = min(diag ? 128 * (qb - j) + r + tt.causal_off + 1 - c0 : W, tt.Nk - 128 * j - c0);
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < W; ++c)
           if (c >= lim_c) su[c] = 0xff800000u;  // -inf
       }
-      float mc[8];
+      float mx;
+      if constexpr (REP == 1) {
+        float mc[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        float m = fmax3(__uint_as_float(su[k]), __uint_as_float(su[k + 8]), __uint_as_float(su[k + 16]));
+        for (int k = 0; k < 8; ++k) {
+          float m = fmax3(__uint_as_float(su[k]), __uint_as_float(su[k + 8]), __uint_as_float(su[k + 16]));
 #pragma unroll
-        for (int c = 24; c < 120; c += 16) m = fmax3(m, __uint_as_float(su[c + k]), __uint_as_float(su[c + 8 + k]));
-        mc[k] = fmaxf(m, __uint_as_float(su[120 + k]));
+          for (int c = 24; c < 120; c += 16) m = fmax3(m, __uint_as_float(su[c + k]), __uint_as_float(su[c + 8 + k]));
+          mc[k] = fmaxf(m, __uint_as_float(su[120 + k]));
+        }
+        mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
+      } else {
+        float mc[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {  // four chains over k, k + 4, ..., k + W - 4
+          float m = __uint_as_float(su[k]);
+#pragma unroll
+          for (int c = 4; c + 4 < W; c += 8) m = fmax3(m, __uint_as_float(su[c + k]), __uint_as_float(su[c + 4 + k]));
+          mc[k] = fmaxf(m, __uint_as_float(su[W - 4 + k]));
+        }
+        mx = fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
       }
-      const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
       const float cand = mx * sl2;
       float alpha = 1.f;
       if (cand > m_ref + 8.f) {  // also taken on the first visible tile (m_ref = -inf)
@@ -271,7 +303,44 @@ __global__ void __launch_bounds__(192, 2)
       l *= alpha;
       const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
       const uint64_t sl2_2 = f2_pack(sl2, sl2), mneg_2 = f2_pack(mneg, mneg);
-      l += softmax_exp_store<F16, false, 0u>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[0]);
+      if constexpr (REP == 1) {
+        l += softmax_exp_store<F16, false, 0u>(su, sl2_2, mneg_2, tS_row, ek, &bar_p[0]);
+      } else {
+        // P of this warp's W keys in packed columns c0 / 2 ..; the row's other keys belong to
+        // the other copies, so their P columns are zero in this lane quarter.
+        uint64_t ls2[2] = {0ull, 0ull};
+#pragma unroll
+        for (int c = 0; c < W / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint64_t s2 = f2_pack(__uint_as_float(su[32 * c + 2 * i]), __uint_as_float(su[32 * c + 2 * i + 1]));
+            const uint64_t x2 = ffma2(s2, sl2_2, mneg_2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            const uint64_t p2 = f2_pack(ex2(x0), ex2(x1));
+            ls2[i & 1] = fadd2(ls2[i & 1], p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            pk[i] = pack16<F16>(p0, p1);
+          }
+          tmem_st16(tS_row + c0 / 2 + 16 * c, pk);
+        }
+        uint32_t zero[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) zero[i] = 0u;
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          if (g < c0 / 32 || g >= c0 / 32 + W / 32) tmem_st16(tS_row + 16 * g, zero);
+        const uint64_t t2 = fadd2(ls2[0], ls2[1]);
+        float a, b;
+        f2_unpack(t2, a, b);
+        l += a + b;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_p[0]);
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -282,36 +351,73 @@ __global__ void __launch_bounds__(192, 2)
     // ---------------------------------------------------------------- epilogue
     if (ok) ok = warp_wait(bar_o, 0, ab, lim, WAIT_FWD_EPILOGUE + 1);
     uint8_t* stage = smem + C::OFF_Q;  // Q is no longer read
-    if (ok) {
-      tc_fence_after();
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const uint32_t sstage = smem_u32(stage);
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t u[32];
-        if (o_started) {
-          tmem_ld32(tO_row + c * 32, u);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = 0u;
+    if constexpr (REP == 1) {
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const uint32_t sstage = smem_u32(stage);
+  #pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t u[32];
+          if (o_started) {
+            tmem_ld32(tO_row + c * 32, u);
+          } else {
+  #pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = 0u;
+          }
+          uint32_t w[16];
+  #pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack16<F16>(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
+          const int col0 = c * 32;
+          const uint32_t panel = sstage + (col0 >> 6) * C::PANEL_BYTES;
+          const uint32_t chunk0 = (col0 & 63) >> 3;
+  #pragma unroll
+          for (int q = 0; q < 4; ++q)
+            st_shared_v4(panel + sw128_offset(r, chunk0 + q), w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         }
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          w[i] = pack16<F16>(__uint_as_float(u[2 * i]) * inv_l, __uint_as_float(u[2 * i + 1]) * inv_l);
-        const int col0 = c * 32;
-        const uint32_t panel = sstage + (col0 >> 6) * C::PANEL_BYTES;
-        const uint32_t chunk0 = (col0 & 63) >> 3;
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          st_shared_v4(panel + sw128_offset(r, chunk0 + q), w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        fence_proxy_async_smem();
+        const int row = qb * 128 + r;
+        const float lse_row = (l > 0.f) ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (p.nsplit > 1) {
+          const size_t prow = ((size_t)bh * p.nsplit + split) * p.Np + row;
+          float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D);
+  #pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t u[32];
+            if (o_started) {
+              tmem_ld32(tO_row + c * 32, u);
+            } else {
+  #pragma unroll
+              for (int i = 0; i < 32; ++i) u[i] = 0u;
+            }
+  #pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[c * 8 + q] = make_float4(__uint_as_float(u[4 * q]) * inv_l, __uint_as_float(u[4 * q + 1]) * inv_l,
+                                           __uint_as_float(u[4 * q + 2]) * inv_l, __uint_as_float(u[4 * q + 3]) * inv_l);
+          }
+          p.lse_part[prow] = lse_row;
+        } else if (row < p.N) {
+          p.lse[(size_t)bh * p.N + row] = lse_row;
+        }
       }
-      fence_proxy_async_smem();
-      const int row = qb * 128 + r;
-      const float lse_row = (l > 0.f) ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-      if (p.nsplit > 1) {
-        const size_t prow = ((size_t)bh * p.nsplit + split) * p.Np + row;
-        float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D);
+    } else {
+      // Combine the copies' partial softmaxes of each row i < 128 / REP (the same split-and-merge
+      // rule as the key-range pieces): M = max_w m_w, L = sum_w 2^(m_w - M) l_w,
+      // O = sum_w 2^(m_w - M) O_w / L, LSE = (M + log2 L) ln 2. The K/V ring is free once every
+      // MMA has completed; it holds the copies' m, l and unnormalised O rows, entry
+      // w * 128 / REP + i for copy w of row i (= the lane's TMEM row wq * 32 + lane).
+      constexpr int OS = D + 4;  // padded row stride (floats) of the O scratch
+      static_assert((2 * 128 + 128 * OS) * 4 <= 2 * C::NS * C::TILE_BYTES, "combine scratch fits the K/V ring");
+      constexpr int RPC = 128 / REP;  // rows per copy
+      float* cm = reinterpret_cast<float*>(smem + C::OFF_K);  // [REP][RPC]
+      float* cl = cm + 128;                                   // [REP][RPC]
+      float* co = cl + 128;                                   // [REP][RPC][OS]
+      if (ok) {
+        tc_fence_after();
+        cm[wq * 32 + lane] = m_ref;
+        cl[wq * 32 + lane] = l;
+        float4* orow = reinterpret_cast<float4*>(co + (wq * 32 + lane) * OS);  // copy wq / QPR, row r
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t u[32];
@@ -323,12 +429,68 @@ __global__ void __launch_bounds__(192, 2)
           }
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            dst[c * 8 + q] = make_float4(__uint_as_float(u[4 * q]) * inv_l, __uint_as_float(u[4 * q + 1]) * inv_l,
-                                         __uint_as_float(u[4 * q + 2]) * inv_l, __uint_as_float(u[4 * q + 3]) * inv_l);
+            orow[c * 8 + q] = make_float4(__uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
+                                          __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3]));
         }
-        p.lse_part[prow] = lse_row;
-      } else if (row < p.N) {
-        p.lse[(size_t)bh * p.N + row] = lse_row;
+      }
+      named_bar_sync(1, 128);  // every copy's partial rows are in shared memory
+      if (ok) {
+        // REP threads per row, each on D / REP of its columns
+        const int i = (int)threadIdx.x / REP, part = (int)threadIdx.x % REP;
+        constexpr int CW = D / REP;
+        const int col0 = part * CW;
+        float f[REP], M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < REP; ++w) M = fmaxf(M, cm[w * RPC + i]);
+        float L = 0.f;
+#pragma unroll
+        for (int w = 0; w < REP; ++w) {
+          const float mw = cm[w * RPC + i];
+          f[w] = (mw == -INFINITY) ? 0.f : ex2(mw - M);
+          L += f[w] * cl[w * RPC + i];
+        }
+        const float inv_L = (L > 0.f) ? 1.f / L : 0.f;
+#pragma unroll
+        for (int w = 0; w < REP; ++w) f[w] *= inv_L;
+        float o[CW];
+#pragma unroll
+        for (int c = 0; c < CW; c += 4) {
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int w = 0; w < REP; ++w) {
+            const float4 v4 = *reinterpret_cast<const float4*>(co + (w * RPC + i) * OS + col0 + c);
+            acc.x += f[w] * v4.x;
+            acc.y += f[w] * v4.y;
+            acc.z += f[w] * v4.z;
+            acc.w += f[w] * v4.w;
+          }
+          o[c] = acc.x;
+          o[c + 1] = acc.y;
+          o[c + 2] = acc.z;
+          o[c + 3] = acc.w;
+        }
+        const int row = qb * 128 + i;
+        const float lse_row = (L > 0.f) ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+        if (p.nsplit > 1) {
+          const size_t prow = ((size_t)bh * p.nsplit + split) * p.Np + row;
+          float4* dst = reinterpret_cast<float4*>(p.o_part + prow * D + col0);
+#pragma unroll
+          for (int c = 0; c < CW / 4; ++c) dst[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+          if (part == 0) p.lse_part[prow] = lse_row;
+        } else {
+          const uint32_t sstage = smem_u32(stage);
+#pragma unroll
+          for (int k = 0; k < CW / 8; ++k) {
+            const int col = col0 + 8 * k;
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) w4[e] = pack16<F16>(o[8 * k + 2 * e], o[8 * k + 2 * e + 1]);
+            st_shared_v4(sstage + (col >> 6) * C::PANEL_BYTES + sw128_offset(i, (col & 63) >> 3), w4[0], w4[1], w4[2],
+                         w4[3]);
+          }
+          fence_proxy_async_smem();
+          if (part == 0 && row < p.N) p.lse[(size_t)bh * p.N + row] = lse_row;
+        }
       }
     }
     named_bar_sync(1, 128);  // the whole output tile is staged
@@ -348,15 +510,15 @@ __global__ void __launch_bounds__(192, 2)
   }
 }
 
-template <int D, bool F16>
+template <int D, bool F16, int REP>
 cudaError_t launch_fwd_solo(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& to, const FwdParams& p, long long BH, cudaStream_t stream) {
   using C = FwdSoloCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(fa_fwd_solo_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(fa_fwd_solo_kernel<D, F16, REP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const dim3 grid = grid_work(p.nb * p.nsplit, BH, p.order_group);
-  fa_fwd_solo_kernel<D, F16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
+  fa_fwd_solo_kernel<D, F16, REP><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError();
 }
 

@@ -160,6 +160,10 @@ cudaError_t launch_fwd_merge(const FwdMergeParams& p, cudaStream_t stream);
 // and the tiles per CTA that follow (1 or 2).
 bool fwd_one_tile(int D, int nb);
 int fwd_tiles_per_cta(int D, int nb);
+// Copies of the query rows per 128-row tile (at d = 64: 4 for at most 32 rows, 2 for at most
+// 64, each copy scoring its share of every KV step's keys; else 1); the Q tensor map's box is
+// 128 / that many rows high.
+int fwd_rep(int D, int Nq);
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,

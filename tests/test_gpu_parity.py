@@ -68,6 +68,13 @@ SMALL = [
     # a single query tile runs the one-tile kernel (S double-buffered, columns split)
     (1, 2, 100, 128, True, None),
     (2, 1, 128, 128, False, "bernoulli"),
+    # at most 32 (64) rows at d = 64: four (two) copies of the rows, each scoring its share of
+    # every step's keys, combined at the end; just past that, the per-row form of the same kernel
+    (1, 3, 32, 64, True, None),
+    (2, 1, 20, 64, False, "ones"),
+    (2, 1, 33, 64, False, None),
+    (1, 2, 64, 64, True, None),
+    (1, 1, 65, 64, True, None),
 ]
 
 
@@ -193,6 +200,12 @@ DECODE = [
     (1, 3, 8, 3000, 64, False, 5, "f16"),
     (1, 2, 40, 900, 256, True, 0, "bf16"),      # head dim 256
     (2, 2, 4, 5000, 128, True, 0, "f16"),       # fp16, bottom-right causal, library's split
+    (2, 3, 32, 16384, 64, False, 0, "bf16"),    # 32 queries at d = 64: four row copies, library's split
+    (1, 2, 5, 3, 64, True, 0, "bf16"),          # fewer keys than queries: rows 0-1 see no key
+    (3, 1, 1, 130, 64, False, 0, "bf16"),       # one query, a ragged second key tile
+    (1, 2, 33, 700, 64, True, 0, "f16"),        # 33 queries: two copies of 64 rows
+    (2, 2, 64, 16384, 64, True, 0, "bf16"),     # 64 queries, bottom-right causal, library's split
+    (1, 3, 40, 1000, 64, False, 3, "bf16"),     # two copies, three key-range pieces
 ]
 
 
