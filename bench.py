@@ -172,7 +172,7 @@ def oracle_sample(wl, nheads: int, seed: int, dtype: str = "bf16"):
     return flops, dt, oracle.num_threads()
 
 
-def heads_for_seconds(wl, target_s: float, rate_gflops: float = 20.0) -> int:
+def heads_for_seconds(wl, target_s: float, rate_gflops: float = 50.0) -> int:
     per_head = 3.5 * fwd_flops(1, 1, wl["N"], wl["d"], wl["causal"],
                                wl.get("p_on", 0.25) + 0.03 if wl["block_sparse"] else 1.0)
     return max(1, min(wl["B"] * wl["H"], int(target_s * rate_gflops * 1e9 / per_head)))
@@ -612,7 +612,9 @@ def run_gpu(args, wl, rank, world, local_rank, dist_on):
                                      "per-GPU figures on this rank",
                          "points": points, "configs": named, "clocks": sclk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        nh = heads_for_seconds(wl, 12.0)
+        # one head first to measure this host's rate, then enough heads for ~12 s of oracle work
+        f1, t1, _ = oracle_sample(wl, 1, 2999, args.dtype)
+        nh = max(1, min(B * H, int(12.0 / max(t1, 1e-3))))
         f, t, cores = oracle_sample(wl, nh, 3000, args.dtype)
         line["cpu_baseline"] = {"value": f / t / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": f"{nh} whole head(s) of {N}x{d} (fwd+bwd, fp64) of {B * H} heads; "
