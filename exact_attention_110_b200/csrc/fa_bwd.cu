@@ -779,7 +779,7 @@ __global__ void __launch_bounds__(512, 1)
       }
       ++it;
     }
-    if (issuer) bulk_wait_group0();  // every reduction complete before the CTA exits
+    // The last reductions complete while dK is written (its staging area is not a dQ slot).
     // -------------------------------------------------------------- epilogue: dK (dS carries the scale)
     if (ok) ok = warp_wait(bar_acc, 0, ab, lim, WAIT_BWD_EPILOGUE + 2);
     // dO ring stage 0 (SPLIT: panel slots 2-3), free once every MMA retired
@@ -796,6 +796,7 @@ __global__ void __launch_bounds__(512, 1)
       bulk_commit_group();
       bulk_wait_group_read0();
     }
+    if (issuer) bulk_wait_group0();  // every dQ reduction and the dK store complete before the CTA exits
   }
 
   tc_fence_before();

@@ -51,9 +51,10 @@
 
 namespace fa {
 
-// ONE: one query tile per CTA (see TILES). Chosen at launch: always at d = 256, and for a
-// problem with a single query tile (N_q <= 128, e.g. decoding), where the two-tile form would
-// leave its second tile empty; two ping-ponged tiles otherwise.
+// ONE: one query tile per CTA (see TILES). Chosen at launch: always at d = 256, and at d = 128
+// for a problem with a single query tile (N_q <= 128, e.g. decoding), where the two-tile form
+// would leave its second tile empty; two ping-ponged tiles otherwise (short sequences and d = 64
+// single tiles run the kernel of fa_fwd_solo.cu instead).
 template <int D, bool ONE>
 struct FwdCfg {
   static constexpr int THREADS = 384;  // warp 0 TMA, warp 1 MMA, warps 4-11 softmax
@@ -822,7 +823,8 @@ __global__ void __launch_bounds__(384, 1)
 
 // The one-tile kernel (one CTA per SM) runs d = 256, and a single query tile (decode) at d = 128;
 // a single tile at d = 64 goes to the two-CTAs-per-SM kernel below, whose second CTA hides
-// the first one's chain (decode at Nq <= 128, 16384 keys: K/V read 3.3 -> 3.8 TB/s).
+// the first one's chain (decode at Nq = 128, 16384 keys: K/V read 3.3 -> 3.7 TB/s; fewer rows
+// also copy them across the lane quarters, fwd_rep).
 bool fwd_one_tile(int D, int nb) { return D == 256 || (nb == 1 && D == 128); }
 
 // Short sequences (few query tiles per head) run one query tile per CTA, two CTAs per SM
