@@ -382,6 +382,12 @@ fa_status plan_bwd_main(int dtype, const void* q, const void* k, const void* v, 
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
   p.f16 = f16;
+  // Persistent CTAs (each walks several (head, key tile) items, the next item's loads overlapping
+  // the previous one's epilogue) pay off when an item is short: at most 8 query tiles per key
+  // tile, no causal mask (whose longest-first order the hardware block scheduler balances
+  // better than a static assignment). Measured: N = 512 +6-7%, N = 1024 d = 64 +3%; from 16
+  // query tiles on and on causal grids they lose (-5% to -19%); block masks make items unequal too.
+  p.persist = (sh.d != 256 && !causal && block_mask == nullptr && p.nb <= 8) ? 1 : 0;
   m->BH = BH;
   m->d = sh.d;
   return FA_OK;

@@ -39,6 +39,10 @@
 //    the dQ drain); dP_{i+1}.
 //  * TMEM: S^T/P^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D); dQ: d = 128
 //    reuses the dP^T columns once dP^T has been read, d = 64 has its own [384,448).
+//  * PERSIST: one CTA per SM walks several (b, h, key tile) items (cta_item); ring counters and
+//    barrier phases run on across items, the next item's loads overlap the previous item's
+//    epilogue, and three more barriers (dV / dK read out of TMEM, dV store done reading its
+//    staging buffer) keep the next item's first dV / dK MMAs and dS writes behind it.
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -90,7 +94,7 @@ struct BwdCfg {
   static constexpr int OFF_DEL = OFF_LSE + NS * 512;          // [NS][128] fp32: -D
   static constexpr int OFF_BAR = OFF_DEL + NS * 512;
   static constexpr int NQB = SPLIT ? RING : NS;               // full/empty barrier pairs of the Q ring
-  static constexpr int NBAR = 1 + 2 * NQB + 2 * NS_DO + 9;
+  static constexpr int NBAR = 1 + 2 * NQB + 2 * NS_DO + 12;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int TMEM_COLS = 512;
@@ -146,7 +150,25 @@ __device__ __forceinline__ void stage_row16(uint32_t taddr, uint32_t sstage, int
   }
 }
 
-template <int D, bool F16>
+// Work item w of this CTA (cta_item): head bh, key tile j (SPLIT: item 2j + half hh of d;
+// causal: j = 0 is the heaviest) and the first query tile whose last row sees key tile j's
+// first key. Every role walks the same items.
+template <bool SPLIT, bool PERSIST>
+__device__ __forceinline__ bool bwd_item(const BwdParams& p, int w, int& bh, int& j, int& hh, int& i_begin) {
+  int xj;
+  if (!cta_item(p.BH, p.nbk * (SPLIT ? 2 : 1), p.order_group, PERSIST ? 1 : 0, w, bh, xj)) return false;
+  j = SPLIT ? (xj >> 1) : xj;
+  hh = SPLIT ? (xj & 1) : 0;
+  const int i_first = 128 * j - 127 - p.causal_off;
+  i_begin = (p.causal && i_first > 0) ? (i_first + 127) / 128 : 0;
+  return true;
+}
+__device__ __forceinline__ BwdTiles bwd_tiles(const BwdParams& p, int bh) {
+  const uint8_t* bmask = p.block_mask == nullptr ? nullptr : p.block_mask + (size_t)bh * p.mask_stride;
+  return BwdTiles{p.nb, p.nbk, p.Nk, p.causal, p.causal_off, bmask};
+}
+
+template <int D, bool F16, bool PERSIST>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -175,20 +197,18 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bar_dsfree = bar_ds + 1;     // MMAs reading dS^T_i done
   uint64_t* bar_dq = bar_dsfree + 1;     // dQ_i ready in TMEM
   uint64_t* bar_dqfree = bar_dq + 1;     // dQ_i read out of TMEM
-  uint64_t* bar_acc = bar_dqfree + 1;    // dK, dV final (all MMAs retired)
+  uint64_t* bar_acc = bar_dqfree + 1;    // dK, dV of the item final (all its MMAs retired)
   uint64_t* bar_done = bar_acc + 1;
+  uint64_t* bar_dvfree = bar_done + 1;   // dV read out of TMEM by the epilogue (the next item may overwrite)
+  uint64_t* bar_dkfree = bar_dvfree + 1; // dK read out of TMEM by the epilogue
+  uint64_t* bar_vst = bar_dkfree + 1;    // the dV store has read its staging area (the dS buffer)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   AbortState* ab = reinterpret_cast<AbortState*>(smem + C::OFF_MISC + 4);
 
-  int bh, xj;  // head and work item: key tile j (SPLIT: 2j + half of d); causal: j = 0 is the heaviest
-  if (!cta_work(p.BH, p.nbk * (C::SPLIT ? 2 : 1), p.order_group, bh, xj)) return;
-  const uint8_t* bmask = p.block_mask == nullptr ? nullptr : p.block_mask + (size_t)bh * p.mask_stride;
-  const BwdTiles tt{p.nb, p.nbk, p.Nk, p.causal, p.causal_off, bmask};
-  const int j = C::SPLIT ? (xj >> 1) : xj;
-  const int hh = C::SPLIT ? (xj & 1) : 0;
-  // causal: the first query tile whose last row sees key tile j's first key
-  const int i_first = 128 * j - 127 - p.causal_off;
-  const int i_begin = (p.causal && i_first > 0) ? (i_first + 127) / 128 : 0;
+  {
+    int bh0, j0, hh0, ib0;
+    if (!bwd_item<C::SPLIT, PERSIST>(p, 0, bh0, j0, hh0, ib0)) return;
+  }
   const uint64_t lim = p.timeout_ns;
 
   if (warp == 0 && lane == 0) {
@@ -210,6 +230,9 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(bar_dqfree, 4);
     mbar_init(bar_acc, 1);
     mbar_init(bar_done, 1);
+    mbar_init(bar_dvfree, 8);  // one arrive per P/dS warp
+    mbar_init(bar_dkfree, 4);  // one arrive per dQ-drain warp
+    mbar_init(bar_vst, 1);
     ab->flag = 0;
     fence_mbar_init();
   }
@@ -234,41 +257,57 @@ __global__ void __launch_bounds__(512, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmdO);
       if constexpr (!C::SPLIT) {
-        mbar_arrive_expect_tx(bar_kv, 2 * C::TILE_BYTES);
-        for (int pn = 0; pn < C::PANELS; ++pn) {
-          tma_load_3d(smem + C::OFF_K + pn * C::PANEL_BYTES, &tmK, bar_kv, pn * 64, j * 128, bh);
-          tma_load_3d(smem + C::OFF_V + pn * C::PANEL_BYTES, &tmV, bar_kv, pn * 64, j * 128, bh);
-        }
-        int it = 0;
+        int it = 0;  // active query tiles loaded so far, over all items (ring position)
         int issued[NS], issued_do[NS_DO];
         for (int s = 0; s < NS; ++s) issued[s] = -1;
         for (int s = 0; s < NS_DO; ++s) issued_do[s] = -1;
         bool ok = true;
-        for (int i = i_begin; i < tt.nb; ++i) {
-          if (!bwd_tile_active(tt, i, j)) continue;
-          // Q_i first: its stage frees at dK_{i-NS}, before dO_i's stage frees at dV_{i-NS_DO}.
-          const int s = it % NS;
-          const uint32_t ph = (it / NS) & 1;
-          ok = mbar_wait(&bar_qe[s], ph ^ 1, ab, lim, WAIT_BWD_LOAD + 1);
-          if (!ok) break;
-          mbar_arrive_expect_tx(&bar_qf[s], C::TILE_BYTES + 1024);
-          for (int pn = 0; pn < C::PANELS; ++pn)
-            tma_load_3d(smem + C::OFF_Q + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &bar_qf[s], pn * 64, i * 128,
-                        bh);
-          const size_t vec = (size_t)bh * p.Np + (size_t)i * 128;
-          bulk_load(smem + C::OFF_LSE + s * 512, p.lse2 + vec, 512, &bar_qf[s]);
-          bulk_load(smem + C::OFF_DEL + s * 512, p.delta + vec, 512, &bar_qf[s]);
-          issued[s] = ph;
-          const int sd = it % NS_DO;
-          const uint32_t phd = (it / NS_DO) & 1;
-          ok = mbar_wait(&bar_doe[sd], phd ^ 1, ab, lim, WAIT_BWD_LOAD + 4);
-          if (!ok) break;
-          mbar_arrive_expect_tx(&bar_dof[sd], C::TILE_BYTES);
-          for (int pn = 0; pn < C::PANELS; ++pn)
-            tma_load_3d(smem + C::OFF_DO + sd * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmdO, &bar_dof[sd], pn * 64,
-                        i * 128, bh);
-          issued_do[sd] = phd;
-          ++it;
+        int w = 0;
+        for (; ok && (PERSIST || w == 0); ++w) {
+          int bh, j, hh, i_begin;
+          if (!bwd_item<C::SPLIT, PERSIST>(p, w, bh, j, hh, i_begin)) break;
+          const BwdTiles tt = bwd_tiles(p, bh);
+          auto load_tile = [&](int i) -> bool {
+            // Q_i first: its stage frees at dK_{i-NS}, before dO_i's stage frees at dV_{i-NS_DO}.
+            const int s = it % NS;
+            const uint32_t ph = (it / NS) & 1;
+            if (!mbar_wait(&bar_qe[s], ph ^ 1, ab, lim, WAIT_BWD_LOAD + 1)) return false;
+            mbar_arrive_expect_tx(&bar_qf[s], C::TILE_BYTES + 1024);
+            for (int pn = 0; pn < C::PANELS; ++pn)
+              tma_load_3d(smem + C::OFF_Q + s * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmQ, &bar_qf[s], pn * 64,
+                          i * 128, bh);
+            const size_t vec = (size_t)bh * p.Np + (size_t)i * 128;
+            bulk_load(smem + C::OFF_LSE + s * 512, p.lse2 + vec, 512, &bar_qf[s]);
+            bulk_load(smem + C::OFF_DEL + s * 512, p.delta + vec, 512, &bar_qf[s]);
+            issued[s] = ph;
+            const int sd = it % NS_DO;
+            const uint32_t phd = (it / NS_DO) & 1;
+            if (!mbar_wait(&bar_doe[sd], phd ^ 1, ab, lim, WAIT_BWD_LOAD + 4)) return false;
+            mbar_arrive_expect_tx(&bar_dof[sd], C::TILE_BYTES);
+            for (int pn = 0; pn < C::PANELS; ++pn)
+              tma_load_3d(smem + C::OFF_DO + sd * C::TILE_BYTES + pn * C::PANEL_BYTES, &tmdO, &bar_dof[sd], pn * 64,
+                          i * 128, bh);
+            issued_do[sd] = phd;
+            ++it;
+            return true;
+          };
+          int i = i_begin;
+          while (i < tt.nb && !bwd_tile_active(tt, i, j)) ++i;
+          if (w > 0) {
+            // A later item of a persistent CTA: its first query tile enters the ring as soon as a
+            // stage is free, while the previous item still computes; K_j and V_j once no MMA
+            // reads the previous item's K and V.
+            if (i < tt.nb) ok = load_tile(i++);
+            if (ok) ok = mbar_wait(bar_acc, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_LOAD + 6);
+            if (!ok) break;
+          }
+          mbar_arrive_expect_tx(bar_kv, 2 * C::TILE_BYTES);
+          for (int pn = 0; pn < C::PANELS; ++pn) {
+            tma_load_3d(smem + C::OFF_K + pn * C::PANEL_BYTES, &tmK, bar_kv, pn * 64, j * 128, bh);
+            tma_load_3d(smem + C::OFF_V + pn * C::PANEL_BYTES, &tmV, bar_kv, pn * 64, j * 128, bh);
+          }
+          for (; ok && i < tt.nb; ++i)
+            if (bwd_tile_active(tt, i, j)) ok = load_tile(i);
         }
         AbortState none{0};
         if (!ok) {
@@ -277,7 +316,12 @@ __global__ void __launch_bounds__(512, 1)
           for (int s = 0; s < NS_DO; ++s)
             if (issued_do[s] >= 0) mbar_wait(&bar_dof[s], issued_do[s], &none, lim, WAIT_BWD_LOAD + 5);
         }
+        // K/V of the last item whose load was issued landed before the CTA can exit
+        if (w > 0) mbar_wait(bar_kv, (uint32_t)(w - 1) & 1u, &none, lim, WAIT_BWD_LOAD + 3);
       } else {
+        int bh, j, hh, i_begin;
+        bwd_item<C::SPLIT, PERSIST>(p, 0, bh, j, hh, i_begin);  // d = 256 runs one item per CTA
+        const BwdTiles tt = bwd_tiles(p, bh);
         // K_j (all four panels) stays; everything else streams through the panel ring in the
         // order the MMA issuer consumes it. First tile i0: Q(i0) panels 0-3 (S^T), then V and
         // dO(i0) panels p = 0-3 in pairs (dP^T). Then per tile i (next active tile i'):
@@ -335,9 +379,8 @@ __global__ void __launch_bounds__(512, 1)
         if (!ok)
           for (int s = 0; s < C::RING; ++s)
             if (issued[s] >= 0) mbar_wait(&bar_qf[s], issued[s], &none, lim, WAIT_BWD_LOAD + 2);
+        mbar_wait(bar_kv, 0, &none, lim, WAIT_BWD_LOAD + 3);  // K landed before the CTA can exit
       }
-      AbortState none{0};
-      mbar_wait(bar_kv, 0, &none, lim, WAIT_BWD_LOAD + 3);  // K/V landed before the CTA can exit
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -357,7 +400,7 @@ __global__ void __launch_bounds__(512, 1)
       const uint64_t dO_mn = sdesc_sw128(sdO, C::PANEL_BYTES, 1024);
       const uint64_t dS_k = sdesc_sw128(sDS, 16, 1024);              // dS^T as K-major A (dK)
       const uint64_t dS_mn = sdesc_sw128(sDS, C::PANEL_BYTES, 1024); // dS^T read MN-major (dQ)
-      bool ok = mbar_wait_spin(bar_kv, 0, ab, lim, WAIT_BWD_MMA + 1);
+      bool ok = true;
 
       if constexpr (!C::SPLIT) {
         auto issue_s = [&](int st) {
@@ -377,88 +420,119 @@ __global__ void __launch_bounds__(512, 1)
           }
         };
 
-        int i = i_begin;
-        while (i < tt.nb && !bwd_tile_active(tt, i, j)) ++i;
-        int it = 0;
-        if (ok && i < tt.nb) {
-          ok = mbar_wait_spin(&bar_qf[0], 0, ab, lim, WAIT_BWD_MMA + 2);
-          if (ok) {
-            tc_fence_after();
-            issue_s(0);
-            umma_commit(bar_s);
-            ok = mbar_wait_spin(&bar_dof[0], 0, ab, lim, WAIT_BWD_MMA + 9);
+        int it = 0;  // active query tiles so far, over all items
+        for (int w = 0; ok && (PERSIST || w == 0); ++w) {
+          int bh, j, hh, i_begin;
+          if (!bwd_item<C::SPLIT, PERSIST>(p, w, bh, j, hh, i_begin)) break;
+          const BwdTiles tt = bwd_tiles(p, bh);
+          ok = mbar_wait_spin(bar_kv, (uint32_t)w & 1u, ab, lim, WAIT_BWD_MMA + 1);
+          if (!ok) break;
+          int i = i_begin;
+          while (i < tt.nb && !bwd_tile_active(tt, i, j)) ++i;
+          int ni = 0;  // this item's active query tiles so far
+          if (i < tt.nb) {
+            ok = mbar_wait_spin(&bar_qf[it % NS], (uint32_t)(it / NS) & 1u, ab, lim, WAIT_BWD_MMA + 2);
+            if (ok) {
+              tc_fence_after();
+              issue_s(it % NS);
+              umma_commit(bar_s);
+              // d = 128: the dP^T columns hold the previous item's last dQ until it is drained
+              if (C::DQ_ALIAS && it > 0) ok = mbar_wait_spin(bar_dqfree, (uint32_t)(it - 1) & 1u, ab, lim, WAIT_BWD_MMA + 7);
+            }
+            if (ok) ok = mbar_wait_spin(&bar_dof[it % NS_DO], (uint32_t)(it / NS_DO) & 1u, ab, lim, WAIT_BWD_MMA + 9);
+            if (ok) {
+              tc_fence_after();
+              issue_dp(it % NS_DO);
+              umma_commit(bar_dp);
+            }
           }
-          if (ok) {
-            tc_fence_after();
-            issue_dp(0);
-            umma_commit(bar_dp);
-          }
-        }
-        while (ok && i < tt.nb) {
-          const int s = it % NS;
-          int inext = i + 1;
-          while (inext < tt.nb && !bwd_tile_active(tt, inext, j)) ++inext;
-          const bool has_next = inext < tt.nb;
-          const int sn = (it + 1) % NS;
-          const int sd = it % NS_DO, sdn = (it + 1) % NS_DO;
-          const uint32_t acc = it > 0 ? 1u : 0u;
-          const uint64_t dOs = dO_mn + (uint64_t)(sd * TILE16), dQs = dQ_mn + (uint64_t)(s * TILE16);
+          while (ok && i < tt.nb) {
+            const int s = it % NS;
+            int inext = i + 1;
+            while (inext < tt.nb && !bwd_tile_active(tt, inext, j)) ++inext;
+            const bool has_next = inext < tt.nb;
+            const int sn = (it + 1) % NS;
+            const int sd = it % NS_DO, sdn = (it + 1) % NS_DO;
+            const uint32_t acc = ni > 0 ? 1u : 0u;
+            const uint64_t dOs = dO_mn + (uint64_t)(sd * TILE16), dQs = dQ_mn + (uint64_t)(s * TILE16);
 
-          // dV += P^T dO_i (reduction over the 128 queries of tile i), A = P^T from TMEM
-          ok = mbar_wait_spin(bar_p, it & 1, ab, lim, WAIT_BWD_MMA + 3);
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, dOs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV,
-                    kk > 0 ? 1u : acc);
-          umma_commit(&bar_doe[sd]);  // dO_i read by dP_i and dV_i
-          // S^T_{i+1} over P^T_i (the dV MMAs above read it first: tcgen05.mma runs in order)
-          if (has_next) {
-            ok = mbar_wait_spin(&bar_qf[sn], ((it + 1) / NS) & 1, ab, lim, WAIT_BWD_MMA + 4);
+            // dV += P^T dO_i (reduction over the 128 queries of tile i), A = P^T from TMEM
+            ok = mbar_wait_spin(bar_p, it & 1, ab, lim, WAIT_BWD_MMA + 3);
+            // the item's first dV overwrites the accumulator the previous item's epilogue reads
+            if (ok && ni == 0 && w > 0) ok = mbar_wait_spin(bar_dvfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 11);
             if (!ok) break;
             tc_fence_after();
-            issue_s(sn);
-            umma_commit(bar_s);
-          }
-          ok = mbar_wait_spin(bar_ds, it & 1, ab, lim, WAIT_BWD_MMA + 5);
-          if (!ok) break;
-          if (!C::DQ_ALIAS && it > 0) {  // d = 64: the dQ columns must have been drained
-            ok = mbar_wait_spin(bar_dqfree, (it - 1) & 1, ab, lim, WAIT_BWD_MMA + 6);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, dOs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV,
+                      kk > 0 ? 1u : acc);
+            umma_commit(&bar_doe[sd]);  // dO_i read by dP_i and dV_i
+            // S^T_{i+1} over P^T_i (the dV MMAs above read it first: tcgen05.mma runs in order)
+            if (has_next) {
+              ok = mbar_wait_spin(&bar_qf[sn], ((it + 1) / NS) & 1, ab, lim, WAIT_BWD_MMA + 4);
+              if (!ok) break;
+              tc_fence_after();
+              issue_s(sn);
+              umma_commit(bar_s);
+            }
+            ok = mbar_wait_spin(bar_ds, it & 1, ab, lim, WAIT_BWD_MMA + 5);
             if (!ok) break;
-          }
-          tc_fence_after();
-          // dQ_i (d = 128: into the dP^T columns, already read by the dS phase)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {  // reduction over the 128 keys of tile j
-            const uint64_t kdesc = dK_mn + (uint64_t)(kk * (2048 >> 4)), sdesc = dS_mn + (uint64_t)(kk * (2048 >> 4));
-            umma_ss(tDQ, sdesc, kdesc, IDESC_Q, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(bar_dq);
-          // dK += dS^T Q_i
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t aoff16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
-            umma_ss(tDK, dS_k + aoff16, dQs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV, kk > 0 ? 1u : acc);
-          }
-          umma_commit(bar_dsfree);
-          umma_commit(&bar_qe[s]);
-          // dP^T_{i+1}
-          if (has_next) {
-            if (C::DQ_ALIAS) {  // the dP^T columns hold dQ_i until the drain warps have read it
-              ok = mbar_wait_spin(bar_dqfree, it & 1, ab, lim, WAIT_BWD_MMA + 7);
+            if (!C::DQ_ALIAS && it > 0) {  // d = 64: the dQ columns must have been drained
+              ok = mbar_wait_spin(bar_dqfree, (it - 1) & 1, ab, lim, WAIT_BWD_MMA + 6);
               if (!ok) break;
             }
-            ok = mbar_wait_spin(&bar_dof[sdn], ((it + 1) / NS_DO) & 1, ab, lim, WAIT_BWD_MMA + 10);
-            if (!ok) break;
             tc_fence_after();
-            issue_dp(sdn);
-            umma_commit(bar_dp);
+            // dQ_i (d = 128: into the dP^T columns, already read by the dS phase)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {  // reduction over the 128 keys of tile j
+              const uint64_t kdesc = dK_mn + (uint64_t)(kk * (2048 >> 4)), sdesc = dS_mn + (uint64_t)(kk * (2048 >> 4));
+              umma_ss(tDQ, sdesc, kdesc, IDESC_Q, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(bar_dq);
+            if (ni == 0 && w > 0) {  // likewise dK
+              ok = mbar_wait_spin(bar_dkfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 12);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            // dK += dS^T Q_i
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t aoff16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
+              umma_ss(tDK, dS_k + aoff16, dQs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV, kk > 0 ? 1u : acc);
+            }
+            umma_commit(bar_dsfree);
+            umma_commit(&bar_qe[s]);
+            // dP^T_{i+1}
+            if (has_next) {
+              if (C::DQ_ALIAS) {  // the dP^T columns hold dQ_i until the drain warps have read it
+                ok = mbar_wait_spin(bar_dqfree, it & 1, ab, lim, WAIT_BWD_MMA + 7);
+                if (!ok) break;
+              }
+              ok = mbar_wait_spin(&bar_dof[sdn], ((it + 1) / NS_DO) & 1, ab, lim, WAIT_BWD_MMA + 10);
+              if (!ok) break;
+              tc_fence_after();
+              issue_dp(sdn);
+              umma_commit(bar_dp);
+            }
+            i = inext;
+            ++it;
+            ++ni;
           }
-          i = inext;
-          ++it;
+          if (ok && ni == 0 && w > 0) {
+            // No query tile (a block mask can empty a key tile): the commit below would otherwise
+            // not wait for the previous item's epilogue, and the epilogue warps could see this
+            // item's accumulator barrier phase complete before they waited for the previous one.
+            ok = mbar_wait_spin(bar_dvfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 11);
+            if (ok) ok = mbar_wait_spin(bar_dkfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 12);
+          }
+          if (!ok) break;
+          umma_commit(bar_acc);  // this item's dK and dV are final once every MMA so far retires
         }
       } else {
+        int bh, j, hh, i_begin;
+        bwd_item<C::SPLIT, PERSIST>(p, 0, bh, j, hh, i_begin);  // d = 256 runs one item per CTA
+        const BwdTiles tt = bwd_tiles(p, bh);
+        ok = mbar_wait_spin(bar_kv, 0, ab, lim, WAIT_BWD_MMA + 1);
         // Panels come off the ring in the producer's order; each is released by a commit right
         // after the MMAs that read it (commits track every earlier MMA, so release is in order).
         // dV and dK take one 64-column panel of this CTA's half at a time (two N = 64 groups).
@@ -562,8 +636,8 @@ __global__ void __launch_bounds__(512, 1)
           i = inext;
           ++it;
         }
+        umma_commit(bar_acc);
       }
-      umma_commit(bar_acc);
       umma_commit(bar_done);
       AbortState none{0};
       mbar_wait(bar_done, 0, &none, lim, WAIT_BWD_MMA + 8);
@@ -583,144 +657,168 @@ __global__ void __launch_bounds__(512, 1)
     constexpr uint32_t EMU = FA_BWD_EXP_EMU_MASK;
     const Ex2PolyConsts ek = ex2_poly_consts();
     bool ok = true;
-    int it = 0;
-    for (int i = i_begin; i < tt.nb; ++i) {
-      if (!bwd_tile_active(tt, i, j)) continue;
-      const int s = it % NS;
-      const float* nlse2 = reinterpret_cast<const float*>(smem + C::OFF_LSE + s * 512) + 64 * h;
-      const float* ndel = reinterpret_cast<const float*>(smem + C::OFF_DEL + s * 512) + 64 * h;
-      // Causal band: key 128j+kr is visible to query 128i+q iff 128j+kr <= 128i+q+causal_off,
-      // i.e. q >= qmin (q >= kr on the diagonal tile of the square problem).
-      const bool diag = tt.causal && (128 * j + 127 > 128 * i + tt.causal_off);
-      const int qmin = kr + 128 * (j - i) - tt.causal_off;
-      // Keys of a partial last tile beyond N_k (zero rows from TMA) take no part: P = 0 there,
-      // so nothing non-finite can reach dQ through them.
-      const bool kpad = 128 * j + kr >= tt.Nk;
-      const int qoff = 64 * h;  // query index of column 0 of this group
+    int it = 0;  // active query tiles so far, over all items
+    for (int w = 0; PERSIST || w == 0; ++w) {
+      int bh, j, hh, i_begin;
+      if (!bwd_item<C::SPLIT, PERSIST>(p, w, bh, j, hh, i_begin)) break;
+      const BwdTiles tt = bwd_tiles(p, bh);
+      int ni = 0;  // this item's active query tiles so far
+      for (int i = i_begin; i < tt.nb; ++i) {
+        if (!bwd_tile_active(tt, i, j)) continue;
+        const int s = it % NS;
+        const float* nlse2 = reinterpret_cast<const float*>(smem + C::OFF_LSE + s * 512) + 64 * h;
+        const float* ndel = reinterpret_cast<const float*>(smem + C::OFF_DEL + s * 512) + 64 * h;
+        // Causal band: key 128j+kr is visible to query 128i+q iff 128j+kr <= 128i+q+causal_off,
+        // i.e. q >= qmin (q >= kr on the diagonal tile of the square problem).
+        const bool diag = tt.causal && (128 * j + 127 > 128 * i + tt.causal_off);
+        const int qmin = kr + 128 * (j - i) - tt.causal_off;
+        // Keys of a partial last tile beyond N_k (zero rows from TMA) take no part: P = 0 there,
+        // so nothing non-finite can reach dQ through them.
+        const bool kpad = 128 * j + kr >= tt.Nk;
+        const int qoff = 64 * h;  // query index of column 0 of this group
 
-      // ---- P phase: P^T = exp2(S^T * scale*log2e - LSE*log2e), back into TMEM as bf16
-      ok = warp_wait(bar_s, it & 1, ab, lim, WAIT_BWD_COMPUTE + 1);
-      if (!ok) break;
-      tc_fence_after();
-      float pf[64];  // P in fp32, kept for the dS phase
-      {
-        uint32_t sa[32], sb[32];
-        tmem_ld32_async(tS_row, sa);
-        tmem_wait_ld_tied(sa);
-        tmem_ld32_async(tS_row + 32, sb);  // in flight while chunk 0 is processed
+        // ---- P phase: P^T = exp2(S^T * scale*log2e - LSE*log2e), back into TMEM as bf16
+        ok = warp_wait(bar_s, it & 1, ab, lim, WAIT_BWD_COMPUTE + 1);
+        if (!ok) break;
+        tc_fence_after();
+        float pf[64];  // P in fp32, kept for the dS phase
+        {
+          uint32_t sa[32], sb[32];
+          tmem_ld32_async(tS_row, sa);
+          tmem_wait_ld_tied(sa);
+          tmem_ld32_async(tS_row + 32, sb);  // in flight while chunk 0 is processed
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t (&su)[32] = c == 0 ? sa : sb;
-          if (c == 1) tmem_wait_ld_tied(sb);
-          uint32_t pk[16];
+          for (int c = 0; c < 2; ++c) {
+            uint32_t (&su)[32] = c == 0 ? sa : sb;
+            if (c == 1) tmem_wait_ld_tied(sb);
+            uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            const int q = 32 * c + 2 * e;  // local query index of this 4-query group
-            const float4 nl = *reinterpret_cast<const float4*>(&nlse2[q]);
-            const uint64_t x01 = ffma2(f2_pack(__uint_as_float(su[2 * e]), __uint_as_float(su[2 * e + 1])), sl2_2,
-                                       f2_pack(nl.x, nl.y));
-            const uint64_t x23 = ffma2(f2_pack(__uint_as_float(su[2 * e + 2]), __uint_as_float(su[2 * e + 3])),
-                                       sl2_2, f2_pack(nl.z, nl.w));
-            float p0, p1, p2, p3;
-            if ((EMU >> e) & 1u) {
-              f2_unpack(ex2_poly2(x01, ek), p0, p1);
-            } else {
-              float x0, x1;
-              f2_unpack(x01, x0, x1);
-              p0 = ex2(x0);
-              p1 = ex2(x1);
+            for (int e = 0; e < 16; e += 2) {
+              const int q = 32 * c + 2 * e;  // local query index of this 4-query group
+              const float4 nl = *reinterpret_cast<const float4*>(&nlse2[q]);
+              const uint64_t x01 = ffma2(f2_pack(__uint_as_float(su[2 * e]), __uint_as_float(su[2 * e + 1])), sl2_2,
+                                         f2_pack(nl.x, nl.y));
+              const uint64_t x23 = ffma2(f2_pack(__uint_as_float(su[2 * e + 2]), __uint_as_float(su[2 * e + 3])),
+                                         sl2_2, f2_pack(nl.z, nl.w));
+              float p0, p1, p2, p3;
+              if ((EMU >> e) & 1u) {
+                f2_unpack(ex2_poly2(x01, ek), p0, p1);
+              } else {
+                float x0, x1;
+                f2_unpack(x01, x0, x1);
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+              }
+              if ((EMU >> (e + 1)) & 1u) {
+                f2_unpack(ex2_poly2(x23, ek), p2, p3);
+              } else {
+                float x2, x3;
+                f2_unpack(x23, x2, x3);
+                p2 = ex2(x2);
+                p3 = ex2(x3);
+              }
+              if (diag) {  // key kr is visible to query qoff+q iff qoff+q >= qmin
+                const int qq = qoff + q;
+                if (qq < qmin) p0 = 0.f;
+                if (qq + 1 < qmin) p1 = 0.f;
+                if (qq + 2 < qmin) p2 = 0.f;
+                if (qq + 3 < qmin) p3 = 0.f;
+              }
+              if (kpad) p0 = p1 = p2 = p3 = 0.f;
+              pf[q] = p0;
+              pf[q + 1] = p1;
+              pf[q + 2] = p2;
+              pf[q + 3] = p3;
+              pk[e] = pack16<F16>(p0, p1);
+              pk[e + 1] = pack16<F16>(p2, p3);
             }
-            if ((EMU >> (e + 1)) & 1u) {
-              f2_unpack(ex2_poly2(x23, ek), p2, p3);
-            } else {
-              float x2, x3;
-              f2_unpack(x23, x2, x3);
-              p2 = ex2(x2);
-              p3 = ex2(x3);
-            }
-            if (diag) {  // key kr is visible to query qoff+q iff qoff+q >= qmin
-              const int qq = qoff + q;
-              if (qq < qmin) p0 = 0.f;
-              if (qq + 1 < qmin) p1 = 0.f;
-              if (qq + 2 < qmin) p2 = 0.f;
-              if (qq + 3 < qmin) p3 = 0.f;
-            }
-            if (kpad) p0 = p1 = p2 = p3 = 0.f;
-            pf[q] = p0;
-            pf[q + 1] = p1;
-            pf[q + 2] = p2;
-            pf[q + 3] = p3;
-            pk[e] = pack16<F16>(p0, p1);
-            pk[e + 1] = pack16<F16>(p2, p3);
+            tmem_st16(tS_row + c * 16, pk);  // columns [64h + 16c, +16): scores already read
           }
-          tmem_st16(tS_row + c * 16, pk);  // columns [64h + 16c, +16): scores already read
         }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_p);
 
-      // ---- dS phase: dS^T = P^T o (dP^T - D) into shared-memory panel h
-      ok = warp_wait(bar_dp, it & 1, ab, lim, WAIT_BWD_COMPUTE + 2);
-      if (ok && it > 0) ok = warp_wait(bar_dsfree, (it - 1) & 1, ab, lim, WAIT_BWD_COMPUTE + 3);
-      if (!ok) break;
-      tc_fence_after();
-      {
-        uint32_t da[32], db[32];
-        tmem_ld32_async(tDP_row, da);
-        tmem_wait_ld_tied(da);
-        tmem_ld32_async(tDP_row + 32, db);
-        const uint32_t panel = sDS + h * C::PANEL_BYTES;
+        // ---- dS phase: dS^T = P^T o (dP^T - D) into shared-memory panel h
+        ok = warp_wait(bar_dp, it & 1, ab, lim, WAIT_BWD_COMPUTE + 2);
+        if (ok && it > 0) ok = warp_wait(bar_dsfree, (it - 1) & 1, ab, lim, WAIT_BWD_COMPUTE + 3);
+        // the previous item's dV store reads its staging area, the dS buffer
+        if (ok && PERSIST && ni == 0 && w > 0) ok = warp_wait(bar_vst, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_COMPUTE + 4);
+        if (!ok) break;
+        tc_fence_after();
+        {
+          uint32_t da[32], db[32];
+          tmem_ld32_async(tDP_row, da);
+          tmem_wait_ld_tied(da);
+          tmem_ld32_async(tDP_row + 32, db);
+          const uint32_t panel = sDS + h * C::PANEL_BYTES;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t (&du)[32] = c == 0 ? da : db;
-          if (c == 1) tmem_wait_ld_tied(db);
-          uint32_t dk[16];
+          for (int c = 0; c < 2; ++c) {
+            uint32_t (&du)[32] = c == 0 ? da : db;
+            if (c == 1) tmem_wait_ld_tied(db);
+            uint32_t dk[16];
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            const int q = 32 * c + 2 * e;
-            const float4 nd = *reinterpret_cast<const float4*>(&ndel[q]);
-            const uint64_t t01 = fadd2(f2_pack(__uint_as_float(du[2 * e]), __uint_as_float(du[2 * e + 1])),
-                                       f2_pack(nd.x, nd.y));
-            const uint64_t t23 = fadd2(f2_pack(__uint_as_float(du[2 * e + 2]), __uint_as_float(du[2 * e + 3])),
-                                       f2_pack(nd.z, nd.w));
-            const uint64_t ds01 = fmul2(f2_pack(pf[q], pf[q + 1]), t01);
-            const uint64_t ds23 = fmul2(f2_pack(pf[q + 2], pf[q + 3]), t23);
-            float d0, d1, d2, d3;
-            f2_unpack(ds01, d0, d1);
-            f2_unpack(ds23, d2, d3);
-            dk[e] = pack16<F16>(d0, d1);
-            dk[e + 1] = pack16<F16>(d2, d3);
+            for (int e = 0; e < 16; e += 2) {
+              const int q = 32 * c + 2 * e;
+              const float4 nd = *reinterpret_cast<const float4*>(&ndel[q]);
+              const uint64_t t01 = fadd2(f2_pack(__uint_as_float(du[2 * e]), __uint_as_float(du[2 * e + 1])),
+                                         f2_pack(nd.x, nd.y));
+              const uint64_t t23 = fadd2(f2_pack(__uint_as_float(du[2 * e + 2]), __uint_as_float(du[2 * e + 3])),
+                                         f2_pack(nd.z, nd.w));
+              const uint64_t ds01 = fmul2(f2_pack(pf[q], pf[q + 1]), t01);
+              const uint64_t ds23 = fmul2(f2_pack(pf[q + 2], pf[q + 3]), t23);
+              float d0, d1, d2, d3;
+              f2_unpack(ds01, d0, d1);
+              f2_unpack(ds23, d2, d3);
+              dk[e] = pack16<F16>(d0, d1);
+              dk[e + 1] = pack16<F16>(d2, d3);
+            }
+            // dS^T row kr, local queries 32c..32c+31 -> 16-byte chunks 4c .. 4c+3 of panel h
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq)
+              st_shared_v4(panel + sw128_offset(kr, c * 4 + qq), dk[4 * qq], dk[4 * qq + 1], dk[4 * qq + 2],
+                           dk[4 * qq + 3]);
           }
-          // dS^T row kr, local queries 32c..32c+31 -> 16-byte chunks 4c .. 4c+3 of panel h
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq)
-            st_shared_v4(panel + sw128_offset(kr, c * 4 + qq), dk[4 * qq], dk[4 * qq + 1], dk[4 * qq + 2],
-                         dk[4 * qq + 3]);
         }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_ds);
+        ++it;
+        ++ni;
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_ds);
-      ++it;
-    }
-    // -------------------------------------------------------------- epilogue: dV (group h: panel h)
-    if (ok) ok = warp_wait(bar_acc, 0, ab, lim, WAIT_BWD_EPILOGUE + 1);
-    uint8_t* stage = smem + C::OFF_Q;  // Q ring stage 0 is free once every MMA retired
-    if (ok && h < C::PANELS_H) {
-      tc_fence_after();
-      stage_row16<64, F16>(tmem + lane_off + C::T_DV + 64u * h, smem_u32(stage + h * C::PANEL_BYTES), kr, p.inv_scale,
-                         it == 0);
-      fence_proxy_async_smem();
-    }
-    named_bar_sync(1, 256);
-    if (warp == 4 && lane == 0 && *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
-      for (int pn = 0; pn < C::PANELS_H; ++pn)
-        tma_store_3d(&tmdV, stage + pn * C::PANEL_BYTES, C::DH * hh + pn * 64, j * 128, bh);
-      bulk_commit_group();
-      bulk_wait_group_read0();
+      // -------------------------------------------------------------- epilogue: dV (group h: panel h)
+      if (ok) ok = warp_wait(bar_acc, (uint32_t)w & 1u, ab, lim, WAIT_BWD_EPILOGUE + 1);
+      // Staging: one item per CTA: Q ring stage 0 (SPLIT: panels 0-1), free once every MMA retired.
+      // Persistent CTAs: the dS buffer, since the ring may already hold the next item's first tile
+      // (this group's next dS phase waits for the store to have read it).
+      uint8_t* stage = smem + (PERSIST ? C::OFF_DS : C::OFF_Q);
+      if (ok && h < C::PANELS_H) {
+        tc_fence_after();
+        stage_row16<64, F16>(tmem + lane_off + C::T_DV + 64u * h, smem_u32(stage + h * C::PANEL_BYTES), kr, p.inv_scale,
+                           ni == 0);
+        fence_proxy_async_smem();
+      }
+      if (PERSIST) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_dvfree);  // dV read out: the next item's first dV may overwrite it
+      }
+      // staged; a persistent CTA also stops every warp after a failed wait
+      bool all_ok = true;
+      if (PERSIST)
+        all_ok = named_bar_and(1, 256, ok);
+      else
+        named_bar_sync(1, 256);
+      if (warp == 4 && lane == 0 && *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
+        for (int pn = 0; pn < C::PANELS_H; ++pn)
+          tma_store_3d(&tmdV, stage + pn * C::PANEL_BYTES, C::DH * hh + pn * 64, j * 128, bh);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+        if (PERSIST) mbar_arrive(bar_vst);
+      }
+      if (!all_ok) break;
     }
   } else if (warp >= 12) {
     // ------------------------------------------------------------------ dQ drain
@@ -737,66 +835,88 @@ __global__ void __launch_bounds__(512, 1)
     const bool issuer = (wq == 0 && lane == 0);  // issues the bulk reductions of the warpgroup
     if (issuer) tma_prefetch_desc(&tmdQa);
     bool ok = true;
-    int it = 0;
+    int it = 0;         // active query tiles so far, over all items
     uint32_t nred = 0;  // bulk reductions issued so far (staging slot = nred % DQ_SLOTS)
-    for (int i = i_begin; i < tt.nb; ++i) {
-      if (!bwd_tile_active(tt, i, j)) continue;
-      ok = warp_wait(bar_dq, it & 1, ab, lim, WAIT_BWD_DQ + 1);
-      // Read the whole row and release the TMEM columns before anything else (at d = 128 the
-      // next dP^T is written there). When aborting (!ok) the values are not used; the columns
-      // stay allocated until every role has left.
-      uint32_t u[C::DH];
-      tc_fence_after();
-      if constexpr (C::DH == 128) {
+    for (int w = 0; PERSIST || w == 0; ++w) {
+      int bh, j, hh, i_begin;
+      if (!bwd_item<C::SPLIT, PERSIST>(p, w, bh, j, hh, i_begin)) break;
+      const BwdTiles tt = bwd_tiles(p, bh);
+      int ni = 0;  // this item's active query tiles so far
+      for (int i = i_begin; i < tt.nb; ++i) {
+        if (!bwd_tile_active(tt, i, j)) continue;
+        ok = warp_wait(bar_dq, it & 1, ab, lim, WAIT_BWD_DQ + 1);
+        // Read the whole row and release the TMEM columns before anything else (at d = 128 the
+        // next dP^T is written there). When aborting (!ok) the values are not used; the columns
+        // stay allocated until every role has left.
+        uint32_t u[C::DH];
+        tc_fence_after();
+        if constexpr (C::DH == 128) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32_async(tDQ_row + c * 32, *reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
+          for (int c = 0; c < 4; ++c) tmem_ld32_async(tDQ_row + c * 32, *reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_wait_ld_tied(*reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
-      } else {
-        tmem_ld64(tDQ_row, u);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0 && ok) mbar_arrive(bar_dqfree);
-      // the four warps leave together: they meet at named barriers below
-      if (!named_bar_and(3, 128, ok)) break;
-      const int row0 = bh * p.Np + i * 128;
-#pragma unroll
-      for (int c = 0; c < C::DQ_CHUNKS; ++c, ++nred) {
-        if (issuer && nred >= C::DQ_SLOTS) bulk_wait_group_read<C::DQ_SLOTS - 1>();
-        named_bar_sync(3, 128);  // the slot's previous reduction has read it
-        const uint32_t slot = sDQS + (nred % C::DQ_SLOTS) * C::DQ_SLOT_BYTES;
-#pragma unroll
-        for (int k = 0; k < 8; ++k)  // 16-byte chunk k of row ln: columns 32c + 4k .. +3
-          st_shared_v4(slot + sw128_offset(ln, k), u[32 * c + 4 * k], u[32 * c + 4 * k + 1], u[32 * c + 4 * k + 2],
-                       u[32 * c + 4 * k + 3]);
-        fence_proxy_async_smem();
-        named_bar_sync(3, 128);  // slot written
-        if (issuer) {
-          tma_reduce_add_2d(&tmdQa, slot, C::DH * hh + 32 * c, row0);
-          bulk_commit_group();
+          for (int c = 0; c < 4; ++c) tmem_wait_ld_tied(*reinterpret_cast<uint32_t (*)[32]>(&u[c * 32]));
+        } else {
+          tmem_ld64(tDQ_row, u);
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0 && ok) mbar_arrive(bar_dqfree);
+        // the four warps leave together: they meet at named barriers below
+        if (!named_bar_and(3, 128, ok)) break;
+        const int row0 = bh * p.Np + i * 128;
+#pragma unroll
+        for (int c = 0; c < C::DQ_CHUNKS; ++c, ++nred) {
+          if (issuer && nred >= C::DQ_SLOTS) bulk_wait_group_read<C::DQ_SLOTS - 1>();
+          named_bar_sync(3, 128);  // the slot's previous reduction has read it
+          const uint32_t slot = sDQS + (nred % C::DQ_SLOTS) * C::DQ_SLOT_BYTES;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)  // 16-byte chunk k of row ln: columns 32c + 4k .. +3
+            st_shared_v4(slot + sw128_offset(ln, k), u[32 * c + 4 * k], u[32 * c + 4 * k + 1], u[32 * c + 4 * k + 2],
+                         u[32 * c + 4 * k + 3]);
+          fence_proxy_async_smem();
+          named_bar_sync(3, 128);  // slot written
+          if (issuer) {
+            tma_reduce_add_2d(&tmdQa, slot, C::DH * hh + 32 * c, row0);
+            bulk_commit_group();
+          }
+        }
+        ++it;
+        ++ni;
       }
-      ++it;
+      // -------------------------------------------------------------- epilogue: dK (dS carries the scale)
+      if (ok) ok = warp_wait(bar_acc, (uint32_t)w & 1u, ab, lim, WAIT_BWD_EPILOGUE + 2);
+      // Staging: one item per CTA: dO ring stage 0 (SPLIT: ring panel slots 2-3), free once every
+      // MMA retired, so the last dQ reductions complete meanwhile. Persistent CTAs: the dQ slots
+      // once those reductions have read them, since the dO ring may hold the next item's first tile.
+      uint8_t* stage = smem + (PERSIST ? C::OFF_DQS : C::SPLIT ? C::OFF_Q + 2 * C::PANEL_BYTES : C::OFF_DO);
+      if (PERSIST) {
+        if (issuer) bulk_wait_group_read0();
+        named_bar_sync(2, 128);
+      }
+      if (ok) {
+        tc_fence_after();
+        stage_row16<C::DH, F16>(tmem + lane_off + C::T_DK, smem_u32(stage), ln, 1.f, ni == 0);
+        fence_proxy_async_smem();
+      }
+      if (PERSIST) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_dkfree);  // dK read out: the next item's first dK may overwrite it
+      }
+      bool all_ok = true;
+      if (PERSIST)
+        all_ok = named_bar_and(2, 128, ok);
+      else
+        named_bar_sync(2, 128);
+      if (wq == 0 && lane == 0 && *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
+        for (int pn = 0; pn < C::PANELS_H; ++pn)
+          tma_store_3d(&tmdK, stage + pn * C::PANEL_BYTES, C::DH * hh + pn * 64, j * 128, bh);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+      }
+      if (!all_ok) break;
     }
-    // The last reductions complete while dK is written (its staging area is not a dQ slot).
-    // -------------------------------------------------------------- epilogue: dK (dS carries the scale)
-    if (ok) ok = warp_wait(bar_acc, 0, ab, lim, WAIT_BWD_EPILOGUE + 2);
-    // dO ring stage 0 (SPLIT: panel slots 2-3), free once every MMA retired
-    uint8_t* stage = smem + (C::SPLIT ? C::OFF_Q + 2 * C::PANEL_BYTES : C::OFF_DO);
-    if (ok) {
-      tc_fence_after();
-      stage_row16<C::DH, F16>(tmem + lane_off + C::T_DK, smem_u32(stage), ln, 1.f, it == 0);
-      fence_proxy_async_smem();
-    }
-    named_bar_sync(2, 128);
-    if (wq == 0 && lane == 0 && *reinterpret_cast<volatile int*>(&ab->flag) == 0) {
-      for (int pn = 0; pn < C::PANELS_H; ++pn)
-        tma_store_3d(&tmdK, stage + pn * C::PANEL_BYTES, C::DH * hh + pn * 64, j * 128, bh);
-      bulk_commit_group();
-      bulk_wait_group_read0();
-    }
-    if (issuer) bulk_wait_group0();  // every dQ reduction and the dK store complete before the CTA exits
+    if (issuer) bulk_wait_group0();  // every dQ reduction and dK store complete before the CTA exits
   }
 
   tc_fence_before();
@@ -808,30 +928,45 @@ __global__ void __launch_bounds__(512, 1)
   }
 }
 
-template <int D, bool F16>
+template <int D, bool F16, bool PERSIST>
 static cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
                                 const CUtensorMap& tdqa, const BwdParams& p, long long BH, cudaStream_t stream) {
   using C = BwdCfg<D>;
-  cudaError_t e =
-      cudaFuncSetAttribute(fa_bwd_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  cudaError_t e = cudaFuncSetAttribute(fa_bwd_kernel<D, F16, PERSIST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const dim3 grid = grid_work(p.nbk * (C::SPLIT ? 2 : 1), BH, p.order_group);  // SPLIT: two CTAs per key tile
-  fa_bwd_kernel<D, F16><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdk, tdv, tdqa, p);
+  const int items = p.nbk * (C::SPLIT ? 2 : 1);  // SPLIT: two CTAs per key tile
+  dim3 grid;
+  if (PERSIST) {  // one persistent CTA per SM walks the items (cta_item)
+    const long long total = BH * items, sms = device_sm_count();
+    grid = dim3((unsigned)(total < sms ? total : sms));
+  } else {
+    grid = grid_work(items, BH, p.order_group);
+  }
+  fa_bwd_kernel<D, F16, PERSIST><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdk, tdv, tdqa, p);
   return cudaGetLastError();
+}
+
+template <int D, bool F16>
+static cudaError_t launch_bwd_p(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
+                                const CUtensorMap& tdqa, const BwdParams& p, long long BH, cudaStream_t stream) {
+  if (D != 256 && p.persist > 0) return launch_bwd_t<D, F16, D != 256>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+  return launch_bwd_t<D, F16, false>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
 }
 
 cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
                             const CUtensorMap& tdqa, const BwdParams& p, long long BH, cudaStream_t stream) {
   if (p.f16) {
-    if (D == 64) return launch_bwd_t<64, true>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
-    if (D == 256) return launch_bwd_t<256, true>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
-    return launch_bwd_t<128, true>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+    if (D == 64) return launch_bwd_p<64, true>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+    if (D == 256) return launch_bwd_p<256, true>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+    return launch_bwd_p<128, true>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
   }
-  if (D == 64) return launch_bwd_t<64, false>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
-  if (D == 256) return launch_bwd_t<256, false>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
-  return launch_bwd_t<128, false>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+  if (D == 64) return launch_bwd_p<64, false>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+  if (D == 256) return launch_bwd_p<256, false>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
+  return launch_bwd_p<128, false>(tq, tk, tv, tdo, tdk, tdv, tdqa, p, BH, stream);
 }
 
 }  // namespace fa
