@@ -336,10 +336,12 @@ NAMED_CONFIGS = {
 }
 
 
-def time_kernels(fa, t, shape, causal, mask, scale, steps, warmup):
-    """Per-kernel CUDA-event times (ms, mean over `steps`) of one fwd+bwd step on the views in
-    `t` (q, k, v, do, o, dq, dk, dv of `shape`; lse; ws), after `warmup` untimed steps, and the
-    whole-loop time per step."""
+def time_kernels(fa, t, shape, causal, mask, scale, steps, warmup, min_warm_s=0.0, min_timed_s=0.0):
+    """Per-kernel CUDA-event times (ms, mean over the timed steps) of one fwd+bwd step on the
+    views in `t` (q, k, v, do, o, dq, dk, dv of `shape`; lse; ws), after at least `warmup` untimed
+    steps and `min_warm_s` seconds of them, and the whole-loop time per step. At least `steps`
+    steps are timed, more when that takes under `min_timed_s` (short steps from an idle GPU
+    would otherwise be timed while the clocks ramp up)."""
     import torch
     q, k, v, do, o, dq, dk, dv = (t[x] for x in ("q", "k", "v", "do", "o", "dq", "dk", "dv"))
     lse, ws = t["lse"], t["ws"]
@@ -363,6 +365,14 @@ def time_kernels(fa, t, shape, causal, mask, scale, steps, warmup):
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
+    n_warm, t0 = warmup, time.perf_counter()
+    while time.perf_counter() - t0 < min_warm_s:
+        step()
+        torch.cuda.synchronize()
+        n_warm += 1
+    if min_warm_s > 0 and n_warm > warmup:
+        per_step = (time.perf_counter() - t0) / (n_warm - warmup)
+        steps = max(steps, math.ceil(min_timed_s / per_step))
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
@@ -372,6 +382,11 @@ def time_kernels(fa, t, shape, causal, mask, scale, steps, warmup):
     torch.cuda.synchronize()
     k_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(4)]
     return k_ms, start.elapsed_time(end) / steps
+
+
+# Each sweep point: at least 30 ms of warm-up steps, then at least `--sweep-steps` steps and
+# 20 ms timed (a point's step takes 0.2 to 8 ms).
+SWEEP_WARM_S, SWEEP_TIMED_S = 0.03, 0.02
 
 
 def run_sweep(fa, dev, dtype, steps, warmup, peaks):
@@ -402,7 +417,8 @@ def run_sweep(fa, dev, dtype, steps, warmup, peaks):
         mask = None if mask_np is None else torch.from_numpy(mask_np).to(dev)
         density = float(mask_np.mean()) if mask_np is not None else 1.0
         (f_ms, p_ms, m_ms, d_ms), step_ms = time_kernels(fa, views(B, H, N, d), (B, H, N, d), causal, mask,
-                                                          1.0 / math.sqrt(d), steps, warmup)
+                                                          1.0 / math.sqrt(d), steps, warmup, SWEEP_WARM_S,
+                                                          SWEEP_TIMED_S)
         ff = fwd_flops(B, H, N, d, causal, density)
         fwd_t = ff / (f_ms * 1e-3) / 1e12
         fb_t = 3.5 * ff / (step_ms * 1e-3) / 1e12
@@ -608,6 +624,9 @@ def run_gpu(args, wl, rank, world, local_rank, dist_on):
         line["sweep"] = {"unit": UNIT, "peak": peaks["bf16_tflops"],
                          "peak_kind": f"bf16 dense burst ({peaks['source']})",
                          "steps": args.sweep_steps, "warmup": args.warmup, "dtype": args.dtype,
+                         "timing": f"per point: >= {args.warmup} warm-up steps and >= {SWEEP_WARM_S * 1e3:.0f} ms "
+                                   f"of them, then >= {args.sweep_steps} steps and >= "
+                                   f"{SWEEP_TIMED_S * 1e3:.0f} ms timed",
                          "workload": "16k tokens, hidden 2048: B = 16384/N, H = 2048/d, bf16 N(0,1); "
                                      "per-GPU figures on this rank",
                          "points": points, "configs": named, "clocks": sclk.summary()}
