@@ -81,6 +81,7 @@ struct Workspace {
   float* delta;
   float* lse2;
   float* dq_acc;
+  unsigned long long* counters;
   size_t bytes;
 };
 
@@ -93,7 +94,8 @@ Workspace layout(void* base, int B, int H, int N, int d) {
   w.delta = reinterpret_cast<float*>(p);
   w.lse2 = reinterpret_cast<float*>(p + s_vec);
   w.dq_acc = reinterpret_cast<float*>(p + 2 * s_vec);
-  w.bytes = 2 * s_vec + s_acc;
+  w.counters = reinterpret_cast<unsigned long long*>(p + 2 * s_vec + s_acc);  // 256 bytes, two used
+  w.bytes = 2 * s_vec + s_acc + 256;
   return w;
 }
 
@@ -322,6 +324,7 @@ fa_status plan_bwd_pre(int dtype, const void* o, const void* dO, const float* ls
   p->delta = w.delta;
   p->lse2 = w.lse2;
   p->dq_acc = w.dq_acc;
+  p->counters = w.counters;
   p->rows = (long long)sh.B * sh.H * sh.Nq;
   p->N = sh.Nq;
   p->Np = (sh.Nq + 127) / 128 * 128;
@@ -368,6 +371,7 @@ fa_status plan_bwd_main(int dtype, const void* q, const void* k, const void* v, 
   p.delta = w.delta;
   p.lse2 = w.lse2;
   p.dq_acc = w.dq_acc;
+  p.counters = w.counters;
   p.block_mask = block_mask;
   p.mask_stride = block_mask_head_stride;
   p.N = sh.Nq;
@@ -382,12 +386,12 @@ fa_status plan_bwd_main(int dtype, const void* q, const void* k, const void* v, 
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
   p.f16 = f16;
-  // Persistent CTAs (each walks several (head, key tile) items, the next item's loads overlapping
-  // the previous one's epilogue) pay off when an item is short: at most 8 query tiles per key
-  // tile, no causal mask (whose longest-first order the hardware block scheduler balances
-  // better than a static assignment). Measured: N = 512 +6-7%, N = 1024 d = 64 +3%; from 16
-  // query tiles on and on causal grids they lose (-5% to -19%); block masks make items unequal too.
-  p.persist = (sh.d != 256 && !causal && block_mask == nullptr && p.nb <= 8) ? 1 : 0;
+  // Persistent CTAs (one per SM, each taking (head, key tile) items from a counter in the
+  // workspace, the next item's loads overlapping the previous one's epilogue) pay off when an
+  // item is short: at most 8 query tiles per key tile. Measured (backward kernel alone): N = 512
+  // d = 128 +9-11%, BERT-large shape +4-6%, N = 1024 d = 64 +4%, GPT-2 shape (causal) +1.5%;
+  // from 16 query tiles on they lose (-1% to -6%), so longer problems keep one CTA per item.
+  p.persist = (sh.d != 256 && p.nb <= 8) ? 1 : 0;
   m->BH = BH;
   m->d = sh.d;
   return FA_OK;

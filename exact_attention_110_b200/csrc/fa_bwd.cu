@@ -94,9 +94,9 @@ struct BwdCfg {
   static constexpr int OFF_DEL = OFF_LSE + NS * 512;          // [NS][128] fp32: -D
   static constexpr int OFF_BAR = OFF_DEL + NS * 512;
   static constexpr int NQB = SPLIT ? RING : NS;               // full/empty barrier pairs of the Q ring
-  static constexpr int NBAR = 1 + 2 * NQB + 2 * NS_DO + 12;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16;
+  static constexpr int NBAR = 1 + 2 * NQB + 2 * NS_DO + 16;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // TMEM address, abort flag, item ring [2]
+  static constexpr int SMEM_BYTES = OFF_MISC + 32;
   static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + DH;
   static constexpr bool DQ_ALIAS = (DH == 128);          // dQ reuses the dP^T columns
@@ -150,18 +150,32 @@ __device__ __forceinline__ void stage_row16(uint32_t taddr, uint32_t sstage, int
   }
 }
 
-// Work item w of this CTA (cta_item): head bh, key tile j (SPLIT: item 2j + half hh of d;
-// causal: j = 0 is the heaviest) and the first query tile whose last row sees key tile j's
-// first key. Every role walks the same items.
-template <bool SPLIT, bool PERSIST>
-__device__ __forceinline__ bool bwd_item(const BwdParams& p, int w, int& bh, int& j, int& hh, int& i_begin) {
-  int xj;
-  if (!cta_item(p.BH, p.nbk * (SPLIT ? 2 : 1), p.order_group, PERSIST ? 1 : 0, w, bh, xj)) return false;
+// Key tile j (SPLIT: item 2j + half hh of d) of work item xj of a head, and the first query
+// tile whose last row sees key tile j's first key.
+template <bool SPLIT>
+__device__ __forceinline__ bool bwd_item_of(const BwdParams& p, int xj, int& j, int& hh, int& i_begin) {
   j = SPLIT ? (xj >> 1) : xj;
   hh = SPLIT ? (xj & 1) : 0;
   const int i_first = 128 * j - 127 - p.causal_off;
   i_begin = (p.causal && i_first > 0) ? (i_first + 127) / 128 : 0;
   return true;
+}
+
+// Work item number x of the grid order (x >= 0: the numbers persistent CTAs take from the
+// work counter) or, for x < 0, this CTA's own item in a one-CTA-per-item grid: head bh, key
+// tile j (SPLIT: item 2j + half hh of d; causal: j = 0 is the heaviest) and the first query tile
+// whose last row sees key tile j's first key. False past the last item.
+template <bool SPLIT>
+__device__ __forceinline__ bool bwd_item(const BwdParams& p, long long x, int& bh, int& j, int& hh, int& i_begin) {
+  const int items = p.nbk * (SPLIT ? 2 : 1);
+  int xj;
+  if (x < 0) {
+    if (!cta_work(p.BH, items, p.order_group, bh, xj)) return false;
+  } else {
+    if (x >= p.BH * items) return false;
+    work_item(x, p.BH, items, p.order_group, bh, xj);
+  }
+  return bwd_item_of<SPLIT>(p, xj, j, hh, i_begin);
 }
 __device__ __forceinline__ BwdTiles bwd_tiles(const BwdParams& p, int bh) {
   const uint8_t* bmask = p.block_mask == nullptr ? nullptr : p.block_mask + (size_t)bh * p.mask_stride;
@@ -202,12 +216,15 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bar_dvfree = bar_done + 1;   // dV read out of TMEM by the epilogue (the next item may overwrite)
   uint64_t* bar_dkfree = bar_dvfree + 1; // dK read out of TMEM by the epilogue
   uint64_t* bar_vst = bar_dkfree + 1;    // the dV store has read its staging area (the dS buffer)
+  uint64_t* bar_itf = bar_vst + 1;       // [2] persistent: item ring slot written by the producer
+  uint64_t* bar_ite = bar_itf + 2;       // [2] persistent: item ring slot read by every other role
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   AbortState* ab = reinterpret_cast<AbortState*>(smem + C::OFF_MISC + 4);
+  volatile int* item_ring = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);  // [2] {bh, item}; bh < 0: none
 
-  {
+  if (!PERSIST) {
     int bh0, j0, hh0, ib0;
-    if (!bwd_item<C::SPLIT, PERSIST>(p, 0, bh0, j0, hh0, ib0)) return;
+    if (!bwd_item<C::SPLIT>(p, -1, bh0, j0, hh0, ib0)) return;
   }
   const uint64_t lim = p.timeout_ns;
 
@@ -233,6 +250,10 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(bar_dvfree, 8);  // one arrive per P/dS warp
     mbar_init(bar_dkfree, 4);  // one arrive per dQ-drain warp
     mbar_init(bar_vst, 1);
+    for (int r = 0; r < 2; ++r) {
+      mbar_init(&bar_itf[r], 1);
+      mbar_init(&bar_ite[r], 13);  // the MMA issuer, the eight P/dS warps, the four drain warps
+    }
     ab->flag = 0;
     fence_mbar_init();
   }
@@ -264,8 +285,27 @@ __global__ void __launch_bounds__(512, 1)
         bool ok = true;
         int w = 0;
         for (; ok && (PERSIST || w == 0); ++w) {
+          long long x = -1;
+          if (PERSIST) {
+            // Item number w of this CTA: its block index first, then from the work counter; it goes
+            // to the other roles through ring slot w & 1 (n_total: no more items).
+            const int rs = w & 1;
+            const uint32_t use = (uint32_t)(w >> 1);
+            if (use > 0 && !mbar_wait(&bar_ite[rs], (use - 1) & 1u, ab, lim, WAIT_BWD_LOAD + 7)) {
+              ok = false;
+              break;
+            }
+            x = w == 0 ? (long long)blockIdx.x : (long long)gridDim.x + (long long)atomicAdd(&p.counters[0], 1ull);
+          }
           int bh, j, hh, i_begin;
-          if (!bwd_item<C::SPLIT, PERSIST>(p, w, bh, j, hh, i_begin)) break;
+          const bool have = bwd_item<C::SPLIT>(p, x, bh, j, hh, i_begin);
+          if (PERSIST) {
+            const int rs = w & 1;
+            item_ring[2 * rs] = have ? bh : -1;
+            item_ring[2 * rs + 1] = C::SPLIT ? 2 * j + hh : j;
+            mbar_arrive(&bar_itf[rs]);
+          }
+          if (!have) break;
           const BwdTiles tt = bwd_tiles(p, bh);
           auto load_tile = [&](int i) -> bool {
             // Q_i first: its stage frees at dK_{i-NS}, before dO_i's stage frees at dV_{i-NS_DO}.
@@ -320,7 +360,7 @@ __global__ void __launch_bounds__(512, 1)
         if (w > 0) mbar_wait(bar_kv, (uint32_t)(w - 1) & 1u, &none, lim, WAIT_BWD_LOAD + 3);
       } else {
         int bh, j, hh, i_begin;
-        bwd_item<C::SPLIT, PERSIST>(p, 0, bh, j, hh, i_begin);  // d = 256 runs one item per CTA
+        bwd_item<C::SPLIT>(p, -1, bh, j, hh, i_begin);  // d = 256 runs one item per CTA
         const BwdTiles tt = bwd_tiles(p, bh);
         // K_j (all four panels) stays; everything else streams through the panel ring in the
         // order the MMA issuer consumes it. First tile i0: Q(i0) panels 0-3 (S^T), then V and
@@ -423,7 +463,18 @@ __global__ void __launch_bounds__(512, 1)
         int it = 0;  // active query tiles so far, over all items
         for (int w = 0; ok && (PERSIST || w == 0); ++w) {
           int bh, j, hh, i_begin;
-          if (!bwd_item<C::SPLIT, PERSIST>(p, w, bh, j, hh, i_begin)) break;
+          if (PERSIST) {
+            const int rs = w & 1;
+            ok = mbar_wait_spin(&bar_itf[rs], (uint32_t)(w >> 1) & 1u, ab, lim, WAIT_BWD_MMA + 13);
+            if (!ok) break;
+            const int2 it2 = make_int2(item_ring[2 * rs], item_ring[2 * rs + 1]);
+            mbar_arrive(&bar_ite[rs]);
+            if (it2.x < 0) break;
+            bh = it2.x;
+            bwd_item_of<C::SPLIT>(p, it2.y, j, hh, i_begin);
+          } else if (!bwd_item<C::SPLIT>(p, -1, bh, j, hh, i_begin)) {
+            break;
+          }
           const BwdTiles tt = bwd_tiles(p, bh);
           ok = mbar_wait_spin(bar_kv, (uint32_t)w & 1u, ab, lim, WAIT_BWD_MMA + 1);
           if (!ok) break;
@@ -530,7 +581,7 @@ __global__ void __launch_bounds__(512, 1)
         }
       } else {
         int bh, j, hh, i_begin;
-        bwd_item<C::SPLIT, PERSIST>(p, 0, bh, j, hh, i_begin);  // d = 256 runs one item per CTA
+        bwd_item<C::SPLIT>(p, -1, bh, j, hh, i_begin);  // d = 256 runs one item per CTA
         const BwdTiles tt = bwd_tiles(p, bh);
         ok = mbar_wait_spin(bar_kv, 0, ab, lim, WAIT_BWD_MMA + 1);
         // Panels come off the ring in the producer's order; each is released by a commit right
@@ -660,7 +711,23 @@ __global__ void __launch_bounds__(512, 1)
     int it = 0;  // active query tiles so far, over all items
     for (int w = 0; PERSIST || w == 0; ++w) {
       int bh, j, hh, i_begin;
-      if (!bwd_item<C::SPLIT, PERSIST>(p, w, bh, j, hh, i_begin)) break;
+      if (PERSIST) {
+        const int rs = w & 1;
+        if (!warp_wait(&bar_itf[rs], (uint32_t)(w >> 1) & 1u, ab, lim, WAIT_BWD_COMPUTE + 5)) {
+          ok = false;
+          break;
+        }
+        int2 it2 = make_int2(0, 0);
+        if (lane == 0) it2 = make_int2(item_ring[2 * rs], item_ring[2 * rs + 1]);
+        it2.x = __shfl_sync(0xffffffffu, it2.x, 0);
+        it2.y = __shfl_sync(0xffffffffu, it2.y, 0);
+        if (lane == 0) mbar_arrive(&bar_ite[rs]);
+        if (it2.x < 0) break;
+        bh = it2.x;
+        bwd_item_of<C::SPLIT>(p, it2.y, j, hh, i_begin);
+      } else if (!bwd_item<C::SPLIT>(p, -1, bh, j, hh, i_begin)) {
+        break;
+      }
       const BwdTiles tt = bwd_tiles(p, bh);
       int ni = 0;  // this item's active query tiles so far
       for (int i = i_begin; i < tt.nb; ++i) {
@@ -839,7 +906,23 @@ __global__ void __launch_bounds__(512, 1)
     uint32_t nred = 0;  // bulk reductions issued so far (staging slot = nred % DQ_SLOTS)
     for (int w = 0; PERSIST || w == 0; ++w) {
       int bh, j, hh, i_begin;
-      if (!bwd_item<C::SPLIT, PERSIST>(p, w, bh, j, hh, i_begin)) break;
+      if (PERSIST) {
+        const int rs = w & 1;
+        if (!warp_wait(&bar_itf[rs], (uint32_t)(w >> 1) & 1u, ab, lim, WAIT_BWD_DQ + 2)) {
+          ok = false;
+          break;
+        }
+        int2 it2 = make_int2(0, 0);
+        if (lane == 0) it2 = make_int2(item_ring[2 * rs], item_ring[2 * rs + 1]);
+        it2.x = __shfl_sync(0xffffffffu, it2.x, 0);
+        it2.y = __shfl_sync(0xffffffffu, it2.y, 0);
+        if (lane == 0) mbar_arrive(&bar_ite[rs]);
+        if (it2.x < 0) break;
+        bh = it2.x;
+        bwd_item_of<C::SPLIT>(p, it2.y, j, hh, i_begin);
+      } else if (!bwd_item<C::SPLIT>(p, -1, bh, j, hh, i_begin)) {
+        break;
+      }
       const BwdTiles tt = bwd_tiles(p, bh);
       int ni = 0;  // this item's active query tiles so far
       for (int i = i_begin; i < tt.nb; ++i) {
@@ -925,6 +1008,15 @@ __global__ void __launch_bounds__(512, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (PERSIST && threadIdx.x == 0) {
+    // The last CTA to finish leaves the counters zeroed for the next launch on this workspace
+    // (every CTA has taken its last item number by now).
+    __threadfence();
+    if (atomicAdd(&p.counters[1], 1ull) == (unsigned long long)gridDim.x - 1ull) {
+      p.counters[0] = 0ull;
+      p.counters[1] = 0ull;
+    }
   }
 }
 

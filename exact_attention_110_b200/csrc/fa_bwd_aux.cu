@@ -54,6 +54,10 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdPreParams p) {
     p.delta[out] = 0.f;
     p.lse2[out] = -INFINITY;
   }
+  if (tid == 0 && p.counters != nullptr) {  // the persistent backward's work counters
+    p.counters[0] = 0ull;
+    p.counters[1] = 0ull;
+  }
   // Zero the dQ accumulator (float4 stores).
   const long long nvec = (p.rows / p.N) * (long long)p.Np * D / 4;
   float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);

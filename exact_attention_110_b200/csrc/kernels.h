@@ -54,28 +54,21 @@ __device__ __forceinline__ bool cta_work(long long BH, int items, int group, int
   bh = (int)(g * G + rem % gsz);
   return true;
 }
-// Work item `w` (0, 1, ...) of this CTA. persist = 0: the grid has one CTA per item (grid_work)
-// and w = 0 is the only one. persist > 0: a one-dimensional grid of persistent CTAs takes
-// items blockIdx.x, blockIdx.x + gridDim.x, ... of the same order (head by head, or the causal
-// longest-first groups), so a CTA walks several items and each item's prologue overlaps the
-// previous one's epilogue. False when this CTA has no item w.
-__device__ __forceinline__ bool cta_item(long long BH, int items, int group, int persist, int w, int& bh,
-                                         int& item) {
-  if (persist == 0) return w == 0 && cta_work(BH, items, group, bh, item);
-  const long long x = blockIdx.x + (long long)w * gridDim.x;
-  if (x >= BH * items) return false;
+// Head and item of work-item number x in grid order (the order cta_work gives the CTAs of a
+// one-CTA-per-item grid: head by head, or the causal longest-first groups), for persistent
+// CTAs that take item numbers from a counter. x < BH * items.
+__device__ __forceinline__ void work_item(long long x, long long BH, int items, int group, int& bh, int& item) {
   if (group <= 0) {
     const long long b = x / items;
     bh = (int)b;
     item = (int)(x - b * items);
-    return true;
+    return;
   }
   const long long G = group < BH ? group : BH;
   const long long g = x / (G * items), rem = x - g * G * items;
   const long long gsz = BH - g * G < G ? BH - g * G : G;
   item = (int)(rem / gsz);
   bh = (int)(g * G + rem % gsz);
-  return true;
 }
 inline dim3 grid_work(int items, long long BH, int group) {
   return group > 0 ? dim3((unsigned)(items * BH)) : grid_bh((unsigned)items, BH);
@@ -118,6 +111,7 @@ struct BwdPreParams {
   float* delta;          // [BH][Np]  = -D = -rowsum(dO o O)
   float* lse2;           // [BH][Np]  = -LSE * log2(e) + log2(scale)
   float* dq_acc;         // [BH][Np][D], zeroed here
+  unsigned long long* counters;  // [2] backward work-scheduling counters, zeroed here
   long long rows;        // BH * N
   int N, Np, D;
   float log2_scale;      // log2(scale), scale > 0: folds the softmax scale into P (see fa_bwd.cu)
@@ -140,7 +134,8 @@ struct BwdParams {
   float scale_log2;      // scale * log2(e)
   unsigned long long timeout_ns;
   int f16;               // element type: fp16 if non-zero, bf16 otherwise
-  int persist;           // 0: one CTA per (head, key tile); > 0: persistent CTAs (cta_item)
+  int persist;           // 0: one CTA per (head, key tile); > 0: persistent CTAs
+  unsigned long long* counters;  // persistent: [0] items handed out after each CTA's first, [1] CTAs done
 };
 
 struct FwdMergeParams {

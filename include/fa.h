@@ -85,7 +85,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 /*
  * Bytes of caller-provided device workspace fa_bwd needs: fp32 D [B][H][Np], fp32 scaled
  * LSE [B][H][Np] and the fp32 dQ accumulator [B][H][Np][d] (Np = N rounded up to 128),
- * each 256-byte aligned. Returns 0 for sizes fa_bwd would reject.
+ * each 256-byte aligned, then 256 bytes of work-scheduling counters. Returns 0 for sizes
+ * fa_bwd would reject.
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -108,7 +109,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
 /*
  * The three stages of fa_bwd, exposed so each kernel can be launched (and timed) alone.
  * fa_bwd_preprocess: D_i = sum_t dO_it * O_it (the row sums of dP o P, from the softmax
- *   Jacobian [P3] §4.1), the scaled LSE, and zeroes the fp32 dQ accumulator. HBM-bound.
+ *   Jacobian [P3] §4.1), the scaled LSE, and zeroes the fp32 dQ accumulator and the
+ *   scheduling counters. HBM-bound.
  * fa_bwd_main: per key tile, recompute S and P, accumulate dK and dV on chip, write dk and
  *   dv (bf16), and add each tile's dQ contribution into the fp32 accumulator.
  * fa_bwd_dq_finish: dq = bf16(accumulator).

@@ -53,19 +53,20 @@ def test_fwd_argument_checks(lib):
     assert fwd(lib, scale=math.nan) == 1 and fwd(lib, scale=math.inf) == 1
     assert fwd(lib, d=96) == 2                   # unsupported head dim
     assert fwd(lib, d=512) == 2                  # (d = 256 is supported)
-    assert lib.fa_bwd_workspace_bytes(1, 1, 128, 256) == 2 * 512 + 128 * 256 * 4  # and a backward one
+    assert lib.fa_bwd_workspace_bytes(1, 1, 128, 256) == 2 * 512 + 128 * 256 * 4 + 256  # and a backward one
     assert fwd(lib, N=0) == 1                    # empty sequence -> INVALID
     assert fwd(lib, B=65536, H=65536) == 2      # B*H above the TMA head coordinate's range
 
 
 def test_workspace_size_and_checks(lib):
-    # D, scaled LSE (fp32 each) and the fp32 dQ accumulator, each 256-byte aligned.
+    # D, scaled LSE (fp32 each) and the fp32 dQ accumulator, each 256-byte aligned, then 256
+    # bytes of work-scheduling counters.
     B, H, N, d = 2, 3, 256, 64
     vec = (B * H * N * 4 + 255) // 256 * 256
     acc = (B * H * N * d * 4 + 255) // 256 * 256
-    assert lib.fa_bwd_workspace_bytes(B, H, N, d) == 2 * vec + acc
+    assert lib.fa_bwd_workspace_bytes(B, H, N, d) == 2 * vec + acc + 256
     # any N: the vectors and the accumulator are padded to whole 128-row tiles
-    assert lib.fa_bwd_workspace_bytes(1, 1, 100, 64) == 2 * 512 + 128 * 64 * 4
+    assert lib.fa_bwd_workspace_bytes(1, 1, 100, 64) == 2 * 512 + 128 * 64 * 4 + 256
     assert lib.fa_bwd_workspace_bytes(1, 1, 0, 64) == 0
     assert lib.fa_bwd_workspace_bytes(1, 1, 128, 80) == 0
     need = lib.fa_bwd_workspace_bytes(1, 1, 128, 64)
