@@ -15,6 +15,11 @@
 #include "kernels.h"
 #include "ptx.cuh"
 
+// Row groups (preprocess) or elements (dQ finish) a thread has in flight per step. Measured at
+// N = 4096, d = 128: preprocess 4.42 -> 4.81 TB/s, dQ finish 5.47 -> 6.14 TB/s with 2; 4 lowers
+// the preprocess again (54 registers halve its occupancy).
+#define FA_AUX_UNROLL 2
+
 namespace fa {
 
 template <int D, bool F16>
@@ -27,24 +32,35 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const BwdPreParams p) {
   // warp-uniform so the full-mask shuffles below always see all 32 lanes.
   constexpr int RPW = 32 / TPR;
   const long long warp_g = tid >> 5, nwarps = nthreads >> 5;
-  for (long long r0 = warp_g * RPW; r0 < p.rows; r0 += nwarps * RPW) {
-    const long long row = r0 + lane / TPR;
-    float acc = 0.f;
-    if (row < p.rows) {
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(p.o + row * D) + sub);
-      const uint4 b = __ldg(reinterpret_cast<const uint4*>(p.dout + row * D) + sub);
-      acc = unpack16_lo<F16>(a.x) * unpack16_lo<F16>(b.x) + unpack16_hi<F16>(a.x) * unpack16_hi<F16>(b.x);
-      acc += unpack16_lo<F16>(a.y) * unpack16_lo<F16>(b.y) + unpack16_hi<F16>(a.y) * unpack16_hi<F16>(b.y);
-      acc += unpack16_lo<F16>(a.z) * unpack16_lo<F16>(b.z) + unpack16_hi<F16>(a.z) * unpack16_hi<F16>(b.z);
-      acc += unpack16_lo<F16>(a.w) * unpack16_lo<F16>(b.w) + unpack16_hi<F16>(a.w) * unpack16_hi<F16>(b.w);
+  // U row groups per step, their loads issued before any of their reductions (more bytes in
+  // flight per thread).
+  constexpr int U = FA_AUX_UNROLL;
+  for (long long r0 = warp_g * RPW; r0 < p.rows; r0 += nwarps * RPW * U) {
+    uint4 a[U], b[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long row = r0 + (long long)u * nwarps * RPW + lane / TPR;
+      a[u] = b[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (row < p.rows) {
+        a[u] = __ldg(reinterpret_cast<const uint4*>(p.o + row * D) + sub);
+        b[u] = __ldg(reinterpret_cast<const uint4*>(p.dout + row * D) + sub);
+      }
     }
 #pragma unroll
-    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, TPR);
-    if (sub == 0 && row < p.rows) {
-      const long long bh = row / p.N, i = row % p.N;
-      const long long out = bh * p.Np + i;
-      p.delta[out] = -acc;                               // stored negated: the backward adds it
-      p.lse2[out] = p.log2_scale - p.lse[row] * 1.4426950408889634f;  // log2(scale) - LSE*log2(e)
+    for (int u = 0; u < U; ++u) {
+      const long long row = r0 + (long long)u * nwarps * RPW + lane / TPR;
+      float acc = unpack16_lo<F16>(a[u].x) * unpack16_lo<F16>(b[u].x) + unpack16_hi<F16>(a[u].x) * unpack16_hi<F16>(b[u].x);
+      acc += unpack16_lo<F16>(a[u].y) * unpack16_lo<F16>(b[u].y) + unpack16_hi<F16>(a[u].y) * unpack16_hi<F16>(b[u].y);
+      acc += unpack16_lo<F16>(a[u].z) * unpack16_lo<F16>(b[u].z) + unpack16_hi<F16>(a[u].z) * unpack16_hi<F16>(b[u].z);
+      acc += unpack16_lo<F16>(a[u].w) * unpack16_lo<F16>(b[u].w) + unpack16_hi<F16>(a[u].w) * unpack16_hi<F16>(b[u].w);
+#pragma unroll
+      for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, TPR);
+      if (sub == 0 && row < p.rows) {
+        const long long bh = row / p.N, i = row % p.N;
+        const long long out = bh * p.Np + i;
+        p.delta[out] = -acc;                               // stored negated: the backward adds it
+        p.lse2[out] = p.log2_scale - p.lse[row] * 1.4426950408889634f;  // log2(scale) - LSE*log2(e)
+      }
     }
   }
   // Rows of a partial last query tile beyond N: -inf exponent offset (P = 0 there) and D = 0.
@@ -70,18 +86,36 @@ __global__ void __launch_bounds__(256) fa_dq_finish_kernel(const DqFinishParams 
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long nthreads = (long long)gridDim.x * blockDim.x;
   const long long total = p.rows * TPR;
-  for (long long e = tid; e < total; e += nthreads) {
-    const long long row = e / TPR;
-    const int sub = (int)(e % TPR);
-    const long long bh = row / p.N, i = row % p.N;
-    const float4* src = reinterpret_cast<const float4*>(p.dq_acc + (bh * p.Np + i) * D) + 2 * sub;
-    const float4 a = src[0], b = src[1];
-    uint4 w;
-    w.x = pack16<F16>(a.x * p.scale, a.y * p.scale);
-    w.y = pack16<F16>(a.z * p.scale, a.w * p.scale);
-    w.z = pack16<F16>(b.x * p.scale, b.y * p.scale);
-    w.w = pack16<F16>(b.z * p.scale, b.w * p.scale);
-    reinterpret_cast<uint4*>(p.dq + row * D)[sub] = w;
+  constexpr int U = FA_AUX_UNROLL;  // U elements' loads in flight before their stores
+  for (long long e0 = tid; e0 < total; e0 += nthreads * U) {
+    float4 a[U], b[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long e = e0 + (long long)u * nthreads;
+      a[u] = b[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e < total) {
+        const long long row = e / TPR;
+        const int sub = (int)(e % TPR);
+        const long long bh = row / p.N, i = row % p.N;
+        const float4* src = reinterpret_cast<const float4*>(p.dq_acc + (bh * p.Np + i) * D) + 2 * sub;
+        a[u] = src[0];
+        b[u] = src[1];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long e = e0 + (long long)u * nthreads;
+      if (e < total) {
+        const long long row = e / TPR;
+        const int sub = (int)(e % TPR);
+        uint4 w;
+        w.x = pack16<F16>(a[u].x * p.scale, a[u].y * p.scale);
+        w.y = pack16<F16>(a[u].z * p.scale, a[u].w * p.scale);
+        w.z = pack16<F16>(b[u].x * p.scale, b[u].y * p.scale);
+        w.w = pack16<F16>(b[u].z * p.scale, b[u].w * p.scale);
+        reinterpret_cast<uint4*>(p.dq + row * D)[sub] = w;
+      }
+    }
   }
 }
 
