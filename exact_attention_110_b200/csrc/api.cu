@@ -387,11 +387,11 @@ fa_status plan_bwd_main(int dtype, const void* q, const void* k, const void* v, 
   p.timeout_ns = kWaitLimitNs;
   p.f16 = f16;
   // Persistent CTAs (one per SM, each taking (head, key tile) items from a counter in the
-  // workspace, the next item's loads overlapping the previous one's epilogue) pay off when an
-  // item is short: at most 8 query tiles per key tile. Measured (backward kernel alone): N = 512
-  // d = 128 +9-11%, BERT-large shape +4-6%, N = 1024 d = 64 +4%, GPT-2 shape (causal) +1.5%;
-  // from 16 query tiles on they lose (-1% to -6%), so longer problems keep one CTA per item.
-  p.persist = (sh.d != 256 && p.nb <= 8) ? 1 : 0;
+  // workspace, the next item's loads overlapping the previous one's epilogue) for d <= 128 (d =
+  // 256 runs two CTAs per key tile, one per half of d). Measured (backward kernel alone, against
+  // one CTA per item): N = 512 d = 128 +10-11%, BERT-large shape +12%, N = 1024 d = 64 +4%, N = 2048
+  // +1%, N = 4096 d = 64 +2%, N = 4096 and 16384 at d = 128 and causal N = 4096 unchanged.
+  p.persist = (sh.d != 256) ? 1 : 0;
   m->BH = BH;
   m->d = sh.d;
   return FA_OK;

@@ -477,6 +477,13 @@ __global__ void __launch_bounds__(512, 1)
           }
           const BwdTiles tt = bwd_tiles(p, bh);
           ok = mbar_wait_spin(bar_kv, (uint32_t)w & 1u, ab, lim, WAIT_BWD_MMA + 1);
+          if (PERSIST && ok && w > 0) {
+            // This item's first dV and dK MMAs overwrite the accumulators the previous item's
+            // epilogue reads; it reads them out right after its accumulator barrier, well within
+            // the K/V load just waited for. Waiting here keeps the per-tile loop free of checks.
+            ok = mbar_wait_spin(bar_dvfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 11);
+            if (ok) ok = mbar_wait_spin(bar_dkfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 12);
+          }
           if (!ok) break;
           int i = i_begin;
           while (i < tt.nb && !bwd_tile_active(tt, i, j)) ++i;
@@ -509,8 +516,6 @@ __global__ void __launch_bounds__(512, 1)
 
             // dV += P^T dO_i (reduction over the 128 queries of tile i), A = P^T from TMEM
             ok = mbar_wait_spin(bar_p, it & 1, ab, lim, WAIT_BWD_MMA + 3);
-            // the item's first dV overwrites the accumulator the previous item's epilogue reads
-            if (ok && ni == 0 && w > 0) ok = mbar_wait_spin(bar_dvfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 11);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
@@ -540,11 +545,6 @@ __global__ void __launch_bounds__(512, 1)
               umma_ss(tDQ, sdesc, kdesc, IDESC_Q, kk > 0 ? 1u : 0u);
             }
             umma_commit(bar_dq);
-            if (ni == 0 && w > 0) {  // likewise dK
-              ok = mbar_wait_spin(bar_dkfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 12);
-              if (!ok) break;
-              tc_fence_after();
-            }
             // dK += dS^T Q_i
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
@@ -569,13 +569,9 @@ __global__ void __launch_bounds__(512, 1)
             ++it;
             ++ni;
           }
-          if (ok && ni == 0 && w > 0) {
-            // No query tile (a block mask can empty a key tile): the commit below would otherwise
-            // not wait for the previous item's epilogue, and the epilogue warps could see this
-            // item's accumulator barrier phase complete before they waited for the previous one.
-            ok = mbar_wait_spin(bar_dvfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 11);
-            if (ok) ok = mbar_wait_spin(bar_dkfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 12);
-          }
+          // (An item without query tiles -- a block mask can empty a key tile -- commits only after
+          // the waits above, so the epilogue warps cannot see its accumulator phase complete
+          // before they waited for the previous one.)
           if (!ok) break;
           umma_commit(bar_acc);  // this item's dK and dV are final once every MMA so far retires
         }
@@ -710,19 +706,23 @@ __global__ void __launch_bounds__(512, 1)
     bool ok = true;
     int it = 0;  // active query tiles so far, over all items
     for (int w = 0; PERSIST || w == 0; ++w) {
-      int bh, j, hh, i_begin;
+      int bh = 0, j = 0, hh = 0, i_begin = 0;
       if (PERSIST) {
         const int rs = w & 1;
-        if (!warp_wait(&bar_itf[rs], (uint32_t)(w >> 1) & 1u, ab, lim, WAIT_BWD_COMPUTE + 5)) {
-          ok = false;
-          break;
-        }
-        int2 it2 = make_int2(0, 0);
-        if (lane == 0) it2 = make_int2(item_ring[2 * rs], item_ring[2 * rs + 1]);
+        bool got = warp_wait(&bar_itf[rs], (uint32_t)(w >> 1) & 1u, ab, lim, WAIT_BWD_COMPUTE + 5);
+        int2 it2 = make_int2(-1, 0);
+        if (got && lane == 0) it2 = make_int2(item_ring[2 * rs], item_ring[2 * rs + 1]);
         it2.x = __shfl_sync(0xffffffffu, it2.x, 0);
         it2.y = __shfl_sync(0xffffffffu, it2.y, 0);
-        if (lane == 0) mbar_arrive(&bar_ite[rs]);
-        if (it2.x < 0) break;
+        if (got && lane == 0) mbar_arrive(&bar_ite[rs]);
+        // The previous item's dV store reads its staging area, the dS buffer, which this item's
+        // first dS phase overwrites (waiting here keeps the per-tile loop free of checks).
+        if (got && w > 0 && it2.x >= 0) got = warp_wait(bar_vst, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_COMPUTE + 4);
+        // Every warp of the two groups takes the same decision: they meet at named barriers.
+        if (!named_bar_and(1, 256, got && it2.x >= 0)) {
+          ok = ok && named_bar_and(1, 256, got);
+          break;
+        }
         bh = it2.x;
         bwd_item_of<C::SPLIT>(p, it2.y, j, hh, i_begin);
       } else if (!bwd_item<C::SPLIT>(p, -1, bh, j, hh, i_begin)) {
@@ -810,9 +810,7 @@ __global__ void __launch_bounds__(512, 1)
         // ---- dS phase: dS^T = P^T o (dP^T - D) into shared-memory panel h
         ok = warp_wait(bar_dp, it & 1, ab, lim, WAIT_BWD_COMPUTE + 2);
         if (ok && it > 0) ok = warp_wait(bar_dsfree, (it - 1) & 1, ab, lim, WAIT_BWD_COMPUTE + 3);
-        // the previous item's dV store reads its staging area, the dS buffer
-        if (ok && PERSIST && ni == 0 && w > 0) ok = warp_wait(bar_vst, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_COMPUTE + 4);
-        if (!ok) break;
+          if (!ok) break;
         tc_fence_after();
         {
           uint32_t da[32], db[32];
@@ -905,19 +903,20 @@ __global__ void __launch_bounds__(512, 1)
     int it = 0;         // active query tiles so far, over all items
     uint32_t nred = 0;  // bulk reductions issued so far (staging slot = nred % DQ_SLOTS)
     for (int w = 0; PERSIST || w == 0; ++w) {
-      int bh, j, hh, i_begin;
+      int bh = 0, j = 0, hh = 0, i_begin = 0;
       if (PERSIST) {
         const int rs = w & 1;
-        if (!warp_wait(&bar_itf[rs], (uint32_t)(w >> 1) & 1u, ab, lim, WAIT_BWD_DQ + 2)) {
-          ok = false;
-          break;
-        }
-        int2 it2 = make_int2(0, 0);
-        if (lane == 0) it2 = make_int2(item_ring[2 * rs], item_ring[2 * rs + 1]);
+        const bool got = warp_wait(&bar_itf[rs], (uint32_t)(w >> 1) & 1u, ab, lim, WAIT_BWD_DQ + 2);
+        int2 it2 = make_int2(-1, 0);
+        if (got && lane == 0) it2 = make_int2(item_ring[2 * rs], item_ring[2 * rs + 1]);
         it2.x = __shfl_sync(0xffffffffu, it2.x, 0);
         it2.y = __shfl_sync(0xffffffffu, it2.y, 0);
-        if (lane == 0) mbar_arrive(&bar_ite[rs]);
-        if (it2.x < 0) break;
+        if (got && lane == 0) mbar_arrive(&bar_ite[rs]);
+        // Every warp of the group takes the same decision: they meet at named barriers.
+        if (!named_bar_and(2, 128, got && it2.x >= 0)) {
+          ok = ok && named_bar_and(2, 128, got);
+          break;
+        }
         bh = it2.x;
         bwd_item_of<C::SPLIT>(p, it2.y, j, hh, i_begin);
       } else if (!bwd_item<C::SPLIT>(p, -1, bh, j, hh, i_begin)) {
