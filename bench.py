@@ -384,9 +384,11 @@ def time_kernels(fa, t, shape, causal, mask, scale, steps, warmup, min_warm_s=0.
     return k_ms, start.elapsed_time(end) / steps
 
 
-# Each sweep point: at least 30 ms of warm-up steps, then at least `--sweep-steps` steps and
-# 20 ms timed (a point's step takes 0.2 to 8 ms).
-SWEEP_WARM_S, SWEEP_TIMED_S = 0.03, 0.02
+# Each sweep point: at least 10 ms of warm-up steps, then at least `--sweep-steps` steps and
+# 10 ms timed (a point's step takes 0.2 to 8 ms): short steps are no longer timed while the
+# clocks ramp up from idle, and long ones see about the load of the headline's timed region
+# (30 + 20 ms put the N >= 4096 points under the power cap).
+SWEEP_WARM_S, SWEEP_TIMED_S = 0.01, 0.01
 
 
 def run_sweep(fa, dev, dtype, steps, warmup, peaks):
