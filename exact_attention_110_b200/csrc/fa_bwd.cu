@@ -39,10 +39,13 @@
 //    the dQ drain); dP_{i+1}.
 //  * TMEM: S^T/P^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D); dQ: d = 128
 //    reuses the dP^T columns once dP^T has been read, d = 64 has its own [384,448).
-//  * PERSIST: one CTA per SM walks several (b, h, key tile) items (cta_item); ring counters and
-//    barrier phases run on across items, the next item's loads overlap the previous item's
-//    epilogue, and three more barriers (dV / dK read out of TMEM, dV store done reading its
-//    staging buffer) keep the next item's first dV / dK MMAs and dS writes behind it.
+//  * PERSIST (d <= 128): one CTA per SM walks several (b, h, key tile) items, its block index
+//    first and then numbers taken from a counter in the workspace (bwd_item, work_item), which
+//    the producer passes to the other roles through a two-slot ring in shared memory. Ring
+//    counters and barrier phases run on across items, the next item's loads overlap the
+//    previous item's epilogue, and three more barriers (dV / dK read out of TMEM, dV store done
+//    reading its staging buffer) keep the next item's first dV / dK MMAs and dS writes behind it;
+//    they are waited at the item's start, so the per-tile loops carry no per-item checks.
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -1029,7 +1032,7 @@ static cudaError_t launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   if (e != cudaSuccess) return e;
   const int items = p.nbk * (C::SPLIT ? 2 : 1);  // SPLIT: two CTAs per key tile
   dim3 grid;
-  if (PERSIST) {  // one persistent CTA per SM walks the items (cta_item)
+  if (PERSIST) {  // one persistent CTA per SM walks the items (bwd_item)
     const long long total = BH * items, sms = device_sm_count();
     grid = dim3((unsigned)(total < sms ? total : sms));
   } else {
