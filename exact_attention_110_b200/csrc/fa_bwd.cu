@@ -480,13 +480,6 @@ __global__ void __launch_bounds__(512, 1)
           }
           const BwdTiles tt = bwd_tiles(p, bh);
           ok = mbar_wait_spin(bar_kv, (uint32_t)w & 1u, ab, lim, WAIT_BWD_MMA + 1);
-          if (PERSIST && ok && w > 0) {
-            // This item's first dV and dK MMAs overwrite the accumulators the previous item's
-            // epilogue reads; it reads them out right after its accumulator barrier, well within
-            // the K/V load just waited for. Waiting here keeps the per-tile loop free of checks.
-            ok = mbar_wait_spin(bar_dvfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 11);
-            if (ok) ok = mbar_wait_spin(bar_dkfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 12);
-          }
           if (!ok) break;
           int i = i_begin;
           while (i < tt.nb && !bwd_tile_active(tt, i, j)) ++i;
@@ -506,6 +499,13 @@ __global__ void __launch_bounds__(512, 1)
               issue_dp(it % NS_DO);
               umma_commit(bar_dp);
             }
+          }
+          if (PERSIST && ok && w > 0) {
+            // This item's first dV and dK MMAs overwrite the accumulators the previous item's
+            // epilogue reads out; its first S^T and dP^T above use other columns and may run
+            // meanwhile. Waiting here, once per item, keeps the per-tile loop free of checks.
+            ok = mbar_wait_spin(bar_dvfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 11);
+            if (ok) ok = mbar_wait_spin(bar_dkfree, (uint32_t)(w - 1) & 1u, ab, lim, WAIT_BWD_MMA + 12);
           }
           while (ok && i < tt.nb) {
             const int s = it % NS;
