@@ -97,12 +97,16 @@ struct BwdCfg {
   static constexpr int OFF_DEL = OFF_LSE + NS * 512;          // [NS][128] fp32: -D
   static constexpr int OFF_BAR = OFF_DEL + NS * 512;
   static constexpr int NQB = SPLIT ? RING : NS;               // full/empty barrier pairs of the Q ring
-  static constexpr int NBAR = 1 + 2 * NQB + 2 * NS_DO + 16;
+  static constexpr int NBAR = 1 + 2 * NQB + 2 * NS_DO + 18;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // TMEM address, abort flag, item ring [2]
   static constexpr int SMEM_BYTES = OFF_MISC + 32;
   static constexpr int TMEM_COLS = 512;
-  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + DH;
-  static constexpr bool DQ_ALIAS = (DH == 128);          // dQ reuses the dP^T columns
+  // SDB (d = 64): S^T/P^T double-buffered in [0,128) and [128,256) by the parity of the active
+  // query tile, so S^T_{i+1} is issued before the issuer waits for P^T_i; dQ then shares the dP^T
+  // columns as at d = 128 (measured +1-2 % on every d = 64 shape; d = 128 has no columns to spare).
+  static constexpr bool SDB = D == 64;
+  static constexpr uint32_t T_S = 0, T_DP = SDB ? 256 : 128, T_DV = SDB ? 384 : 256, T_DK = T_DV + DH;
+  static constexpr bool DQ_ALIAS = (DH == 128) || SDB;   // dQ reuses the dP^T columns
   static constexpr uint32_t T_DQ = DQ_ALIAS ? T_DP : 384u;
   // setmaxnreg split of the launch allocation (512 x 128, checked by the build script):
   // control warpgroup (TMA, MMA, 2 idle warps), two P/dS warpgroups, dQ-drain warpgroup.
@@ -221,6 +225,13 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* bar_vst = bar_dkfree + 1;    // the dV store has read its staging area (the dS buffer)
   uint64_t* bar_itf = bar_vst + 1;       // [2] persistent: item ring slot written by the producer
   uint64_t* bar_ite = bar_itf + 2;       // [2] persistent: item ring slot read by every other role
+  uint64_t* bar_s1 = bar_ite + 2;        // SDB: bar_s and bar_p of the odd active tiles (S^T buffer 1)
+  uint64_t* bar_p1 = bar_s1 + 1;
+  // S^T / P^T barrier of active tile number `n` and the parity of its phase
+  auto bar_s_of = [&](int n) { return (C::SDB && (n & 1)) ? bar_s1 : bar_s; };
+  auto bar_p_of = [&](int n) { return (C::SDB && (n & 1)) ? bar_p1 : bar_p; };
+  auto sp_par = [&](int n) -> uint32_t { return (uint32_t)(C::SDB ? (n >> 1) : n) & 1u; };
+  auto s_col = [&](int n) -> uint32_t { return C::SDB ? (uint32_t)(n & 1) * 128u : 0u; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   AbortState* ab = reinterpret_cast<AbortState*>(smem + C::OFF_MISC + 4);
   volatile int* item_ring = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);  // [2] {bh, item}; bh < 0: none
@@ -253,6 +264,8 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(bar_dvfree, 8);  // one arrive per P/dS warp
     mbar_init(bar_dkfree, 4);  // one arrive per dQ-drain warp
     mbar_init(bar_vst, 1);
+    mbar_init(bar_s1, 1);
+    mbar_init(bar_p1, 8);
     for (int r = 0; r < 2; ++r) {
       mbar_init(&bar_itf[r], 1);
       mbar_init(&bar_ite[r], 13);  // the MMA issuer, the eight P/dS warps, the four drain warps
@@ -446,12 +459,12 @@ __global__ void __launch_bounds__(512, 1)
       bool ok = true;
 
       if constexpr (!C::SPLIT) {
-        auto issue_s = [&](int st) {
+        auto issue_s = [&](int st, uint32_t dst) {
           const uint64_t b = dQ_k + (uint64_t)(st * TILE16);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off16 = ((kk >> 2) * C::PANEL_BYTES + (kk & 3) * 32) >> 4;
-            umma_ss(tS, dK_k + off16, b + off16, IDESC_S, kk > 0 ? 1u : 0u);
+            umma_ss(dst, dK_k + off16, b + off16, IDESC_S, kk > 0 ? 1u : 0u);
           }
         };
         auto issue_dp = [&](int st) {
@@ -488,8 +501,8 @@ __global__ void __launch_bounds__(512, 1)
             ok = mbar_wait_spin(&bar_qf[it % NS], (uint32_t)(it / NS) & 1u, ab, lim, WAIT_BWD_MMA + 2);
             if (ok) {
               tc_fence_after();
-              issue_s(it % NS);
-              umma_commit(bar_s);
+              issue_s(it % NS, tS + s_col(it));
+              umma_commit(bar_s_of(it));
               // d = 128: the dP^T columns hold the previous item's last dQ until it is drained
               if (C::DQ_ALIAS && it > 0) ok = mbar_wait_spin(bar_dqfree, (uint32_t)(it - 1) & 1u, ab, lim, WAIT_BWD_MMA + 7);
             }
@@ -517,21 +530,29 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t acc = ni > 0 ? 1u : 0u;
             const uint64_t dOs = dO_mn + (uint64_t)(sd * TILE16), dQs = dQ_mn + (uint64_t)(s * TILE16);
 
+            if (C::SDB && has_next) {
+              // S^T_{i+1} into the other buffer, whose P^T_{i-1} the previous dV has read already
+              ok = mbar_wait_spin(&bar_qf[sn], ((it + 1) / NS) & 1, ab, lim, WAIT_BWD_MMA + 4);
+              if (!ok) break;
+              tc_fence_after();
+              issue_s(sn, tS + s_col(it + 1));
+              umma_commit(bar_s_of(it + 1));
+            }
             // dV += P^T dO_i (reduction over the 128 queries of tile i), A = P^T from TMEM
-            ok = mbar_wait_spin(bar_p, it & 1, ab, lim, WAIT_BWD_MMA + 3);
+            ok = mbar_wait_spin(bar_p_of(it), sp_par(it), ab, lim, WAIT_BWD_MMA + 3);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              umma_ts(tDV, tS + (kk >> 2) * 64 + (kk & 3) * 8, dOs + (uint64_t)(kk * (2048 >> 4)), IDESC_KV,
-                      kk > 0 ? 1u : acc);
+              umma_ts(tDV, tS + s_col(it) + (kk >> 2) * 64 + (kk & 3) * 8, dOs + (uint64_t)(kk * (2048 >> 4)),
+                      IDESC_KV, kk > 0 ? 1u : acc);
             umma_commit(&bar_doe[sd]);  // dO_i read by dP_i and dV_i
             // S^T_{i+1} over P^T_i (the dV MMAs above read it first: tcgen05.mma runs in order)
-            if (has_next) {
+            if (!C::SDB && has_next) {
               ok = mbar_wait_spin(&bar_qf[sn], ((it + 1) / NS) & 1, ab, lim, WAIT_BWD_MMA + 4);
               if (!ok) break;
               tc_fence_after();
-              issue_s(sn);
+              issue_s(sn, tS);
               umma_commit(bar_s);
             }
             ok = mbar_wait_spin(bar_ds, it & 1, ab, lim, WAIT_BWD_MMA + 5);
@@ -749,15 +770,15 @@ __global__ void __launch_bounds__(512, 1)
         const int qlim = kpad ? 64 : (diag ? qmin - 64 * h : -1);
 
         // ---- P phase: P^T = exp2(S^T * scale*log2e - LSE*log2e), back into TMEM as bf16
-        ok = warp_wait(bar_s, it & 1, ab, lim, WAIT_BWD_COMPUTE + 1);
+        ok = warp_wait(bar_s_of(it), sp_par(it), ab, lim, WAIT_BWD_COMPUTE + 1);
         if (!ok) break;
         tc_fence_after();
         float pf[64];  // P in fp32, kept for the dS phase
         {
           uint32_t sa[32], sb[32];
-          tmem_ld32_async(tS_row, sa);
+          tmem_ld32_async(tS_row + s_col(it), sa);
           tmem_wait_ld_tied(sa);
-          tmem_ld32_async(tS_row + 32, sb);  // in flight while chunk 0 is processed
+          tmem_ld32_async(tS_row + s_col(it) + 32, sb);  // in flight while chunk 0 is processed
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             uint32_t (&su)[32] = c == 0 ? sa : sb;
@@ -802,13 +823,13 @@ __global__ void __launch_bounds__(512, 1)
               pk[e] = pack16<F16>(p0, p1);
               pk[e + 1] = pack16<F16>(p2, p3);
             }
-            tmem_st16(tS_row + c * 16, pk);  // columns [64h + 16c, +16): scores already read
+            tmem_st16(tS_row + s_col(it) + c * 16, pk);  // columns [64h + 16c, +16): scores already read
           }
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_p);
+        if (lane == 0) mbar_arrive(bar_p_of(it));
 
         // ---- dS phase: dS^T = P^T o (dP^T - D) into shared-memory panel h
         ok = warp_wait(bar_dp, it & 1, ab, lim, WAIT_BWD_COMPUTE + 2);
