@@ -73,10 +73,16 @@ def reduce_max(value: float, dist_on: bool, device=None) -> float:
 
 
 def kernel_source_hash() -> str:
+    """Hash of the backward kernel's code (its source and the PTX wrappers) with comments and
+    whitespace removed, so that a comment edit does not retire a traffic record."""
     import hashlib
+    import re
     m = hashlib.sha256()
     for f in ("exact_attention_110_b200/csrc/fa_bwd.cu", "exact_attention_110_b200/csrc/ptx.cuh"):
-        m.update((ROOT / f).read_bytes())
+        text = (ROOT / f).read_text()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)  # block comments
+        text = re.sub(r"//[^\n]*", " ", text)                 # line comments
+        m.update(" ".join(text.split()).encode())
     return m.hexdigest()[:16]
 
 

@@ -36,16 +36,18 @@
 //    write dV.
 //  * MMA order per query tile i: dV_i as soon as P_i is in TMEM; S_{i+1} (the compute warps
 //    start the next P phase while the tensor core still works on tile i); dQ_i; dK_i (covers
-//    the dQ drain); dP_{i+1}.
-//  * TMEM: S^T/P^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D); dQ: d = 128
-//    reuses the dP^T columns once dP^T has been read, d = 64 has its own [384,448).
+//    the dQ drain); dP_{i+1}. d = 64 issues S_{i+1} first, into the other S^T buffer.
+//  * TMEM, d = 128: S^T/P^T [0,128), dP^T [128,256), dV [256,384), dK [384,512). d = 64: S^T/P^T
+//    double-buffered [0,128) and [128,256) by the parity of the active tile, dP^T [256,384),
+//    dV [384,448), dK [448,512). dQ reuses the dP^T columns once dP^T has been read.
 //  * PERSIST (d <= 128): one CTA per SM walks several (b, h, key tile) items, its block index
 //    first and then numbers taken from a counter in the workspace (bwd_item, work_item), which
 //    the producer passes to the other roles through a two-slot ring in shared memory. Ring
 //    counters and barrier phases run on across items, the next item's loads overlap the
 //    previous item's epilogue, and three more barriers (dV / dK read out of TMEM, dV store done
 //    reading its staging buffer) keep the next item's first dV / dK MMAs and dS writes behind it;
-//    they are waited at the item's start, so the per-tile loops carry no per-item checks.
+//    they are waited once per item (the issuer after the item's first S^T and dP^T), so the
+//    per-tile loops carry no per-item checks.
 #include "kernels.h"
 #include "ptx.cuh"
 
