@@ -46,10 +46,12 @@ def test_back_to_back_launches_on_one_workspace(fa, oracle_mod, causal):
         H.assert_grads_close([H.to_f64(x)[sl] for x in (dq, dk, dv)], g_ref, f"head {b},{h}")
 
 
-def test_block_mask_that_empties_a_key_tile(fa, oracle_mod):
+@pytest.mark.parametrize("d", [64, 128])
+def test_block_mask_that_empties_a_key_tile(fa, oracle_mod, d):
     # Key tile 2 is off for every query tile: its items have no query tile to walk, and their
-    # dK and dV must come out as exact zeros while the persistent CTAs carry on to later items.
-    B, Hh, N, d = 2, 80, 512, 128
+    # dK and dV must come out as exact zeros while the persistent CTAs carry on to later items
+    # (at d = 64 the S^T buffers alternate by active tile, which such items do not advance).
+    B, Hh, N = 2, 80, 512
     nb = N // 128
     mask = np.ones((nb, nb), np.uint8)
     mask[:, 2] = 0
