@@ -33,3 +33,27 @@ def test_warmup_below_three_is_refused():
     out = subprocess.run([sys.executable, str(ROOT / "bench.py"), "--warmup", "2"], capture_output=True, text=True,
                          cwd=ROOT, timeout=120)
     assert out.returncode != 0 and "warmup" in out.stderr
+
+
+def test_traffic_record_matches_the_current_backward_code(tmp_path, monkeypatch):
+    # The roofline's DRAM traffic comes from profiles/traffic.json, keyed to a hash of the
+    # backward's code without comments: the committed record must match the committed code,
+    # a comment edit must keep the key, and a code edit must retire it.
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", ROOT / "bench.py")
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    key = "bwd_main N=4096 d=128 causal=0 bs=0"
+    assert bench.recorded_traffic(key) is not None
+    h0 = bench.kernel_source_hash()
+    src = tmp_path / "exact_attention_110_b200" / "csrc"
+    src.mkdir(parents=True)
+    for f in ("fa_bwd.cu", "ptx.cuh"):
+        (src / f).write_text((ROOT / "exact_attention_110_b200" / "csrc" / f).read_text())
+    monkeypatch.setattr(bench, "ROOT", tmp_path)
+    assert bench.kernel_source_hash() == h0
+    bwd = src / "fa_bwd.cu"
+    bwd.write_text(bwd.read_text() + "\n// a comment\n/* and a block\n comment */\n")
+    assert bench.kernel_source_hash() == h0
+    bwd.write_text(bwd.read_text() + "\nstatic int fa_unused_probe = 1;\n")
+    assert bench.kernel_source_hash() != h0
